@@ -1,0 +1,260 @@
+"""fp64 CPU oracle for jagged HSTU pointwise attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+may import this package.  The CUDA library never calls it and shares no code
+with it.  The arithmetic lives in ``hstu_oracle.c`` (plain C, double
+precision, OpenMP over rows); this module only compiles it with gcc, converts
+arrays and calls it through ctypes.
+
+Parity pins (what ties each function to the pages rather than to itself) are
+in ``tests/test_oracle_pins.py``; every function here is pinned.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hstu_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "libhstu_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+MASK_CAUSAL = 0
+MASK_MTGR = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (double precision, no fast-math, no FMA contraction)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = C.CDLL(build())
+            _declare(_lib)
+    return _lib
+
+
+_p = C.c_void_p
+_i32 = C.c_int32
+_i64 = C.c_int64
+_f64 = C.c_double
+
+
+def _declare(L):
+    L.hstu_oracle_indices.argtypes = [_i32, _p, _p, _i32, _p, _p, _i32, _i32, _p, _p, _p, _p]
+    L.hstu_oracle_attn_fwd.argtypes = [_i32, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _i32, _p,
+                                       _i32, _i32, _p, _p, _f64, _i64, _p, _p]
+    L.hstu_oracle_ln_mul_fwd.argtypes = [_i64, _i32, _p, _p, _p, _p, _f64, _p, _p, _p]
+    L.hstu_oracle_ln_mul_bwd.argtypes = [_i64, _i32, _p, _p, _p, _p, _f64, _p, _p, _p, _p, _p]
+    L.hstu_oracle_attn_bwd.argtypes = [_i32, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _i32, _p,
+                                       _i32, _i32, _p, _p, _f64, _p, _p, _p, _p, _p, _p]
+    L.hstu_oracle_mfalcon.argtypes = [_i32, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p,
+                                      _p, _i32, _p, _i32, _f64, _i64, _p, _p]
+    L.hstu_oracle_num_threads.restype = C.c_int
+    L.hstu_oracle_set_num_threads.argtypes = [C.c_int]
+
+
+def num_threads() -> int:
+    return int(lib().hstu_oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    lib().hstu_oracle_set_num_threads(int(n))
+
+
+# ----------------------------------------------------------------------------
+# array helpers
+# ----------------------------------------------------------------------------
+
+def f32(x) -> np.ndarray:
+    """Exact float32 copy of a bf16/fp32 torch tensor or numpy array."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float32).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _c(x, dtype):
+    return np.ascontiguousarray(np.asarray(x, dtype=dtype))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _kind(w) -> int:
+    return MASK_MTGR if w.kind == "mtgr" else MASK_CAUSAL
+
+
+def _segs(w):
+    if w.kind == "mtgr":
+        return _c(w.n_static, np.int32), _c(w.n_realtime, np.int32)
+    return None, None
+
+
+# ----------------------------------------------------------------------------
+# public functions (all return float64 numpy arrays)
+# ----------------------------------------------------------------------------
+
+def pair_offsets(offsets) -> np.ndarray:
+    L = np.diff(np.asarray(offsets, dtype=np.int64))
+    po = np.zeros(len(L) + 1, dtype=np.int64)
+    po[1:] = np.cumsum(L * L)
+    return po
+
+
+def indices(offsets, ts, kind: int, n_static=None, n_rt=None, P: int = 256, nb: int = 64):
+    """Per-pair (mask, pos index, time bucket) for every (b, i, j), flattened by pair_offsets."""
+    off = _c(offsets, np.int32)
+    tsa = _c(ts, np.int64)
+    po = pair_offsets(off)
+    n = int(po[-1])
+    m = np.zeros(n, np.uint8)
+    pi = np.zeros(n, np.int16)
+    tb = np.zeros(n, np.int8)
+    ns = None if n_static is None else _c(n_static, np.int32)
+    nr = None if n_rt is None else _c(n_rt, np.int32)
+    lib().hstu_oracle_indices(len(off) - 1, _ptr(off), _ptr(tsa), kind, _ptr(ns), _ptr(nr), P, nb,
+                              _ptr(po), _ptr(m), _ptr(pi), _ptr(tb))
+    return m, pi, tb, po
+
+
+def attn_fwd_raw(offsets, H, dqk, dv, q, k, v, ts, rab_pos, rab_time, kind, n_static, n_rt, alpha,
+                 rows=None, P=256, nb=64):
+    off = _c(offsets, np.int32)
+    q, k, v = f32(q), f32(k), f32(v)
+    tsa = _c(ts, np.int64)
+    rp, rt = f32(rab_pos), f32(rab_time)
+    ns = None if n_static is None else _c(n_static, np.int32)
+    nr = None if n_rt is None else _c(n_rt, np.int32)
+    r = None if rows is None else _c(rows, np.int64)
+    n = int(off[-1]) if r is None else len(r)
+    y = np.zeros((n, H * dv), np.float64)
+    lib().hstu_oracle_attn_fwd(len(off) - 1, _ptr(off), H, dqk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(tsa),
+                               _ptr(rp), P, _ptr(rt), nb, kind, _ptr(ns), _ptr(nr), float(alpha),
+                               0 if r is None else len(r), _ptr(r), _ptr(y))
+    return y
+
+
+def attn_fwd(w, rows=None, q=None, k=None, v=None):
+    """Y = (sum_j mask * SiLU(q.k + rab) v_j) / alpha for the listed token rows (all by default)."""
+    ns, nr = _segs(w)
+    return attn_fwd_raw(w.offsets, w.H, w.d, w.d, w.q if q is None else q, w.k if k is None else k,
+                        w.v if v is None else v, w.ts, w.rab_pos, w.rab_time, _kind(w), ns, nr,
+                        w.alpha, rows, w.n_pos, w.n_tbuckets)
+
+
+def ln_mul_fwd(y, u, gamma, beta, eps=1e-5):
+    """o = LayerNorm(y) * gamma + beta, times u; returns (o, mean, rstd)."""
+    y = _c(y, np.float64)
+    n, D = y.shape
+    u, g, b = f32(u), f32(gamma), f32(beta)
+    o = np.zeros((n, D), np.float64)
+    mu = np.zeros(n, np.float64)
+    rs = np.zeros(n, np.float64)
+    lib().hstu_oracle_ln_mul_fwd(n, D, _ptr(y), _ptr(u), _ptr(g), _ptr(b), float(eps), _ptr(o),
+                                 _ptr(mu), _ptr(rs))
+    return o, mu, rs
+
+
+def ln_mul_bwd(y, u, gamma, beta, grad, eps=1e-5):
+    """Returns (dy, du, dgamma, dbeta) for g = dL/d o."""
+    y = _c(y, np.float64)
+    n, D = y.shape
+    u, g, b, gr = f32(u), f32(gamma), f32(beta), f32(grad)
+    dy = np.zeros((n, D), np.float64)
+    du = np.zeros((n, D), np.float64)
+    dg = np.zeros(D, np.float64)
+    db = np.zeros(D, np.float64)
+    lib().hstu_oracle_ln_mul_bwd(n, D, _ptr(y), _ptr(u), _ptr(g), _ptr(b), float(eps), _ptr(gr),
+                                 _ptr(dy), _ptr(du), _ptr(dg), _ptr(db))
+    return dy, du, dg, db
+
+
+def attn_bwd_raw(offsets, H, dqk, dv, q, k, v, ts, rab_pos, rab_time, kind, n_static, n_rt, alpha, dy,
+                 P=256, nb=64):
+    off = _c(offsets, np.int32)
+    q, k, v = f32(q), f32(k), f32(v)
+    tsa = _c(ts, np.int64)
+    rp, rt = f32(rab_pos), f32(rab_time)
+    ns = None if n_static is None else _c(n_static, np.int32)
+    nr = None if n_rt is None else _c(n_rt, np.int32)
+    dy = _c(dy, np.float64)
+    T = int(off[-1])
+    dq = np.zeros((T, H * dqk), np.float64)
+    dk = np.zeros((T, H * dqk), np.float64)
+    dvv = np.zeros((T, H * dv), np.float64)
+    drp = np.zeros(2 * P - 1, np.float64)
+    drt = np.zeros(nb, np.float64)
+    lib().hstu_oracle_attn_bwd(len(off) - 1, _ptr(off), H, dqk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(tsa),
+                               _ptr(rp), P, _ptr(rt), nb, kind, _ptr(ns), _ptr(nr), float(alpha), _ptr(dy),
+                               _ptr(dq), _ptr(dk), _ptr(dvv), _ptr(drp), _ptr(drt))
+    return dq, dk, dvv, drp, drt
+
+
+def attn_bwd(w, dy):
+    ns, nr = _segs(w)
+    return attn_bwd_raw(w.offsets, w.H, w.d, w.d, w.q, w.k, w.v, w.ts, w.rab_pos, w.rab_time, _kind(w),
+                        ns, nr, w.alpha, dy, w.n_pos, w.n_tbuckets)
+
+
+def mfalcon(w, rows=None):
+    """Per-candidate Y over cached history plus the candidate itself (rows = candidate indices)."""
+    ho, co = _c(w.hist_offsets, np.int32), _c(w.cand_offsets, np.int32)
+    hk, hv = f32(w.hist_k), f32(w.hist_v)
+    cq, ck, cv = f32(w.cand_q), f32(w.cand_k), f32(w.cand_v)
+    hts, cts = _c(w.hist_ts, np.int64), _c(w.cand_ts, np.int64)
+    rp, rt = f32(w.rab_pos), f32(w.rab_time)
+    r = None if rows is None else _c(rows, np.int64)
+    n = int(co[-1]) if r is None else len(r)
+    y = np.zeros((n, w.H * w.d), np.float64)
+    lib().hstu_oracle_mfalcon(len(co) - 1, _ptr(ho), _ptr(co), w.H, w.d, w.d, _ptr(hk), _ptr(hv), _ptr(hts),
+                              _ptr(cq), _ptr(ck), _ptr(cv), _ptr(cts), _ptr(rp), w.n_pos, _ptr(rt),
+                              w.n_tbuckets, float(w.alpha), 0 if r is None else len(r), _ptr(r), _ptr(y))
+    return y
+
+
+# ----------------------------------------------------------------------------
+# whole-layer conveniences
+# ----------------------------------------------------------------------------
+
+def layer_fwd(w, rows=None):
+    """(y, o_pre, mean, rstd) for the listed rows: attention, then LayerNorm(y) * u."""
+    y = attn_fwd(w, rows)
+    u = f32(w.u) if rows is None else f32(w.u)[np.asarray(rows)]
+    o, mu, rs = ln_mul_fwd(y, u, w.gamma, w.beta, w.eps)
+    return y, o, mu, rs
+
+
+def layer_bwd(w):
+    """Full backward of o_pre = LN(attn(q,k,v)) * u for the upstream gradient w.grad."""
+    y = attn_fwd(w)
+    dy, du, dg, db = ln_mul_bwd(y, w.u, w.gamma, w.beta, w.grad, w.eps)
+    dq, dk, dv, drp, drt = attn_bwd(w, dy)
+    return dict(y=y, dy=dy, du=du, dgamma=dg, dbeta=db, dq=dq, dk=dk, dv=dv, d_rab_pos=drp, d_rab_time=drt)
+
+
+def mfalcon_layer(w, rows=None):
+    y = mfalcon(w, rows)
+    u = f32(w.cand_u) if rows is None else f32(w.cand_u)[np.asarray(rows)]
+    o, _, _ = ln_mul_fwd(y, u, w.gamma, w.beta, w.eps)
+    return y, o
