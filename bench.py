@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of jagged HSTU pointwise attention on B200.
+
+One step = one training pass of one HSTU attention layer over the large jagged
+workload (lognormal lengths, 256k tokens, d_model 1024 = 8 x 128, causal +
+rab): forward (attention + LayerNorm(Y)*U) and full backward.  The metric is
+useful TFLOP/s: 4*d per visible (i, j) pair and head for the forward, 8*d for
+the backward (recomputation not counted).  M-FALCON candidates/s are measured
+on the ranking workload (256 users x 2048 cached history, 1024 candidates,
+b_m = 256) in the same run.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch (weak scaling); the only
+collective is the all-reduce of the rab / LayerNorm parameter gradients.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hstu_jagged_pointwise_b200 import workloads as W  # noqa: E402
+
+METRIC = "jagged HSTU attn useful TFLOP/s fwd & fwd+bwd (% bf16 peak); M-FALCON cands/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+# ----------------------------------------------------------------------------
+# workload accounting
+# ----------------------------------------------------------------------------
+
+def causal_pairs(lengths) -> int:
+    L = np.asarray(lengths, dtype=np.int64)
+    return int((L * (L + 1) // 2).sum())
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def alu_fp32_peak_tflops(sm_mhz: float) -> float:
+    # 148 SMs x 128 FP32 lanes x 2 FLOP (FFMA) per clock
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_init(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline (the fp64 oracle, as it stands)
+# ----------------------------------------------------------------------------
+
+def sub_workload(w, seqs):
+    lens = [int(w.offsets[b + 1] - w.offsets[b]) for b in seqs]
+    rows = np.concatenate([np.arange(w.offsets[b], w.offsets[b + 1]) for b in seqs])
+    ts_list = [w.ts[w.offsets[b]:w.offsets[b + 1]] for b in seqs]
+    s = W.make_causal(lens, H=w.H, d=w.d, dtype=w.dtype, seed=0, alpha=w.alpha, ts_list=ts_list,
+                      with_grad=True)
+    rt = torch.as_tensor(rows)
+    for name in ("q", "k", "v", "u", "grad"):
+        setattr(s, name, getattr(w, name)[rt])
+    s.rab_pos, s.rab_time, s.gamma, s.beta = w.rab_pos, w.rab_time, w.gamma, w.beta
+    return s
+
+
+def oracle_sample(w, target_s: float = 12.0):
+    """Bounded sample of the workload for the oracle: whole sequences (shortest first)
+    whose estimated oracle time is about target_s seconds."""
+    import oracle
+    L = w.lengths
+    order = np.argsort(L)
+    # calibrate on the shortest sequence
+    cal = sub_workload(w, [int(order[0])])
+    t0 = time.perf_counter()
+    oracle.layer_bwd(cal)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    rate = 12 * w.d * w.H * causal_pairs([L[order[0]]]) / dt
+    seqs, flops = [], 0.0
+    for b in order[1:]:
+        f = 12 * w.d * w.H * causal_pairs([L[b]])
+        if seqs and (flops + f) / rate > target_s:
+            break
+        seqs.append(int(b))
+        flops += f
+    return sub_workload(w, seqs), seqs
+
+
+def time_oracle(sample):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.layer_bwd(sample)
+    dt = time.perf_counter() - t0
+    useful = 12 * sample.d * sample.H * causal_pairs(sample.lengths)
+    return useful / dt / 1e12, dt, oracle.num_threads()
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    from hstu_jagged_pointwise_b200 import capi, ops
+
+    w = W.large_layer(seed=args.seed + rank)
+    dev = torch.device("cuda", local)
+    H, d = w.H, w.d
+    P_head = causal_pairs(w.lengths)
+    P = P_head * H
+    f_fwd, f_bwd = 4 * d * P, 8 * d * P
+    host = {n: getattr(w, n).contiguous() for n in ("q", "k", "v", "u", "grad")}
+    dv = {n: t.to(dev) for n, t in host.items()}
+    off = torch.as_tensor(w.offsets).to(dev)
+    ts = torch.as_tensor(w.ts).to(dev)
+    rp, rt, g, b = (t.to(dev) for t in (w.rab_pos, w.rab_time, w.gamma, w.beta))
+    layer = ops.Layer(off, ts, H, d, torch.bfloat16, w.alpha, w.max_len)
+    fwd_out = dict(y=torch.empty_like(dv["q"]), o_pre=torch.empty_like(dv["q"]),
+                   mean=torch.empty(w.T, dtype=torch.float32, device=dev),
+                   rstd=torch.empty(w.T, dtype=torch.float32, device=dev))
+    bwd_out = dict(dq=torch.empty_like(dv["q"]), dk=torch.empty_like(dv["k"]), dv=torch.empty_like(dv["v"]),
+                   du=torch.empty_like(dv["u"]), d_rab_pos=torch.empty_like(rp), d_rab_time=torch.empty_like(rt),
+                   d_gamma=torch.empty_like(g), d_beta=torch.empty_like(b))
+    small = None
+    if world > 1:
+        import torch.distributed as dist
+        small = torch.empty(rp.numel() + rt.numel() + 2 * g.numel(), dtype=torch.float32, device=dev)
+
+    def step():
+        layer.forward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, out=fwd_out)
+        layer.backward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, fwd_out, dv["grad"], out=bwd_out)
+        if world > 1:
+            torch.cat([bwd_out["d_rab_pos"], bwd_out["d_rab_time"], bwd_out["d_gamma"], bwd_out["d_beta"]],
+                      out=small)
+            dist.all_reduce(small)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = layer.check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device status {capi.status_string(st)} after warm-up")
+
+    # ---- device-timed region
+    sampler = ClockSampler(local)
+    capi.profile_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    kernels = capi.profile_read()
+    capi.profile_enable(False)
+    ms_max = max_over_ranks(ms, world)
+    if layer.check_device_error() != 0:
+        raise RuntimeError("device status set during the timed region")
+
+    # forward alone (same stream, same inputs)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, out=fwd_out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_fwd = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+
+    # ---- end to end through the C ABI with host buffers
+    pin = {n: t.pin_memory() for n, t in host.items()}
+    small_in = {n: t.pin_memory() for n, t in (("rp", w.rab_pos), ("rt", w.rab_time), ("g", w.gamma),
+                                                ("b", w.beta))}
+    off_h = torch.as_tensor(w.offsets).pin_memory()
+    ts_h = torch.as_tensor(w.ts).pin_memory()
+    outs_h = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in
+              list(bwd_out.items()) + [("o_pre", fwd_out["o_pre"])]}
+    h2d = sum(t.numel() * t.element_size() for t in list(pin.values()) + list(small_in.values()) + [off_h, ts_h])
+    d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
+
+    def e2e_step():
+        for n, t in pin.items():
+            dv[n].copy_(t, non_blocking=True)
+        rp.copy_(small_in["rp"], non_blocking=True)
+        rt.copy_(small_in["rt"], non_blocking=True)
+        g.copy_(small_in["g"], non_blocking=True)
+        b.copy_(small_in["b"], non_blocking=True)
+        off.copy_(off_h, non_blocking=True)
+        ts.copy_(ts_h, non_blocking=True)
+        step()
+        for n, t in outs_h.items():
+            src = fwd_out["o_pre"] if n == "o_pre" else bwd_out[n]
+            t.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(1, min(args.steps, 3))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+
+    # ---- M-FALCON candidates / s
+    mf = None
+    if not args.no_mfalcon:
+        del pin, outs_h
+        mf = run_mfalcon(args, world, rank, local)
+
+    # ---- roofline of the dominant kernel
+    pk, pk_src = peaks()
+    sm_mhz = pk.get("sm_max_mhz", 1965.0)
+    kinfo = {}
+    algo = {
+        "attn_fwd_tc_kernel": ("tensor", f_fwd, "TFLOP/s"),
+        "attn_bwd_dkv_simt_kernel": ("alu", 6 * d * P, "TFLOP/s"),
+        "attn_bwd_dq_simt_kernel": ("alu", 2 * d * P, "TFLOP/s"),
+        "attn_bwd_tc_kernel": ("tensor", f_bwd, "TFLOP/s"),
+        "ln_fwd_kernel": ("hbm", (6 * w.D + 8) * w.T, "GB/s"),
+        "ln_bwd_kernel": ("hbm", (10 * w.D + 8) * w.T, "GB/s"),
+    }
+    launches_total = 0
+    for name, (n, tot) in kernels.items():
+        per_step = n / args.steps
+        launches_total += n
+        avg = tot / n
+        e = {"launches_per_step": per_step, "ms_per_launch": round(avg, 4),
+             "share": round(tot / max(ms * args.steps, 1e-9), 4)}
+        if name in algo:
+            bound, units, unit = algo[name]
+            if unit == "TFLOP/s":
+                ach = units / (avg * 1e-3) / 1e12
+                peak = pk["bf16_tflops_sustained"] if bound == "tensor" else alu_fp32_peak_tflops(sm_mhz)
+            else:
+                ach = units / (avg * 1e-3) / 1e9
+                peak = pk["hbm_gbs"]
+            e.update(bound=bound, achieved=round(ach, 2), peak=round(peak, 1), unit=unit,
+                     frac=round(ach / peak, 4))
+        kinfo[name] = e
+    dominant = max(kernels.items(), key=lambda kv: kv[1][1])[0]
+    dk = kinfo[dominant]
+    roof = {"kernel": dominant, "bound": dk.get("bound"), "achieved": dk.get("achieved"),
+            "peak": dk.get("peak"), "unit": dk.get("unit"), "frac": dk.get("frac"), "traffic": None,
+            "peak_source": f"{pk_src} ({'bf16_tflops_sustained' if dk.get('bound') == 'tensor' else ('hbm_gbs' if dk.get('bound') == 'hbm' else 'FP32 FFMA from unit counts x sm_max_mhz')})"}
+
+    flops_step = f_fwd + f_bwd
+    value = world * flops_step / (ms_max * 1e-3) / 1e12
+    fwd_tflops = world * f_fwd / (ms_fwd * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded lognormal lengths, N(0,1) activations, N(0,0.02) rab tables)",
+        "config": {"workload": w.name, "global_batch_tokens": w.T * world, "sequences_per_gpu": w.B,
+                   "max_seq_len": w.max_len, "H": H, "d": d, "mask": "causal+rab_pos+rab_time",
+                   "parallelism": f"dp{world}", "l2": "inputs larger than L2 (512 MiB per tensor)"},
+        "pct_bf16_peak_fwd_bwd": round(value / world / pk["bf16_tflops_sustained"], 4),
+        "fwd_tflops": round(fwd_tflops, 3),
+        "pct_bf16_peak_fwd": round(fwd_tflops / world / pk["bf16_tflops_sustained"], 4),
+        "peak_source": pk_src,
+        "e2e": {"value": round(world * flops_step / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches_total),
+        "roofline": roof,
+        "kernels": kinfo,
+        "clocks": clocks,
+    }
+    if mf is not None:
+        line["mfalcon"] = mf
+    return line, w
+
+
+def run_mfalcon(args, world, rank, local):
+    from hstu_jagged_pointwise_b200 import ops
+    w = W.mfalcon_ranking(seed=args.seed + rank)
+    dev = torch.device("cuda", local)
+    d = {n: getattr(w, n).to(dev) for n in ("hist_k", "hist_v", "cand_q", "cand_k", "cand_v", "cand_u")}
+    small = {n: getattr(w, n).to(dev) for n in ("rab_pos", "rab_time", "gamma", "beta")}
+    ho = torch.as_tensor(w.hist_offsets).to(dev)
+    co = torch.as_tensor(w.cand_offsets).to(dev)
+    hts = torch.as_tensor(w.hist_ts).to(dev)
+    cts = torch.as_tensor(w.cand_ts).to(dev)
+    m = ops.MFalcon(ho, hts, co, cts, w.H, w.d, w.alpha, w.b_m, int(np.diff(w.hist_offsets).max()),
+                    int(np.diff(w.cand_offsets).max()))
+    out = dict(y=torch.empty_like(d["cand_q"]), o_pre=torch.empty_like(d["cand_q"]))
+
+    def go():
+        m.score(d["hist_k"], d["hist_v"], d["cand_q"], d["cand_k"], d["cand_v"], d["cand_u"], small["rab_pos"],
+                small["rab_time"], small["gamma"], small["beta"], out=out)
+
+    for _ in range(args.warmup):
+        go()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        go()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    if m.check_device_error() != 0:
+        raise RuntimeError("device status set in M-FALCON")
+    n_c = w.T
+    pairs = int(w.H * np.sum(np.diff(w.cand_offsets) * (np.diff(w.hist_offsets) + 1)))
+    pk, _ = peaks()
+    tfl = 4 * w.d * pairs / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "cands_per_s": round(world * n_c / (ms * 1e-3), 1), "ms_per_pass": round(ms, 4),
+            "tflops": round(world * tfl, 3), "pct_bf16_peak": round(tfl / pk["bf16_tflops_sustained"], 4),
+            "b_m": w.b_m}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = W.large_layer(seed=args.seed)
+    sample, seqs = oracle_sample(w, target_s=max(5.0, 60.0 / max(args.steps + args.warmup, 1)))
+    for _ in range(args.warmup):
+        time_oracle(sample)
+    vals, secs = [], []
+    threads = 1
+    for _ in range(args.steps):
+        v, dt, threads = time_oracle(sample)
+        vals.append(v)
+        secs.append(dt)
+    value = statistics.median(vals)
+    desc = (f"{len(seqs)} whole sequences ({int(sample.T)} tokens, shortest first) of {w.name}; "
+            f"forward + LayerNorm + full backward in fp64")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.median(secs), 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "sample": desc},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-mfalcon", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world, rank, local = dist_init(args.gpus) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    line, w = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample, seqs = oracle_sample(w)
+        v, dt, threads = time_oracle(sample)
+        line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{len(seqs)} whole sequences ({int(sample.T)} tokens, shortest first) "
+                                          f"of {w.name}, fwd+LN+bwd in fp64, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,565 @@
+// attn_fwd_tc.cu -- fused jagged HSTU pointwise attention forward on tcgen05 (sm_100a).
+//
+// Computes, per (sequence, head, 128-row query tile),
+//     Y = (1/alpha) * sum_over_key_tiles  [mask (.) SiLU(Q K^T + rab_pos + rab_time)] V
+// (Meta HSTU blog, section 3 formula and 3.1 pointwise attention; section 3.2
+// relative attention bias; MTGR pages for the dynamic mixed mask; HSTU blog
+// sections 4.2-4.3 for the M-FALCON candidate mask, whose self term is added
+// in the epilogue).  There is no softmax, so no running maximum and no
+// rescaling: P = SiLU(Z) is written once per tile and accumulated.
+//
+// One CTA = 6 warps, two CTAs per SM (each owns 256 TMEM columns and ~108 KB
+// of shared memory, so one CTA's elementwise phase overlaps the other's MMAs):
+//   warps 0-3  elementwise: TMEM S -> bias, mask, SiLU -> bf16 P back into TMEM;
+//              epilogue O/alpha -> global (and the M-FALCON self term)
+//   warp 4     producer: dynamic work fetch + TMA loads of Q, K, V tiles
+//   warp 5     MMA issuer: S = Q K^T (SS), O += P V (TS, P from TMEM)
+// TMEM columns: S/P at [0, 128), O at [128, 128 + D).
+// Every wait is bounded; on timeout the CTA records a status bit, drains its
+// copies and MMAs, frees TMEM and exits.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hstu {
+namespace {
+
+using namespace ptx;
+
+template <int D>
+struct FwdSmem {
+    static constexpr uint32_t kTileBytes = 128u * D * 2u;
+    static constexpr uint32_t q = 0;
+    static constexpr uint32_t k = q + kTileBytes;
+    static constexpr uint32_t v = k + kTileBytes;
+    static constexpr uint32_t rp = v + kTileBytes;              // float[2*kMaxPos]
+    static constexpr uint32_t rt = rp + 2u * kMaxPos * 4u;      // float[64]
+    static constexpr uint32_t cts = rt + kMaxTBuckets * 4u;     // int64[4 warps][128]
+    static constexpr uint32_t item = cts + 4u * 128u * 8u;      // int4[2]
+    static constexpr uint32_t bars = item + 2u * 16u;           // uint64[16]
+    static constexpr uint32_t tmem = bars + 16u * 8u;           // uint32
+    static constexpr uint32_t abort_flag = tmem + 4u;           // int
+    static constexpr uint32_t bytes = abort_flag + 4u;
+    static constexpr uint32_t alloc = bytes + 1024u;            // slack for 1024-B alignment
+};
+
+enum {
+    kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kOFull, kOEmpty,
+    kItFull0, kItFull1, kItEmpty0, kItEmpty1, kDrain, kNumBars
+};
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSCol = 0;
+constexpr uint32_t kOCol = 128;
+constexpr unsigned kFull = 0xffffffffu;
+
+struct Item {
+    int b, row0, h, row_end;   // query rows [row0, row_end) of sequence b, head h
+    int q0, Lq, kv0, Lk, S, R;
+};
+
+template <int KIND>
+__device__ __forceinline__ Item load_item(const FwdParams& p, int4 it) {
+    Item s;
+    s.b = it.x; s.row0 = it.y; s.h = it.z; s.row_end = it.w;
+    s.q0 = p.q_off[s.b];
+    s.Lq = p.q_off[s.b + 1] - s.q0;
+    s.kv0 = p.kv_off[s.b];
+    s.Lk = p.kv_off[s.b + 1] - s.kv0;
+    if (KIND == HSTU_KIND_MTGR) {
+        s.S = p.n_static[s.b];
+        s.R = p.n_rt[s.b];
+    } else {
+        s.S = s.Lq;
+        s.R = 0;
+    }
+    return s;
+}
+
+template <int KIND>
+__device__ __forceinline__ int kv_class(const Item& s, int t) {
+    const int ka = t * kTileN;
+    const int kb = min(ka + kTileN - 1, s.Lk - 1);
+    return tile_class(KIND, s.row0, s.row_end - 1, ka, kb, s.S, s.R);
+}
+
+template <int KIND>
+__device__ __forceinline__ int row_pos(const Item& s, int i) {
+    if (KIND == HSTU_KIND_MFALCON) return s.Lk;   // every candidate sits right after its history
+    return token_pos(KIND, i, s.S, s.R);
+}
+
+template <int KIND>
+__device__ __forceinline__ int col_pos(const Item& s, int j) {
+    if (KIND == HSTU_KIND_MFALCON) return j;
+    return token_pos(KIND, j, s.S, s.R);
+}
+
+__device__ __forceinline__ void flag_timeout(const FwdParams& p, volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicOr(&p.ctrl->status, kStatusTimeout);
+}
+
+// ------------------------------------------------------------------ kernel
+template <int KIND, int D>
+__global__ void __launch_bounds__(kThreads, 2)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using L = FwdSmem<D>;
+    constexpr int kPanels = D / 64;
+    constexpr uint32_t kPanelBytes = 128u * 128u;               // 128 rows x 128 B
+    constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, 0, 1);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    uint8_t* sQ = sm + L::q;
+    uint8_t* sK = sm + L::k;
+    uint8_t* sV = sm + L::v;
+    float* s_rp = reinterpret_cast<float*>(sm + L::rp);
+    float* s_rt = reinterpret_cast<float*>(sm + L::rt);
+    int64_t* s_cts = reinterpret_cast<int64_t*>(sm + L::cts);
+    int4* s_item = reinterpret_cast<int4*>(sm + L::item);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::tmem);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::abort_flag);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int i = tid; i < 2 * p.P - 1; i += kThreads) s_rp[i] = p.rab_pos[i];
+    for (int i = tid; i < p.nb; i += kThreads) s_rt[i] = p.rab_time[i];
+    if (tid == 0) {
+        mbar_init(&bars[kQFull], 1);
+        mbar_init(&bars[kQEmpty], 1);
+        mbar_init(&bars[kKFull], 1);
+        mbar_init(&bars[kKEmpty], 1);
+        mbar_init(&bars[kVFull], 1);
+        mbar_init(&bars[kVEmpty], 1);
+        mbar_init(&bars[kSFull], 1);
+        mbar_init(&bars[kPFull], 128);
+        mbar_init(&bars[kOFull], 1);
+        mbar_init(&bars[kOEmpty], 128);
+        mbar_init(&bars[kItFull0], 1);
+        mbar_init(&bars[kItFull1], 1);
+        mbar_init(&bars[kItEmpty0], 129);
+        mbar_init(&bars[kItEmpty1], 129);
+        mbar_init(&bars[kDrain], 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 5) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 4) {
+        // ============================================================ producer
+        int it_use = 0, q_use = 0, k_use = 0, v_use = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = it_use & 1;
+            if (lane == 0) {
+                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort);
+                if (ok) {
+                    const int idx = atomicAdd(&p.ctrl->counter, 1);
+                    const int4 it = idx < p.ctrl->n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
+                    s_item[slot] = it;
+                    mbar_arrive(&bars[kItFull0 + slot]);
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+            if (!ok) break;
+            int4 it = s_item[slot];                 // lane 0 wrote it; broadcast below
+            it.x = __shfl_sync(kFull, it.x, 0);
+            it.y = __shfl_sync(kFull, it.y, 0);
+            it.z = __shfl_sync(kFull, it.z, 0);
+            it.w = __shfl_sync(kFull, it.w, 0);
+            it_use++;
+            if (it.x < 0) break;
+            const Item s = load_item<KIND>(p, it);
+            if (lane == 0) {
+                ok = mbar_wait(&bars[kQEmpty], (q_use & 1) ^ 1, s_abort);
+                if (ok) {
+                    mbar_arrive_expect_tx(&bars[kQFull], L::kTileBytes);
+                    for (int pn = 0; pn < kPanels; pn++)
+                        tma_load_2d(sQ + pn * kPanelBytes, &tm_q, &bars[kQFull], s.h * D + pn * 64,
+                                    s.q0 + s.row0);
+                    q_use++;
+                }
+                const int n_kt = (s.Lk + kTileN - 1) / kTileN;
+                for (int t = 0; ok && t < n_kt; t++) {
+                    if (kv_class<KIND>(s, t) == 0) continue;
+                    const int y = s.kv0 + t * kTileN;
+                    ok = mbar_wait(&bars[kKEmpty], (k_use & 1) ^ 1, s_abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars[kKFull], L::kTileBytes);
+                    for (int pn = 0; pn < kPanels; pn++)
+                        tma_load_2d(sK + pn * kPanelBytes, &tm_k, &bars[kKFull], s.h * D + pn * 64, y);
+                    k_use++;
+                    ok = mbar_wait(&bars[kVEmpty], (v_use & 1) ^ 1, s_abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars[kVFull], L::kTileBytes);
+                    for (int pn = 0; pn < kPanels; pn++)
+                        tma_load_2d(sV + pn * kPanelBytes, &tm_v, &bars[kVFull], s.h * D + pn * 64, y);
+                    v_use++;
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+        }
+        if (lane == 0) {
+            if (!ok && !*s_abort) flag_timeout(p, s_abort);
+            if (*s_abort) {
+                // drain the copies this warp issued (at most the last one per buffer)
+                volatile int dummy = 0;
+                if (q_use) mbar_wait(&bars[kQFull], (q_use - 1) & 1, &dummy);
+                if (k_use) mbar_wait(&bars[kKFull], (k_use - 1) & 1, &dummy);
+                if (v_use) mbar_wait(&bars[kVFull], (v_use - 1) & 1, &dummy);
+            }
+        }
+    } else if (warp == 5) {
+        // ============================================================ MMA issuer
+        int it_use = 0, q_use = 0, k_use = 0, v_use = 0, p_use = 0, o_use = 0;
+        bool ok = true;
+        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+        while (ok) {
+            const int slot = it_use & 1;
+            int4 it = make_int4(-1, 0, 0, 0);
+            if (lane == 0) {
+                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+                if (ok) it = s_item[slot];
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+            if (!ok) break;
+            it.x = __shfl_sync(kFull, it.x, 0);
+            it_use++;
+            if (it.x < 0) break;
+            if (lane == 0) {
+                const Item s = load_item<KIND>(p, it);
+                const int n_kt = (s.Lk + kTileN - 1) / kTileN;
+                int last = -1;
+                for (int t = 0; t < n_kt; t++)
+                    if (kv_class<KIND>(s, t) != 0) last = t;
+                ok = mbar_wait(&bars[kQFull], q_use & 1, s_abort);
+                q_use++;
+                tc_fence_after();
+                int n_done = 0;
+                for (int t = 0; ok && t <= last; t++) {
+                    if (kv_class<KIND>(s, t) == 0) continue;
+                    ok = mbar_wait(&bars[kKFull], k_use & 1, s_abort);
+                    if (!ok) break;
+                    k_use++;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; kk++) {
+                        const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
+                        mma_ss(tmem + kSCol, sdesc_sw128(aQ + off, 16, 1024),
+                               sdesc_sw128(aK + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bars[kSFull]);
+                    tc_commit(&bars[kKEmpty]);
+                    if (t == last) tc_commit(&bars[kQEmpty]);
+                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort);
+                    if (!ok) break;
+                    p_use++;
+                    ok = mbar_wait(&bars[kVFull], v_use & 1, s_abort);
+                    if (!ok) break;
+                    v_use++;
+                    if (n_done == 0) {
+                        ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort);
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTileN / 16; kk++) {
+                        mma_ts(tmem + kOCol, tmem + kSCol + kk * 8,
+                               sdesc_sw128(aV + kk * 2048, kPanelBytes, 1024), kIdescO,
+                               (n_done > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&bars[kVEmpty]);
+                    n_done++;
+                }
+                if (ok && n_done == 0) {
+                    tc_commit(&bars[kQEmpty]);
+                    ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort);
+                }
+                if (ok) {
+                    o_use++;
+                    tc_commit(&bars[kOFull]);
+                    mbar_arrive(&bars[kItEmpty0 + slot]);
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+        }
+        if (lane == 0) {
+            if (!ok && !*s_abort) flag_timeout(p, s_abort);
+            // every MMA this thread issued completes before TMEM is released
+            volatile int dummy = 0;
+            tc_commit(&bars[kDrain]);
+            mbar_wait(&bars[kDrain], 0, &dummy);
+        }
+    } else {
+        // ============================================================ elementwise (warps 0-3)
+        int it_use = 0, s_use = 0, o_use = 0;
+        const int r = tid;                                  // TMEM lane = tile row
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        int64_t* w_cts = s_cts + warp * 128;
+        const float rp_self = s_rp[p.P - 1];
+        const float rt_zero = s_rt[0];
+        bool ok = true;
+        while (ok) {
+            const int slot = it_use & 1;
+            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+            if (!__all_sync(kFull, ok)) { ok = false; break; }
+            const int4 it = s_item[slot];
+            it_use++;
+            if (it.x < 0) break;
+            const Item s = load_item<KIND>(p, it);
+            const int i = s.row0 + r;
+            const bool row_ok = i < s.row_end;
+            const int ic = min(i, s.row_end - 1);           // clamped row for lookups
+            const int64_t ts_i = p.q_ts[s.q0 + ic];
+            const int pos_i = row_pos<KIND>(s, ic);
+            // this warp's row range (positions and timestamps)
+            int64_t rmin = row_ok ? ts_i : INT64_MAX, rmax = row_ok ? ts_i : INT64_MIN;
+            int pr_lo = row_ok ? pos_i : INT32_MAX, pr_hi = row_ok ? pos_i : INT32_MIN;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                rmin = min(rmin, (int64_t)__shfl_xor_sync(kFull, (long long)rmin, o));
+                rmax = max(rmax, (int64_t)__shfl_xor_sync(kFull, (long long)rmax, o));
+                pr_lo = min(pr_lo, __shfl_xor_sync(kFull, pr_lo, o));
+                pr_hi = max(pr_hi, __shfl_xor_sync(kFull, pr_hi, o));
+            }
+            const bool warp_rows = pr_lo <= pr_hi;          // any valid row in this warp
+            const int n_kt = (s.Lk + kTileN - 1) / kTileN;
+            int n_done = 0;
+            for (int t = 0; t < n_kt; t++) {
+                const int cls = kv_class<KIND>(s, t);
+                if (cls == 0) continue;
+                const int n0 = t * kTileN;
+                // column timestamps of this tile (each warp keeps its own copy)
+                __syncwarp();
+                int64_t cmin = INT64_MAX, cmax = INT64_MIN;
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int jj = lane + 32 * e;
+                    const int j = n0 + jj;
+                    const int64_t tj = j < s.Lk ? p.kv_ts[s.kv0 + j] : 0;
+                    w_cts[jj] = tj;
+                    if (j < s.Lk) {
+                        cmin = min(cmin, tj);
+                        cmax = max(cmax, tj);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    cmin = min(cmin, (int64_t)__shfl_xor_sync(kFull, (long long)cmin, o));
+                    cmax = max(cmax, (int64_t)__shfl_xor_sync(kFull, (long long)cmax, o));
+                }
+                __syncwarp();
+                // uniform-bias test for this warp's 32 rows x 128 columns
+                const int jl = min(n0 + kTileN, s.Lk) - 1;
+                bool fast = warp_rows && cls == 2 && n0 + kTileN <= s.Lk;
+                float cbias = 0.f;
+                if (fast) {
+                    const int dmax = col_pos<KIND>(s, jl) - pr_lo;
+                    const int dmin = col_pos<KIND>(s, n0) - pr_hi;
+                    int pidx = -1;
+                    if (dmax <= -(p.P - 1)) pidx = 0;
+                    else if (dmin >= p.P - 1) pidx = 2 * p.P - 2;
+                    uint64_t lo;
+                    if (rmin > cmax) lo = abs_diff_u64(rmin, cmax);
+                    else if (cmin > rmax) lo = abs_diff_u64(cmin, rmax);
+                    else lo = 0;
+                    const uint64_t hi = max(abs_diff_u64(rmax, cmin), abs_diff_u64(cmax, rmin));
+                    const int tlo = time_bucket_of_delta(lo, p.nb), thi = time_bucket_of_delta(hi, p.nb);
+                    fast = pidx >= 0 && tlo == thi;
+                    if (fast) cbias = s_rp[pidx] + s_rt[tlo];
+                }
+                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
+                if (!__all_sync(kFull, ok)) { ok = false; break; }
+                s_use++;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 4; c++) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
+                    tmem_ld_wait(v);
+                    uint32_t pk[16];
+                    if (fast) {
+#pragma unroll
+                        for (int e = 0; e < 16; e++) {
+                            const float p0 = silu_fast(__uint_as_float(v[2 * e]) + cbias);
+                            const float p1 = silu_fast(__uint_as_float(v[2 * e + 1]) + cbias);
+                            pk[e] = pack_bf16x2(p0, p1);
+                        }
+                    } else {
+                        float pv[32];
+#pragma unroll
+                        for (int e = 0; e < 32; e++) {
+                            const int jj = 32 * c + e;
+                            const int j = n0 + jj;
+                            const int64_t ts_j = w_cts[jj];
+                            bool vis = row_ok && j < s.Lk;
+                            if (KIND != HSTU_KIND_MFALCON)
+                                vis = vis && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
+                            const int pidx = pos_index(pos_i, col_pos<KIND>(s, j), p.P);
+                            const int tb = time_bucket(ts_i, ts_j, p.nb);
+                            const float z = __uint_as_float(v[e]) + s_rp[pidx] + s_rt[tb];
+                            pv[e] = vis ? silu_fast(z) : 0.f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; e++) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+                    }
+                    tmem_st16(tmem + lane_base + kSCol + 16 * c, pk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars[kPFull]);
+                n_done++;
+            }
+            if (!ok) break;
+            // ---------------- epilogue
+            float a_self = 0.f;
+            const __nv_bfloat16* vself = nullptr;
+            if (KIND == HSTU_KIND_MFALCON && row_ok) {
+                const size_t ro = (size_t)(s.q0 + i) * p.ld + (size_t)s.h * D;
+                const uint4* qs = reinterpret_cast<const uint4*>(p.self_q + ro);
+                const uint4* ks = reinterpret_cast<const uint4*>(p.self_k + ro);
+                float dot = 0.f;
+#pragma unroll 4
+                for (int e = 0; e < D / 8; e++) {
+                    const uint4 a = qs[e], b = ks[e];
+                    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+                    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+                    for (int f = 0; f < 4; f++) {
+                        const float2 x = __bfloat1622float2(a2[f]), y2 = __bfloat1622float2(b2[f]);
+                        dot = fmaf(x.x, y2.x, dot);
+                        dot = fmaf(x.y, y2.y, dot);
+                    }
+                }
+                a_self = silu_fast(dot + rp_self + rt_zero);
+                vself = p.self_v + ro;
+            }
+            ok = mbar_wait(&bars[kOFull], o_use & 1, s_abort);
+            if (!__all_sync(kFull, ok)) { ok = false; break; }
+            o_use++;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; c++) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + kOCol + 32 * c, v);
+                tmem_ld_wait(v);
+                if (row_ok) {
+                    float o[32];
+#pragma unroll
+                    for (int e = 0; e < 32; e++) o[e] = n_done ? __uint_as_float(v[e]) : 0.f;
+                    if (KIND == HSTU_KIND_MFALCON) {
+                        const uint4* vs = reinterpret_cast<const uint4*>(vself + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const uint4 a = vs[e];
+                            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+#pragma unroll
+                            for (int f = 0; f < 4; f++) {
+                                const float2 x = __bfloat1622float2(a2[f]);
+                                o[8 * e + 2 * f] = fmaf(a_self, x.x, o[8 * e + 2 * f]);
+                                o[8 * e + 2 * f + 1] = fmaf(a_self, x.y, o[8 * e + 2 * f + 1]);
+                            }
+                        }
+                    }
+                    uint4 w[4];
+                    uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+                    for (int e = 0; e < 16; e++)
+                        wp[e] = pack_bf16x2(o[2 * e] * p.inv_alpha, o[2 * e + 1] * p.inv_alpha);
+                    uint4* dst = reinterpret_cast<uint4*>(p.y + (size_t)(s.q0 + i) * p.ld +
+                                                          (size_t)s.h * D + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) dst[e] = w[e];
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[kOEmpty]);
+            mbar_arrive(&bars[kItEmpty0 + slot]);
+        }
+        if (!ok && lane == 0 && !*s_abort) flag_timeout(p, s_abort);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int KIND, int D>
+cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, int grid, cudaStream_t s) {
+    constexpr uint32_t smem = FwdSmem<D>::alloc;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    prof_begin(kProfAttnFwdTc, s);
+    attn_fwd_tc_kernel<KIND, D><<<grid, kThreads, smem, s>>>(tq, tk, tv, p);
+    prof_end(kProfAttnFwdTc, s);
+    return cudaGetLastError();
+}
+
+template <int KIND, int D>
+int ctas_per_sm_one() {
+    constexpr uint32_t smem = FwdSmem<D>::alloc;
+    cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_fwd_tc_kernel<KIND, D>, kThreads,
+                                                      smem) != cudaSuccess)
+        return 1;
+    return n < 1 ? 1 : (n > 2 ? 2 : n);   // two CTAs fill the SM's 512 TMEM columns
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t s) {
+#define HSTU_FWD_CASE(K, DD) \
+    if (kind == K && d == DD) return launch_one<K, DD>(tq, tk, tv, p, grid, s);
+    HSTU_FWD_CASE(HSTU_KIND_CAUSAL, 128)
+    HSTU_FWD_CASE(HSTU_KIND_CAUSAL, 64)
+    HSTU_FWD_CASE(HSTU_KIND_MTGR, 128)
+    HSTU_FWD_CASE(HSTU_KIND_MTGR, 64)
+    HSTU_FWD_CASE(HSTU_KIND_MFALCON, 128)
+    HSTU_FWD_CASE(HSTU_KIND_MFALCON, 64)
+#undef HSTU_FWD_CASE
+    return cudaErrorInvalidValue;
+}
+
+int attn_fwd_tc_ctas_per_sm(int kind, int d) {
+#define HSTU_OCC_CASE(K, DD) \
+    if (kind == K && d == DD) return ctas_per_sm_one<K, DD>();
+    HSTU_OCC_CASE(HSTU_KIND_CAUSAL, 128)
+    HSTU_OCC_CASE(HSTU_KIND_CAUSAL, 64)
+    HSTU_OCC_CASE(HSTU_KIND_MTGR, 128)
+    HSTU_OCC_CASE(HSTU_KIND_MTGR, 64)
+    HSTU_OCC_CASE(HSTU_KIND_MFALCON, 128)
+    HSTU_OCC_CASE(HSTU_KIND_MFALCON, 64)
+#undef HSTU_OCC_CASE
+    return 1;
+}
+
+}  // namespace hstu

@@ -1,0 +1,139 @@
+// internal.h -- shared declarations of libhstu_b200 (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "hstu_rules.cuh"
+
+namespace hstu {
+
+constexpr int kTileM = 128;         // query rows per tcgen05 tile
+constexpr int kTileN = 128;         // key rows per tcgen05 tile
+constexpr int kMaxPos = 1024;       // largest P the kernels keep in shared memory
+constexpr int kMaxTBuckets = 64;
+constexpr int kSchedBins = 4096;    // distinct sort keys in the scheduler
+constexpr int kMaxSeqLen = kSchedBins * kTileM - 1;
+
+// device status word bits (inside the workspace control block)
+constexpr int kStatusBounds = 1;
+constexpr int kStatusTimeout = 2;
+
+// Control block at the start of every workspace.
+struct Control {
+    int status;      // kStatus* bits, cleared by hstu_check_device_error
+    int n_items;     // work items written by the scheduler
+    int counter;     // dynamic item counter of the persistent kernels
+    int valid;       // 1 when the latest scheduler run accepted the inputs
+    int pad[60];
+};
+static_assert(sizeof(Control) == 256, "control block is 256 bytes");
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Work item: sequence b, query rows [row0, row_end) local to the sequence, head h.
+// Stored as int4 {b, row0, h, row_end}.
+
+struct SchedParams {
+    int kind, B, Tq, Tkv, H;
+    const int32_t* q_off;
+    const int32_t* kv_off;
+    const int32_t* n_static;
+    const int32_t* n_rt;
+    int max_q_len, max_kv_len, b_m;
+    Control* ctrl;
+    int4* items;
+    int* perm;       // [B]
+    int* seq_base;   // [B]
+    long long max_items;
+};
+
+struct FwdParams {
+    const int32_t* q_off;
+    const int32_t* kv_off;
+    const int64_t* q_ts;
+    const int64_t* kv_ts;
+    const int32_t* n_static;
+    const int32_t* n_rt;
+    const float* rab_pos;
+    const float* rab_time;
+    const int4* items;
+    Control* ctrl;
+    __nv_bfloat16* y;
+    const __nv_bfloat16* self_q;   // M-FALCON candidate q/k/v for the self term
+    const __nv_bfloat16* self_k;
+    const __nv_bfloat16* self_v;
+    int H, P, nb, ld;
+    float inv_alpha;
+};
+
+// Generic (CUDA-core, fp32 arithmetic) attention kernels' parameters.
+struct SimtParams {
+    int kind, B, H, P, nb, max_len;
+    const int32_t* off;
+    const int64_t* ts;
+    const int32_t* n_static;
+    const int32_t* n_rt;
+    const float* rab_pos;
+    const float* rab_time;
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* dy;      // backward: dL/dY
+    void* y;             // forward output
+    void* dq;
+    void* dk;
+    void* dv;
+    float* d_rab_pos;
+    float* d_rab_time;
+    float inv_alpha;
+    const Control* ctrl;   // kernels do nothing unless ctrl->valid
+};
+
+struct LnParams {
+    long long T;
+    int D;
+    const void* y;
+    const void* u;
+    const float* gamma;
+    const float* beta;
+    float eps;
+    void* o;
+    float* mean;
+    float* rstd;
+    // backward
+    const void* g;
+    void* dy;
+    void* du;
+    float* part;     // [n_blocks][2][D]
+    int n_part;
+    float* d_gamma;
+    float* d_beta;
+};
+
+// ---- opt-in per-kernel timing (profile.cu)
+enum ProfKind {
+    kProfSchedule = 0, kProfAttnFwdTc, kProfAttnFwdSimt, kProfLnFwd, kProfLnBwd, kProfLnBwdReduce,
+    kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfKinds
+};
+void prof_begin(int kind, cudaStream_t s);
+void prof_end(int kind, cudaStream_t s);
+
+// ---- launchers (return cudaError_t of the launch)
+cudaError_t launch_schedule(const SchedParams& p, cudaStream_t s);
+cudaError_t launch_attn_fwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t s);
+int attn_fwd_tc_ctas_per_sm(int kind, int d);
+cudaError_t launch_attn_fwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
+cudaError_t launch_attn_bwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
+cudaError_t launch_ln_fwd(int dtype_f32, const LnParams& p, cudaStream_t s);
+cudaError_t launch_ln_bwd(int dtype_f32, const LnParams& p, cudaStream_t s);
+int ln_bwd_partials(long long T);
+cudaError_t launch_debug_indices(int B, int kind, const int32_t* off, const int64_t* ts,
+                                 const int32_t* ns, const int32_t* nr, int P, int nb,
+                                 const int64_t* pair_off, int max_len, uint8_t* m, int16_t* pi,
+                                 int8_t* tb, cudaStream_t s);
+
+}  // namespace hstu

@@ -1,0 +1,195 @@
+"""Torch-facing binding of libhstu_b200: argument marshalling only.
+
+Every function takes CUDA tensors, allocates outputs and workspace with torch
+(unless the caller passes them), and calls one C-ABI entry point on the
+current CUDA stream.  All computation runs in the library's kernels.
+
+Layout (see include/hstu.h): q, k, v, u are jagged ``[T, H*d]`` row-major
+tensors (bf16, or fp32 for the fp32 path), ``seq_offsets`` int32 ``[B+1]``,
+``timestamps`` int64 ``[T]``, ``rab_pos`` fp32 ``[2P-1]``, ``rab_time`` fp32
+``[nb]``, ``ln_gamma``/``ln_beta`` fp32 ``[H*d]``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from typing import Optional
+
+import torch
+
+from . import capi
+
+_DTYPES = {torch.bfloat16: capi.HSTU_BF16, torch.float32: capi.HSTU_F32}
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def make_dims(T: int, B: int, H: int, d: int, dtype: torch.dtype, alpha: float, max_seq_len: int,
+              n_pos: int = 256, n_tbuckets: int = 64, ln_eps: float = 1e-5) -> capi.HstuDims:
+    return capi.HstuDims(B=B, T=T, H=H, d_qk=d, d_v=d, dtype=_DTYPES[dtype], n_pos=n_pos,
+                         n_tbuckets=n_tbuckets, max_seq_len=max_seq_len, alpha=float(alpha),
+                         ln_eps=float(ln_eps))
+
+
+def make_mask(kind: str = "causal", n_static: Optional[torch.Tensor] = None,
+              n_realtime: Optional[torch.Tensor] = None) -> capi.HstuMaskSpec:
+    if kind == "causal":
+        return capi.HstuMaskSpec(kind=capi.HSTU_MASK_CAUSAL, n_static=None, n_realtime=None)
+    if kind == "mtgr":
+        _need(n_static, "n_static", torch.int32)
+        _need(n_realtime, "n_realtime", torch.int32)
+        return capi.HstuMaskSpec(kind=capi.HSTU_MASK_MTGR, n_static=n_static.data_ptr(),
+                                 n_realtime=n_realtime.data_ptr())
+    raise ValueError(f"unknown mask kind {kind!r}")
+
+
+def attn_workspace_bytes(dims: capi.HstuDims, mask_kind: int, is_bwd: bool) -> int:
+    n = capi.LIB.hstu_attn_workspace_bytes(C.byref(dims), mask_kind, 1 if is_bwd else 0)
+    if n == 0:
+        raise capi.HstuError(capi.HSTU_ERR_INVALID_ARG, "hstu_attn_workspace_bytes")
+    return int(n)
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A zeroed byte buffer usable as workspace (torch allocations are 256-byte aligned)."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+class Layer:
+    """Holds the shapes, mask and workspace of one jagged HSTU attention layer.
+
+    Reusing a Layer across steps keeps the workspace (and its status word)
+    resident, so the forward/backward calls allocate only their outputs.
+    """
+
+    def __init__(self, seq_offsets: torch.Tensor, timestamps: torch.Tensor, H: int, d: int,
+                 dtype: torch.dtype, alpha: float, max_seq_len: int, mask_kind: str = "causal",
+                 n_static: Optional[torch.Tensor] = None, n_realtime: Optional[torch.Tensor] = None,
+                 n_pos: int = 256, n_tbuckets: int = 64, ln_eps: float = 1e-5):
+        _need(seq_offsets, "seq_offsets", torch.int32)
+        _need(timestamps, "timestamps", torch.int64)
+        self.seq_offsets, self.timestamps = seq_offsets, timestamps
+        self.B = seq_offsets.numel() - 1
+        self.T = timestamps.numel()
+        self.H, self.d, self.dtype = H, d, dtype
+        self.n_static, self.n_realtime = n_static, n_realtime
+        self.dims = make_dims(self.T, self.B, H, d, dtype, alpha, max_seq_len, n_pos, n_tbuckets, ln_eps)
+        self.mask = make_mask(mask_kind, n_static, n_realtime)
+        self.device = seq_offsets.device
+        n = max(attn_workspace_bytes(self.dims, self.mask.kind, False),
+                attn_workspace_bytes(self.dims, self.mask.kind, True))
+        self.ws = workspace(n, self.device)
+
+    @property
+    def D(self) -> int:
+        return self.H * self.d
+
+    def forward(self, q, k, v, u, rab_pos, rab_time, ln_gamma, ln_beta, out: Optional[dict] = None) -> dict:
+        for t, n in ((q, "q"), (k, "k"), (v, "v"), (u, "u")):
+            _need(t, n, self.dtype)
+        for t, n in ((rab_pos, "rab_pos"), (rab_time, "rab_time"), (ln_gamma, "ln_gamma"), (ln_beta, "ln_beta")):
+            _need(t, n, torch.float32)
+        if out is None:
+            out = dict(y=torch.empty_like(q), o_pre=torch.empty_like(q),
+                       mean=torch.empty(self.T, dtype=torch.float32, device=self.device),
+                       rstd=torch.empty(self.T, dtype=torch.float32, device=self.device))
+        st = capi.LIB.hstu_attn_fwd(
+            C.byref(self.dims), C.byref(self.mask), _p(q), _p(k), _p(v), _p(u), _p(self.seq_offsets),
+            _p(self.timestamps), _p(rab_pos), _p(rab_time), _p(ln_gamma), _p(ln_beta), _p(out["y"]),
+            _p(out["o_pre"]), _p(out["mean"]), _p(out["rstd"]), _p(self.ws), self.ws.numel(), _stream())
+        capi.check(st, "hstu_attn_fwd")
+        return out
+
+    def backward(self, q, k, v, u, rab_pos, rab_time, ln_gamma, ln_beta, fwd: dict, d_o_pre,
+                 out: Optional[dict] = None) -> dict:
+        _need(d_o_pre, "d_o_pre", self.dtype)
+        if out is None:
+            out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                       du=torch.empty_like(u),
+                       d_rab_pos=torch.empty_like(rab_pos), d_rab_time=torch.empty_like(rab_time),
+                       d_gamma=torch.empty_like(ln_gamma), d_beta=torch.empty_like(ln_beta))
+        st = capi.LIB.hstu_attn_bwd(
+            C.byref(self.dims), C.byref(self.mask), _p(q), _p(k), _p(v), _p(u), _p(self.seq_offsets),
+            _p(self.timestamps), _p(rab_pos), _p(rab_time), _p(ln_gamma), _p(ln_beta), _p(fwd["y"]),
+            _p(fwd["mean"]), _p(fwd["rstd"]), _p(d_o_pre), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+            _p(out["du"]), _p(out["d_rab_pos"]), _p(out["d_rab_time"]), _p(out["d_gamma"]),
+            _p(out["d_beta"]), _p(self.ws), self.ws.numel(), _stream())
+        capi.check(st, "hstu_attn_bwd")
+        return out
+
+    def check_device_error(self) -> int:
+        return int(capi.LIB.hstu_check_device_error(_p(self.ws), _stream()))
+
+
+class MFalcon:
+    """M-FALCON candidate scoring against cached history K/V (microbatch b_m)."""
+
+    def __init__(self, hist_offsets, hist_ts, cand_offsets, cand_ts, H: int, d: int, alpha: float,
+                 b_m: int, max_hist_len: int, max_cand_len: int, n_pos: int = 256, n_tbuckets: int = 64,
+                 ln_eps: float = 1e-5):
+        for t, n, dt in ((hist_offsets, "hist_offsets", torch.int32), (cand_offsets, "cand_offsets", torch.int32),
+                         (hist_ts, "hist_ts", torch.int64), (cand_ts, "cand_ts", torch.int64)):
+            _need(t, n, dt)
+        self.hist_offsets, self.hist_ts, self.cand_offsets, self.cand_ts = hist_offsets, hist_ts, cand_offsets, cand_ts
+        self.B = cand_offsets.numel() - 1
+        self.b_m = int(b_m)
+        self.H, self.d = H, d
+        self.dims = capi.HstuMfalconDims(B=self.B, T_hist=hist_ts.numel(), T_cand=cand_ts.numel(), H=H, d_qk=d,
+                                         d_v=d, dtype=capi.HSTU_BF16, n_pos=n_pos, n_tbuckets=n_tbuckets,
+                                         max_hist_len=max_hist_len, max_cand_len=max_cand_len,
+                                         alpha=float(alpha), ln_eps=float(ln_eps))
+        n = capi.LIB.hstu_mfalcon_workspace_bytes(C.byref(self.dims), self.b_m)
+        if n == 0:
+            raise capi.HstuError(capi.HSTU_ERR_INVALID_ARG, "hstu_mfalcon_workspace_bytes")
+        self.ws = workspace(int(n), cand_offsets.device)
+
+    def score(self, hist_k, hist_v, cand_q, cand_k, cand_v, cand_u, rab_pos, rab_time, ln_gamma, ln_beta,
+              out: Optional[dict] = None) -> dict:
+        for t, n in ((hist_k, "hist_k"), (hist_v, "hist_v"), (cand_q, "cand_q"), (cand_k, "cand_k"),
+                     (cand_v, "cand_v"), (cand_u, "cand_u")):
+            _need(t, n, torch.bfloat16)
+        if out is None:
+            out = dict(y=torch.empty_like(cand_q), o_pre=torch.empty_like(cand_q))
+        st = capi.LIB.hstu_mfalcon_score(
+            C.byref(self.dims), _p(hist_k), _p(hist_v), _p(self.hist_offsets), _p(self.hist_ts), _p(cand_q),
+            _p(cand_k), _p(cand_v), _p(cand_u), _p(self.cand_offsets), _p(self.cand_ts), _p(rab_pos),
+            _p(rab_time), _p(ln_gamma), _p(ln_beta), self.b_m, _p(out["y"]), _p(out["o_pre"]), _p(self.ws),
+            self.ws.numel(), _stream())
+        capi.check(st, "hstu_mfalcon_score")
+        return out
+
+    def check_device_error(self) -> int:
+        return int(capi.LIB.hstu_check_device_error(_p(self.ws), _stream()))
+
+
+def debug_indices(seq_offsets, timestamps, mask_kind: str = "causal", n_static=None, n_realtime=None,
+                  n_pos: int = 256, n_tbuckets: int = 64):
+    """Per-pair (mask, rab_pos index, time bucket) from the kernels' own device functions."""
+    _need(seq_offsets, "seq_offsets", torch.int32)
+    _need(timestamps, "timestamps", torch.int64)
+    L = (seq_offsets[1:] - seq_offsets[:-1]).to(torch.int64)
+    po = torch.zeros(L.numel() + 1, dtype=torch.int64, device=seq_offsets.device)
+    po[1:] = torch.cumsum(L * L, 0)
+    n = int(po[-1].item())
+    m = torch.zeros(n, dtype=torch.uint8, device=seq_offsets.device)
+    pi = torch.zeros(n, dtype=torch.int16, device=seq_offsets.device)
+    tb = torch.zeros(n, dtype=torch.int8, device=seq_offsets.device)
+    kind = capi.HSTU_MASK_MTGR if mask_kind == "mtgr" else capi.HSTU_MASK_CAUSAL
+    st = capi.LIB.hstu_debug_indices(L.numel(), kind, _p(seq_offsets), _p(timestamps), _p(n_static),
+                                     _p(n_realtime), n_pos, n_tbuckets, _p(po), _p(m), _p(pi), _p(tb), _stream())
+    capi.check(st, "hstu_debug_indices")
+    return m, pi, tb, po

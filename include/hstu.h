@@ -1,0 +1,207 @@
+/*
+ * hstu.h -- C ABI of libhstu_b200: jagged HSTU pointwise attention on B200 (sm_100a).
+ *
+ * The operation (Meta HSTU blog, section 3 "HSTU formula" and 3.1 "Pointwise
+ * Attention"): for every sequence b, head h and query i of a jagged batch,
+ *
+ *     z_ij = q_i . k_j + rab_pos[pidx(i, j)] + rab_time[tb(i, j)]          (section 3.2)
+ *     Y_i  = (1/alpha) * sum_j mask(i, j) * SiLU(z_ij) * v_j               (no row normalisation)
+ *     O_pre_i = (LayerNorm(Y_i) * gamma + beta) (.) u_i                    (LayerNorm over D = H*d_v)
+ *
+ *   pidx(i, j) = clamp(pos(j) - pos(i), -(P-1), P-1) + (P-1)    (rab_pos has 2P-1 entries)
+ *   tb(i, j)   = min(nb - 1, bit_length(|ts(i) - ts(j)|))       (rab_time has nb entries)
+ *   pos(i)     = i, except MTGR candidates, which all sit at pos = S + R
+ *
+ * Masks: HSTU_MASK_CAUSAL (j <= i; MTGR deep-dive section 2, "classic GR causal
+ * mask") and HSTU_MASK_MTGR, the dynamic mixed mask (MTGR deep-dive section 2;
+ * MTGR arXiv report section 3.1): in a row laid out as [S static | R real-time |
+ * K candidates], static tokens see static tokens, a real-time token sees static
+ * tokens and real-time tokens j <= i, a candidate sees itself and every
+ * non-candidate whose timestamp is strictly smaller than its own.
+ * hstu_mfalcon_score is the M-FALCON candidate mask over cached history K/V
+ * (HSTU blog, sections 4.2-4.3): candidates see all history and themselves.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller.  Host structs
+ *    (hstu_dims, hstu_mask_spec, hstu_mfalcon_dims) are read before return and
+ *    may be freed afterwards; the device arrays they point to must stay valid
+ *    until the stream work finishes.  The library keeps no pointer after return
+ *    and allocates no device memory: all scratch comes from `workspace`.
+ *  - Layout: values are row-major [T, H*d] (token-major, heads concatenated),
+ *    element type given by dims.dtype; seq_offsets is int32 [B+1] with
+ *    seq_offsets[0] = 0, non-decreasing, seq_offsets[B] = T; timestamps are
+ *    int64 [T] (seconds); rab_pos fp32 [2P-1]; rab_time fp32 [nb];
+ *    ln_gamma / ln_beta fp32 [H*d_v]; ln_mean / ln_rstd fp32 [T].
+ *  - All work is asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Synchronous argument checks return a negative hstu_status and launch
+ *    nothing.  Errors that only the device can see (offsets that are not
+ *    monotone, a sequence longer than dims.max_seq_len, MTGR segment sizes that
+ *    do not fit, a bounded wait that ran out) are recorded in a status word
+ *    inside `workspace`; the affected launch then does no work.  Read and
+ *    clear it with hstu_check_device_error().
+ *  - Alignment: every tensor pointer 16-byte aligned; H*d*elem_size a multiple of 16.
+ *  - Supported: dtype HSTU_BF16 with d_qk = d_v in {64, 128}; dtype HSTU_F32 with
+ *    d_qk = d_v in {32, 64, 128}; P in [1, 1024]; nb in [1, 64]; H >= 1; H*d_v <= 8192;
+ *    max_seq_len <= 524287.
+ */
+#ifndef HSTU_B200_H
+#define HSTU_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HSTU_API __attribute__((visibility("default")))
+#else
+#define HSTU_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HSTU_OK = 0,
+    HSTU_ERR_INVALID_ARG = -1,   /* a pointer, size or flag failed the host check */
+    HSTU_ERR_UNSUPPORTED = -2,   /* a valid request this build does not implement */
+    HSTU_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed */
+    HSTU_ERR_DEVICE_TIMEOUT = -4,/* a bounded device wait ran out (device status word) */
+    HSTU_ERR_DEVICE_BOUNDS = -5, /* offsets / lengths / segments invalid (device status word) */
+    HSTU_ERR_WORKSPACE = -6      /* workspace missing or smaller than the query returned */
+} hstu_status;
+
+typedef enum { HSTU_BF16 = 0, HSTU_F32 = 1 } hstu_dtype;
+
+typedef enum { HSTU_MASK_CAUSAL = 0, HSTU_MASK_MTGR = 1 } hstu_mask_kind;
+
+/* Mask description.  For HSTU_MASK_MTGR, n_static[b] (profile + long-term
+ * tokens, seen bidirectionally) and n_realtime[b] are DEVICE int32 [B]; the
+ * remaining L_b - n_static[b] - n_realtime[b] tokens of row b are candidates.
+ * Both pointers are ignored for HSTU_MASK_CAUSAL. */
+typedef struct {
+    int32_t kind;                /* hstu_mask_kind */
+    const int32_t* n_static;     /* device [B] */
+    const int32_t* n_realtime;   /* device [B] */
+} hstu_mask_spec;
+
+typedef struct {
+    int32_t B;            /* sequences in the jagged batch */
+    int32_t T;            /* total tokens = seq_offsets[B] */
+    int32_t H;            /* heads */
+    int32_t d_qk;         /* per-head query/key width */
+    int32_t d_v;          /* per-head value width (must equal d_qk) */
+    int32_t dtype;        /* hstu_dtype of q, k, v, u, y, o_pre and the gradients */
+    int32_t n_pos;        /* P: rab_pos has 2P-1 entries (256 in the workloads) */
+    int32_t n_tbuckets;   /* nb: rab_time entries (64 in the workloads) */
+    int32_t max_seq_len;  /* upper bound on every L_b (checked on the device) */
+    float alpha;          /* Y = sum(...) / alpha; > 0 */
+    float ln_eps;         /* LayerNorm epsilon (1e-5 in the workloads) */
+} hstu_dims;
+
+/* Bytes of workspace hstu_attn_fwd (is_bwd = 0) or hstu_attn_bwd (is_bwd = 1)
+ * needs for these dims and mask kind; 0 when the arguments are invalid. */
+HSTU_API size_t hstu_attn_workspace_bytes(const hstu_dims* dims, int32_t mask_kind, int32_t is_bwd);
+
+/* Forward of one HSTU attention layer (formula above).
+ * In:  q, k [T, H*d_qk]; v, u [T, H*d_v]; seq_offsets, timestamps, rab tables,
+ *      mask, ln_gamma, ln_beta.
+ * Out: y [T, H*d_v] (the attention output Y, saved for the backward),
+ *      o_pre [T, H*d_v], ln_mean [T], ln_rstd [T].
+ * Rows of y / o_pre that belong to no sequence are not written. */
+HSTU_API int hstu_attn_fwd(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const void* q, const void* k, const void* v, const void* u,
+                  const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta,
+                  void* y, void* o_pre, float* ln_mean, float* ln_rstd,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of hstu_attn_fwd for the upstream gradient d_o_pre [T, H*d_v].
+ * The A = SiLU(z) matrix is recomputed, never stored.
+ * Out: dq, dk [T, H*d_qk]; dv, du [T, H*d_v] (element type dims.dtype);
+ *      d_rab_pos fp32 [2P-1], d_rab_time fp32 [nb], d_gamma, d_beta fp32 [H*d_v].
+ * Every output is overwritten, not accumulated.  y, ln_mean and ln_rstd are the
+ * forward's outputs for the same inputs. */
+HSTU_API int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const void* q, const void* k, const void* v, const void* u,
+                  const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta,
+                  const void* y, const float* ln_mean, const float* ln_rstd,
+                  const void* d_o_pre,
+                  void* dq, void* dk, void* dv, void* du,
+                  float* d_rab_pos, float* d_rab_time, float* d_gamma, float* d_beta,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* M-FALCON (HSTU blog, sections 4.2-4.3): candidates scored against cached history K/V. */
+typedef struct {
+    int32_t B;            /* users */
+    int32_t T_hist;       /* hist_offsets[B] */
+    int32_t T_cand;       /* cand_offsets[B] */
+    int32_t H, d_qk, d_v; /* heads and per-head widths (d_qk = d_v) */
+    int32_t dtype;        /* HSTU_BF16 only */
+    int32_t n_pos, n_tbuckets;
+    int32_t max_hist_len; /* upper bound on every history length (device-checked) */
+    int32_t max_cand_len; /* upper bound on every user's candidate count (device-checked) */
+    float alpha, ln_eps;
+} hstu_mfalcon_dims;
+
+/* Workspace bytes hstu_mfalcon_score needs; 0 when the arguments are invalid. */
+HSTU_API size_t hstu_mfalcon_workspace_bytes(const hstu_mfalcon_dims* dims, int32_t b_m);
+
+/* For candidate c of user b with n = history length of b, history positions
+ * 0..n-1 and every candidate at position n:
+ *   Y_c = (1/alpha) [ sum_{j<n} SiLU(q_c.k_j + rab_pos[pidx(n, j)] + rab_time[tb(ts_c, ts_j)]) v_j
+ *                     + SiLU(q_c.k_c + rab_pos[P-1] + rab_time[0]) v_c ]
+ *   O_pre_c = (LayerNorm(Y_c) * gamma + beta) (.) u_c
+ * In:  hist_k, hist_v [T_hist, H*d] with hist_offsets int32 [B+1], hist_ts int64 [T_hist];
+ *      cand_q, cand_k, cand_v, cand_u [T_cand, H*d] with cand_offsets [B+1], cand_ts [T_cand].
+ * b_m (> 0) is the candidate microbatch: candidates are processed in groups of b_m
+ * per user; it changes the schedule only, never the results.
+ * Out: y [T_cand, H*d] and o_pre [T_cand, H*d]. */
+HSTU_API int hstu_mfalcon_score(const hstu_mfalcon_dims* dims,
+                       const void* hist_k, const void* hist_v,
+                       const int32_t* hist_offsets, const int64_t* hist_ts,
+                       const void* cand_q, const void* cand_k, const void* cand_v, const void* cand_u,
+                       const int32_t* cand_offsets, const int64_t* cand_ts,
+                       const float* rab_pos, const float* rab_time,
+                       const float* ln_gamma, const float* ln_beta, int32_t b_m,
+                       void* y, void* o_pre, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Integer decisions of the fused kernels, written through the same device
+ * functions they use, for exact comparison in tests.  For every sequence b and
+ * pair (i, j) of it, entry pair_offsets[b] + i*L_b + j (pair_offsets: device
+ * int64 [B+1], prefix sums of L_b^2) receives the mask bit, the rab_pos index
+ * and the rab_time bucket.  Meant for small batches. */
+HSTU_API int hstu_debug_indices(int32_t B, int32_t mask_kind, const int32_t* seq_offsets,
+                       const int64_t* timestamps, const int32_t* n_static, const int32_t* n_realtime,
+                       int32_t n_pos, int32_t n_tbuckets, const int64_t* pair_offsets,
+                       uint8_t* mask_bits, int16_t* pos_idx, int8_t* time_bucket, void* stream);
+
+/* Synchronizes `stream`, reads the device status word inside `workspace`,
+ * clears it and returns it as an hstu_status (HSTU_OK when clean). */
+HSTU_API int hstu_check_device_error(void* workspace, void* stream);
+
+/* Static English text for a status code. */
+HSTU_API const char* hstu_status_string(int status);
+
+/* Opt-in timing of the library's own kernel launches (off by default).
+ * hstu_profile_enable(1) clears the record and starts bracketing every kernel
+ * launch with two CUDA events on its stream; hstu_profile_enable(0) clears and
+ * stops.  hstu_profile_read() synchronizes on the recorded events and fills
+ * launches[k] and total_ms[k] for kernel kinds k < n_kinds (host arrays);
+ * it returns the number of kinds the library knows, or a negative status.
+ * hstu_profile_kind_name(k) names kind k ("" when out of range).  Meant for
+ * benchmarks: recording costs two event records per launch. */
+HSTU_API int hstu_profile_enable(int32_t on);
+HSTU_API int hstu_profile_read(int32_t n_kinds, int32_t* launches, double* total_ms);
+HSTU_API const char* hstu_profile_kind_name(int32_t kind);
+
+/* Library version, e.g. "0.1.0". */
+HSTU_API const char* hstu_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_B200_H */

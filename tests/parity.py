@@ -1,0 +1,101 @@
+"""Helpers shared by the GPU parity tests: tolerances, device copies, runners.
+
+Tolerances: bf16 path -- relative Frobenius error <= 5e-3 and max abs error <=
+3e-2 x RMS(reference); fp32 path -- relative Frobenius error <= 1e-5.  Integer
+work (offsets, masks, index decisions) is compared bit-exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+BF16_REL = 5e-3
+BF16_MAXABS_RMS = 3e-2
+F32_REL = 1e-5
+
+
+def _np(x):
+    if isinstance(x, torch.Tensor):
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def errors(got, ref):
+    g, r = _np(got), _np(ref)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    e = g - r
+    nr = float(np.linalg.norm(r))
+    rel = float(np.linalg.norm(e)) / nr if nr > 0 else float(np.linalg.norm(e))
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    mx = float(np.abs(e).max()) if e.size else 0.0
+    return rel, mx, rms
+
+
+def assert_bf16(got, ref, name):
+    rel, mx, rms = errors(got, ref)
+    assert np.all(np.isfinite(_np(got))), f"{name}: non-finite output"
+    assert rel <= BF16_REL, f"{name}: rel Frobenius {rel:.3e} > {BF16_REL}"
+    assert mx <= BF16_MAXABS_RMS * rms + 1e-30, f"{name}: max abs {mx:.3e} > {BF16_MAXABS_RMS} x RMS {rms:.3e}"
+    return rel, mx, rms
+
+
+def assert_f32(got, ref, name):
+    rel, mx, rms = errors(got, ref)
+    assert rel <= F32_REL, f"{name}: rel Frobenius {rel:.3e} > {F32_REL}"
+    return rel, mx, rms
+
+
+def assert_close(got, ref, name, dtype):
+    return assert_f32(got, ref, name) if dtype == torch.float32 else assert_bf16(got, ref, name)
+
+
+def dev(w, device="cuda"):
+    """Device copies of a workload's tensors (the GPU side of a parity check)."""
+    d = {}
+    for name in ("q", "k", "v", "u", "grad", "hist_k", "hist_v", "cand_q", "cand_k", "cand_v", "cand_u"):
+        t = getattr(w, name)
+        if t is not None:
+            d[name] = t.to(device).contiguous()
+    for name in ("rab_pos", "rab_time", "gamma", "beta"):
+        d[name] = getattr(w, name).to(device).contiguous()
+    for name in ("offsets", "hist_offsets", "cand_offsets", "n_static", "n_realtime"):
+        a = getattr(w, name)
+        if a is not None:
+            d[name] = torch.as_tensor(np.asarray(a, dtype=np.int32)).to(device)
+    for name in ("ts", "hist_ts", "cand_ts"):
+        a = getattr(w, name)
+        if a is not None:
+            d[name] = torch.as_tensor(np.asarray(a, dtype=np.int64)).to(device)
+    return d
+
+
+def run_layer(w, backward=False, device="cuda"):
+    from hstu_jagged_pointwise_b200 import ops
+    d = dev(w, device)
+    layer = ops.Layer(d["offsets"], d["ts"], w.H, w.d, w.dtype, w.alpha, max(w.max_len, 1),
+                      mask_kind=w.kind, n_static=d.get("n_static"), n_realtime=d.get("n_realtime"),
+                      n_pos=w.n_pos, n_tbuckets=w.n_tbuckets, ln_eps=w.eps)
+    fwd = layer.forward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"], d["beta"])
+    out = dict(fwd)
+    if backward:
+        out.update(layer.backward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"],
+                                  d["beta"], fwd, d["grad"]))
+    torch.cuda.synchronize()
+    st = layer.check_device_error()
+    assert st == 0, f"device status {st}"
+    return out, layer, d
+
+
+def run_mfalcon(w, b_m=None, device="cuda", d=None):
+    from hstu_jagged_pointwise_b200 import ops
+    d = d or dev(w, device)
+    lm = max(int(np.diff(w.hist_offsets).max()), 0)
+    lc = max(int(np.diff(w.cand_offsets).max()), 0)
+    m = ops.MFalcon(d["hist_offsets"], d["hist_ts"], d["cand_offsets"], d["cand_ts"], w.H, w.d, w.alpha,
+                    b_m or w.b_m, lm, lc, n_pos=w.n_pos, n_tbuckets=w.n_tbuckets, ln_eps=w.eps)
+    out = m.score(d["hist_k"], d["hist_v"], d["cand_q"], d["cand_k"], d["cand_v"], d["cand_u"], d["rab_pos"],
+                  d["rab_time"], d["gamma"], d["beta"])
+    torch.cuda.synchronize()
+    st = m.check_device_error()
+    assert st == 0, f"device status {st}"
+    return out, d

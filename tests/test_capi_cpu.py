@@ -1,0 +1,113 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports every
+symbol include/hstu.h declares, and rejects bad arguments before any launch."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+capi = pytest.importorskip("hstu_jagged_pointwise_b200.capi")
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "hstu.h")).read()
+    return sorted(set(re.findall(r"HSTU_API\s+[\w\s\*]+?\b(hstu_\w+)\s*\(", src)))
+
+
+def test_exports_match_header():
+    names = header_functions()
+    assert len(names) == 12, names
+    assert set(names) == set(capi.EXPORTS)
+    for n in names:
+        assert hasattr(capi.LIB, n), n
+
+
+def test_no_host_symbols_leak():
+    out = os.popen(f"nm -D --defined-only {capi.LIB_PATH}").read().split("\n")
+    exported = {l.split()[-1] for l in out if " T " in l}
+    assert exported == set(capi.EXPORTS), exported - set(capi.EXPORTS)
+
+
+def test_status_strings_and_version():
+    assert capi.LIB.hstu_version().decode() == "0.1.0"
+    for s in range(-6, 1):
+        assert capi.status_string(s) != "unknown status"
+    assert capi.status_string(-99) == "unknown status"
+
+
+def dims(**kw):
+    base = dict(B=4, T=436, H=2, d_qk=32, d_v=32, dtype=capi.HSTU_F32, n_pos=256, n_tbuckets=64,
+                max_seq_len=255, alpha=255.0, ln_eps=1e-5)
+    base.update(kw)
+    return capi.HstuDims(**base)
+
+
+def test_workspace_query():
+    d = dims()
+    n_f = capi.LIB.hstu_attn_workspace_bytes(C.byref(d), 0, 0)
+    n_b = capi.LIB.hstu_attn_workspace_bytes(C.byref(d), 0, 1)
+    assert n_f > 0 and n_b > n_f and n_f % 256 == 0
+    assert capi.LIB.hstu_attn_workspace_bytes(None, 0, 0) == 0
+    for bad in (dict(d_qk=48, d_v=48), dict(H=0), dict(alpha=0.0), dict(alpha=float("nan")),
+                dict(n_pos=0), dict(n_pos=1025), dict(n_tbuckets=65), dict(d_qk=32, d_v=64),
+                dict(dtype=7), dict(max_seq_len=-1)):
+        assert capi.LIB.hstu_attn_workspace_bytes(C.byref(dims(**bad)), 0, 0) == 0, bad
+    # bf16 supports 64 / 128 only
+    assert capi.LIB.hstu_attn_workspace_bytes(C.byref(dims(dtype=capi.HSTU_BF16)), 0, 0) == 0
+    assert capi.LIB.hstu_attn_workspace_bytes(C.byref(dims(dtype=capi.HSTU_BF16, d_qk=128, d_v=128)), 0, 0) > 0
+    assert capi.LIB.hstu_attn_workspace_bytes(C.byref(dims()), 5, 0) == 0
+
+
+def test_fwd_rejects_bad_arguments_before_launch():
+    d = dims()
+    m = capi.HstuMaskSpec(kind=0, n_static=None, n_realtime=None)
+    nulls = [None] * 15
+    # null dims / mask
+    assert capi.LIB.hstu_attn_fwd(None, C.byref(m), *nulls, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), None, *nulls, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    # unsupported width
+    d2 = dims(d_qk=48, d_v=48)
+    assert capi.LIB.hstu_attn_fwd(C.byref(d2), C.byref(m), *nulls, 0, None) == capi.HSTU_ERR_UNSUPPORTED
+    # MTGR without segment arrays
+    m2 = capi.HstuMaskSpec(kind=1, n_static=None, n_realtime=None)
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m2), *nulls, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    # missing / small / misaligned workspace
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m), *nulls, 0, None) == capi.HSTU_ERR_WORKSPACE
+    buf = (C.c_uint8 * 4096)()
+    base = C.addressof(buf)
+    aligned = (base + 255) // 256 * 256
+    args = [None] * 14 + [C.c_void_p(aligned)]
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m), *args, 16, None) == capi.HSTU_ERR_WORKSPACE
+    args = [None] * 14 + [C.c_void_p(aligned + 8)]
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m), *args, 2048, None) == capi.HSTU_ERR_WORKSPACE
+    # enough workspace but null tensors
+    args = [None] * 14 + [C.c_void_p(aligned)]
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m), *args, 2048, None) == capi.HSTU_ERR_INVALID_ARG
+    # T == 0 is a no-op
+    d0 = dims(B=0, T=0)
+    assert capi.LIB.hstu_attn_fwd(C.byref(d0), C.byref(m), *args, 2048, None) == capi.HSTU_OK
+
+
+def test_mfalcon_rejects_bad_arguments():
+    d = capi.HstuMfalconDims(B=2, T_hist=10, T_cand=4, H=2, d_qk=128, d_v=128, dtype=capi.HSTU_BF16,
+                             n_pos=256, n_tbuckets=64, max_hist_len=8, max_cand_len=4, alpha=9.0,
+                             ln_eps=1e-5)
+    assert capi.LIB.hstu_mfalcon_workspace_bytes(C.byref(d), 256) > 0
+    assert capi.LIB.hstu_mfalcon_workspace_bytes(C.byref(d), 0) == 0
+    nulls = [None] * 14
+    assert capi.LIB.hstu_mfalcon_score(C.byref(d), *nulls, 0, None, None, None, 0, None) == \
+        capi.HSTU_ERR_INVALID_ARG
+    d.dtype = capi.HSTU_F32
+    assert capi.LIB.hstu_mfalcon_score(C.byref(d), *nulls, 4, None, None, None, 0, None) == \
+        capi.HSTU_ERR_UNSUPPORTED
+
+
+def test_debug_indices_rejects_bad_arguments():
+    assert capi.LIB.hstu_debug_indices(1, 0, None, None, None, None, 256, 64, None, None, None, None,
+                                       None) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_debug_indices(1, 3, None, None, None, None, 256, 64, None, None, None, None,
+                                       None) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_debug_indices(0, 0, None, None, None, None, 256, 64, None, None, None, None,
+                                       None) == capi.HSTU_OK

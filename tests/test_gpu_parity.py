@@ -1,0 +1,280 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on the
+same seeded inputs.  Small cases are compared element by element; full-size
+workloads on sampled rows (sequences are independent, so the oracle computes
+only the sampled rows or sequences)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hstu_jagged_pointwise_b200 import workloads as W
+from parity import assert_bf16, assert_close, assert_f32, dev, run_layer, run_mfalcon
+
+pytestmark = pytest.mark.gpu
+
+
+# ----------------------------------------------------------------------------
+# integer decisions: bit-exact
+# ----------------------------------------------------------------------------
+
+def _boundary_ts():
+    return np.array([0, 1, 2, 3, 4, 7, 8, 15, 16, 3599, 3600, 4096, 2**31 - 1, 2**31, 2**40,
+                     2**62 - 1, 2**62, 2**62 + 5, 2**63 - 1], dtype=np.int64)
+
+
+def test_debug_indices_bit_exact():
+    from hstu_jagged_pointwise_b200 import ops
+    cases = []
+    # causal: lengths around the position clamp (254..256 apart) and boundary time deltas
+    ts_a = _boundary_ts()
+    ts_b = W.increasing_ts(np.random.default_rng(0), 300)
+    ts_c = np.array([-2**62, 0, 2**62], dtype=np.int64)
+    cases.append(("causal", [ts_a, ts_b, ts_c, np.array([5], np.int64)], None, None))
+    # MTGR: hand row, tie timestamps, all-static row, no real-time row
+    hand = np.array([0, 10, 20, 30, 40, 35, 15, 40], np.int64)
+    rng = np.random.default_rng(1)
+    u1 = W.mtgr_user(rng, 3, 40, 8, 6)
+    u2 = W.mtgr_user(rng, 2, 280, 0, 30)
+    u3 = W.mtgr_user(rng, 5, 20, 0, 0)
+    cases.append(("mtgr", [hand, u1, u2, u3], [3, 43, 282, 25], [2, 8, 0, 0]))
+    for kind, ts_list, ns, nr in cases:
+        lens = [len(t) for t in ts_list]
+        off = np.zeros(len(lens) + 1, np.int32)
+        off[1:] = np.cumsum(lens)
+        ts = np.concatenate(ts_list)
+        k = oracle.MASK_MTGR if kind == "mtgr" else oracle.MASK_CAUSAL
+        m0, p0, t0, _ = oracle.indices(off, ts, k, ns, nr)
+        dn = lambda a, dt: torch.as_tensor(np.asarray(a, dt)).cuda()
+        m1, p1, t1, _ = ops.debug_indices(dn(off, np.int32), dn(ts, np.int64), kind,
+                                          None if ns is None else dn(ns, np.int32),
+                                          None if nr is None else dn(nr, np.int32))
+        np.testing.assert_array_equal(m1.cpu().numpy(), m0)
+        np.testing.assert_array_equal(p1.cpu().numpy(), p0)
+        np.testing.assert_array_equal(t1.cpu().numpy(), t0)
+
+
+# ----------------------------------------------------------------------------
+# fp32 path (the tiny configuration): relative error <= 1e-5
+# ----------------------------------------------------------------------------
+
+def test_tiny_fp32_forward():
+    w = W.tiny_fp32(seed=0)
+    out, _, _ = run_layer(w)
+    y, o, mu, rs = oracle.layer_fwd(w)
+    assert_f32(out["y"], y, "y")
+    assert_f32(out["o_pre"], o, "o_pre")
+    assert_f32(out["mean"], mu, "mean")
+    assert_f32(out["rstd"], rs, "rstd")
+
+
+@pytest.mark.parametrize("kind", ["causal", "mtgr"])
+def test_fp32_backward(kind):
+    if kind == "causal":
+        w = W.make_causal([17, 64, 100, 255], H=2, d=32, dtype=torch.float32, seed=3, alpha=255.0,
+                          random_affine=True, with_grad=True)
+    else:
+        w = W.make_mtgr([4, 24], [30, 150], [5, 20], [7, 40], H=2, d=32, dtype=torch.float32, seed=4,
+                        random_affine=True, with_grad=True)
+    out, _, _ = run_layer(w, backward=True)
+    ref = oracle.layer_bwd(w)
+    assert_f32(out["y"], ref["y"], "y")
+    for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+        assert_f32(out[k], ref[k], k)
+    assert_f32(out["d_gamma"], ref["dgamma"], "d_gamma")
+    assert_f32(out["d_beta"], ref["dbeta"], "d_beta")
+
+
+# ----------------------------------------------------------------------------
+# bf16 tcgen05 forward: several tiles, ragged tails, empty and 1-token sequences
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_causal_forward_ragged(d):
+    w = W.make_causal([1, 127, 128, 129, 0, 300, 513, 2], H=2, d=d, seed=5)
+    out, _, _ = run_layer(w)
+    y, o, mu, rs = oracle.layer_fwd(w)
+    assert_bf16(out["y"], y, "y")
+    assert_bf16(out["o_pre"], o, "o_pre")
+
+
+def test_bf16_causal_forward_long_positions_and_times():
+    """Rows far from the diagonal (clamped position index) and huge time gaps."""
+    rng = np.random.default_rng(7)
+    ts = np.cumsum(rng.integers(1, 2**40, size=700)).astype(np.int64)
+    w = W.make_causal([700, 900], H=2, d=128, seed=6,
+                      ts_list=[ts, W.increasing_ts(rng, 900)])
+    out, _, _ = run_layer(w)
+    y, o, _, _ = oracle.layer_fwd(w)
+    assert_bf16(out["y"], y, "y")
+    assert_bf16(out["o_pre"], o, "o_pre")
+
+
+def test_bf16_mtgr_forward_small():
+    w = W.make_mtgr([24, 3, 24, 5], [40, 300, 150, 0], [8, 0, 64, 3], [6, 150, 20, 7], H=2, d=128,
+                    seed=8, alpha=500.0)
+    out, _, _ = run_layer(w)
+    y, o, _, _ = oracle.layer_fwd(w)
+    assert_bf16(out["y"], y, "y")
+    assert_bf16(out["o_pre"], o, "o_pre")
+
+
+@pytest.mark.parametrize("kind", ["causal", "mtgr"])
+def test_bf16_backward_small(kind):
+    if kind == "causal":
+        w = W.make_causal([1, 127, 129, 300], H=2, d=128, seed=9, random_affine=True, with_grad=True)
+    else:
+        w = W.make_mtgr([24, 2], [100, 190], [10, 0], [20, 70], H=2, d=128, seed=10, random_affine=True,
+                        with_grad=True)
+    out, _, _ = run_layer(w, backward=True)
+    ref = oracle.layer_bwd(w)
+    assert_bf16(out["y"], ref["y"], "y")
+    for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+        assert_bf16(out[k], ref[k], k)
+    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma")
+    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta")
+
+
+# ----------------------------------------------------------------------------
+# M-FALCON
+# ----------------------------------------------------------------------------
+
+def test_mfalcon_small_and_microbatch_invariance():
+    w = W.make_mfalcon([0, 1, 200, 300, 129], [3, 5, 130, 300, 1], H=2, d=128, seed=11, b_m=256,
+                       alpha=301.0)
+    y_ref, o_ref = oracle.mfalcon_layer(w)
+    out, d = run_mfalcon(w)
+    assert_bf16(out["y"], y_ref, "y")
+    assert_bf16(out["o_pre"], o_ref, "o_pre")
+    for bm in (1, 100, 128, 1000):
+        o2, _ = run_mfalcon(w, b_m=bm, d=d)
+        assert torch.equal(o2["y"], out["y"]), f"b_m={bm} changed the results"
+
+
+def test_mfalcon_permutation_equivariance():
+    w = W.make_mfalcon([400], [200], H=2, d=128, seed=12, alpha=401.0)
+    out, _ = run_mfalcon(w)
+    perm = np.random.default_rng(0).permutation(200)
+    pt = torch.as_tensor(perm)
+    for name in ("cand_q", "cand_k", "cand_v", "cand_u"):
+        setattr(w, name, getattr(w, name)[pt].contiguous())
+    w.cand_ts = w.cand_ts[perm]
+    out2, _ = run_mfalcon(w)
+    assert torch.equal(out2["y"], out["y"][pt.cuda()])
+
+
+# ----------------------------------------------------------------------------
+# the named workloads at full size
+# ----------------------------------------------------------------------------
+
+def test_training_sl_full_forward_backward():
+    w = W.training_sl(seed=0)
+    out, _, _ = run_layer(w, backward=True)
+    ref = oracle.layer_bwd(w)
+    _, o, _, _ = oracle.layer_fwd(w)
+    assert_bf16(out["y"], ref["y"], "y")
+    assert_bf16(out["o_pre"], o, "o_pre")
+    for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+        assert_bf16(out[k], ref[k], k)
+    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma")
+    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta")
+
+
+def _sample_rows(w, rng, per_seq=4, n_seq=12):
+    off = w.offsets
+    seqs = rng.choice(w.B, size=min(n_seq, w.B), replace=False)
+    rows = []
+    for b in seqs:
+        L = int(off[b + 1] - off[b])
+        if L == 0:
+            continue
+        picks = {0, L - 1} | set(rng.integers(0, L, size=per_seq).tolist())
+        rows += [int(off[b]) + i for i in sorted(picks)]
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def test_mtgr_medium_sampled_rows():
+    w = W.mtgr_medium(seed=0)
+    out, _, _ = run_layer(w)
+    rng = np.random.default_rng(2)
+    rows = _sample_rows(w, rng)
+    # make sure every segment kind is sampled: first real-time and candidate rows of a few users
+    extra = []
+    for b in range(6):
+        s0 = int(w.offsets[b])
+        S, R = int(w.n_static[b]), int(w.n_realtime[b])
+        extra += [s0 + S - 1, s0 + S, s0 + S + R, int(w.offsets[b + 1]) - 1]
+    rows = np.unique(np.concatenate([rows, np.array(extra, np.int64)]))
+    y, o, _, _ = oracle.layer_fwd(w, rows)
+    rt = torch.as_tensor(rows).cuda()
+    assert_bf16(out["y"][rt], y, "y")
+    assert_bf16(out["o_pre"][rt], o, "o_pre")
+
+
+def test_mfalcon_ranking_sampled_candidates():
+    w = W.mfalcon_ranking(seed=0)
+    out, _ = run_mfalcon(w)
+    rng = np.random.default_rng(3)
+    rows = np.unique(rng.integers(0, w.T, size=96)).astype(np.int64)
+    y, o = oracle.mfalcon_layer(w, rows)
+    rt = torch.as_tensor(rows).cuda()
+    assert_bf16(out["y"][rt], y, "y")
+    assert_bf16(out["o_pre"][rt], o, "o_pre")
+
+
+def _sub_workload(w, b):
+    """Sequence b of w alone (sequences are independent)."""
+    s0, s1 = int(w.offsets[b]), int(w.offsets[b + 1])
+    ws = W.make_causal([s1 - s0], H=w.H, d=w.d, dtype=w.dtype, seed=0, alpha=w.alpha,
+                       ts_list=[w.ts[s0:s1]], with_grad=True)
+    for name in ("q", "k", "v", "u", "grad"):
+        setattr(ws, name, getattr(w, name)[s0:s1])
+    ws.rab_pos, ws.rab_time, ws.gamma, ws.beta = w.rab_pos, w.rab_time, w.gamma, w.beta
+    return ws, s0, s1
+
+
+def test_large_layer_sampled_forward_and_per_sequence_backward():
+    w = W.large_layer(seed=0)
+    out, _, _ = run_layer(w, backward=True)
+    rng = np.random.default_rng(4)
+    rows = _sample_rows(w, rng, per_seq=3, n_seq=10)
+    y, o, _, _ = oracle.layer_fwd(w, rows)
+    rt = torch.as_tensor(rows).cuda()
+    assert_bf16(out["y"][rt], y, "y")
+    assert_bf16(out["o_pre"][rt], o, "o_pre")
+    # full backward of two whole sequences (the shortest and one near 1000 tokens)
+    L = w.lengths
+    picks = [int(np.argmin(L)), int(np.argmin(np.abs(L - 1000)))]
+    for b in picks:
+        ws, s0, s1 = _sub_workload(w, b)
+        ref = oracle.layer_bwd(ws)
+        for k in ("dq", "dk", "dv", "du"):
+            assert_bf16(out[k][s0:s1], ref[k], f"{k}[seq {b}]")
+
+
+# ----------------------------------------------------------------------------
+# device-side validation and error status
+# ----------------------------------------------------------------------------
+
+def test_invalid_offsets_set_device_status_and_recover():
+    from hstu_jagged_pointwise_b200 import capi
+    w = W.make_causal([100, 50], H=2, d=128, seed=13)
+    out, layer, d = run_layer(w)
+    bad = torch.tensor([0, 120, 150], dtype=torch.int32, device="cuda")   # length 120 > max 100
+    layer.seq_offsets.copy_(bad)
+    layer.forward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"], d["beta"])
+    assert layer.check_device_error() == capi.HSTU_ERR_DEVICE_BOUNDS
+    assert layer.check_device_error() == capi.HSTU_OK          # cleared
+    layer.seq_offsets.copy_(torch.tensor([0, 100, 150], dtype=torch.int32, device="cuda"))
+    out2 = layer.forward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"], d["beta"])
+    torch.cuda.synchronize()
+    assert layer.check_device_error() == capi.HSTU_OK
+    assert torch.equal(out2["y"], out["y"])
+
+
+def test_mtgr_bad_segments_flagged():
+    from hstu_jagged_pointwise_b200 import capi
+    w = W.make_mtgr([2], [10], [3], [4], H=2, d=128, seed=14)
+    out, layer, d = run_layer(w)
+    layer.n_static.fill_(30)       # static + real-time longer than the row
+    layer.forward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"], d["beta"])
+    assert layer.check_device_error() == capi.HSTU_ERR_DEVICE_BOUNDS
