@@ -207,7 +207,7 @@ def time_oracle(sample):
 def run_ours(args, world, rank, local):
     from hstu_jagged_pointwise_b200 import capi, ops
 
-    w = W.large_layer(seed=args.seed + rank)
+    w = W.large_layer(seed=args.seed + rank, total=args.tokens)
     dev = torch.device("cuda", local)
     H, d = w.H, w.d
     P_head = causal_pairs(w.lengths)
@@ -277,6 +277,8 @@ def run_ours(args, world, rank, local):
     ms_fwd = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
 
     # ---- end to end through the C ABI with host buffers
+    if args.no_e2e:
+        return finish(args, world, w, kernels, ms, ms_max, ms_fwd, None, None, None, None, clocks, f_fwd, f_bwd, P, d)
     pin = {n: t.pin_memory() for n, t in host.items()}
     small_in = {n: t.pin_memory() for n, t in (("rp", w.rab_pos), ("rt", w.rab_time), ("g", w.gamma),
                                                 ("b", w.beta))}
@@ -318,7 +320,11 @@ def run_ours(args, world, rank, local):
     if not args.no_mfalcon:
         del pin, outs_h
         mf = run_mfalcon(args, world, rank, local)
+    return finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d)
 
+
+def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d):
+    H = w.H
     # ---- roofline of the dominant kernel
     pk, pk_src = peaks()
     sm_mhz = pk.get("sm_max_mhz", 1965.0)
@@ -370,8 +376,9 @@ def run_ours(args, world, rank, local):
         "fwd_tflops": round(fwd_tflops, 3),
         "pct_bf16_peak_fwd": round(fwd_tflops / world / pk["bf16_tflops_sustained"], 4),
         "peak_source": pk_src,
-        "e2e": {"value": round(world * flops_step / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "e2e": None if ms_e2e is None else {
+            "value": round(world * flops_step / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches_total),
         "roofline": roof,
         "kernels": kinfo,
@@ -430,7 +437,7 @@ def run_mfalcon(args, world, rank, local):
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    w = W.large_layer(seed=args.seed)
+    w = W.large_layer(seed=args.seed, total=args.tokens)
     sample, seqs = oracle_sample(w, target_s=max(5.0, 60.0 / max(args.steps + args.warmup, 1)))
     for _ in range(args.warmup):
         time_oracle(sample)
@@ -463,6 +470,9 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-mfalcon", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--tokens", type=int, default=262144,
+                    help="total tokens of the large-layer workload (smaller values for profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

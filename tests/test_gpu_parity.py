@@ -8,7 +8,8 @@ import torch
 
 import oracle
 from hstu_jagged_pointwise_b200 import workloads as W
-from parity import assert_bf16, assert_close, assert_f32, dev, run_layer, run_mfalcon
+from parity import (assert_bf16, assert_f32, run_layer, run_mfalcon, storage_bwd, storage_fwd,
+                    storage_mfalcon)
 
 pytestmark = pytest.mark.gpu
 
@@ -93,8 +94,9 @@ def test_bf16_causal_forward_ragged(d):
     w = W.make_causal([1, 127, 128, 129, 0, 300, 513, 2], H=2, d=d, seed=5)
     out, _, _ = run_layer(w)
     y, o, mu, rs = oracle.layer_fwd(w)
-    assert_bf16(out["y"], y, "y")
-    assert_bf16(out["o_pre"], o, "o_pre")
+    st = storage_fwd(w)
+    assert_bf16(out["y"], y, "y", st["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", st["o_pre"])
 
 
 def test_bf16_causal_forward_long_positions_and_times():
@@ -105,8 +107,9 @@ def test_bf16_causal_forward_long_positions_and_times():
                       ts_list=[ts, W.increasing_ts(rng, 900)])
     out, _, _ = run_layer(w)
     y, o, _, _ = oracle.layer_fwd(w)
-    assert_bf16(out["y"], y, "y")
-    assert_bf16(out["o_pre"], o, "o_pre")
+    st = storage_fwd(w)
+    assert_bf16(out["y"], y, "y", st["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", st["o_pre"])
 
 
 def test_bf16_mtgr_forward_small():
@@ -114,8 +117,9 @@ def test_bf16_mtgr_forward_small():
                     seed=8, alpha=500.0)
     out, _, _ = run_layer(w)
     y, o, _, _ = oracle.layer_fwd(w)
-    assert_bf16(out["y"], y, "y")
-    assert_bf16(out["o_pre"], o, "o_pre")
+    st = storage_fwd(w)
+    assert_bf16(out["y"], y, "y", st["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", st["o_pre"])
 
 
 @pytest.mark.parametrize("kind", ["causal", "mtgr"])
@@ -127,11 +131,12 @@ def test_bf16_backward_small(kind):
                         with_grad=True)
     out, _, _ = run_layer(w, backward=True)
     ref = oracle.layer_bwd(w)
-    assert_bf16(out["y"], ref["y"], "y")
+    st = storage_bwd(w)
+    assert_bf16(out["y"], ref["y"], "y", st["y"])
     for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
-        assert_bf16(out[k], ref[k], k)
-    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma")
-    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta")
+        assert_bf16(out[k], ref[k], k, st[k])
+    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma", st["dgamma"])
+    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta", st["dbeta"])
 
 
 # ----------------------------------------------------------------------------
@@ -142,9 +147,10 @@ def test_mfalcon_small_and_microbatch_invariance():
     w = W.make_mfalcon([0, 1, 200, 300, 129], [3, 5, 130, 300, 1], H=2, d=128, seed=11, b_m=256,
                        alpha=301.0)
     y_ref, o_ref = oracle.mfalcon_layer(w)
+    st = storage_mfalcon(w)
     out, d = run_mfalcon(w)
-    assert_bf16(out["y"], y_ref, "y")
-    assert_bf16(out["o_pre"], o_ref, "o_pre")
+    assert_bf16(out["y"], y_ref, "y", st["y"])
+    assert_bf16(out["o_pre"], o_ref, "o_pre", st["o_pre"])
     for bm in (1, 100, 128, 1000):
         o2, _ = run_mfalcon(w, b_m=bm, d=d)
         assert torch.equal(o2["y"], out["y"]), f"b_m={bm} changed the results"
@@ -171,12 +177,14 @@ def test_training_sl_full_forward_backward():
     out, _, _ = run_layer(w, backward=True)
     ref = oracle.layer_bwd(w)
     _, o, _, _ = oracle.layer_fwd(w)
-    assert_bf16(out["y"], ref["y"], "y")
-    assert_bf16(out["o_pre"], o, "o_pre")
+    st = storage_bwd(w)
+    sf = storage_fwd(w)
+    assert_bf16(out["y"], ref["y"], "y", st["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", sf["o_pre"])
     for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
-        assert_bf16(out[k], ref[k], k)
-    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma")
-    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta")
+        assert_bf16(out[k], ref[k], k, st[k])
+    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma", st["dgamma"])
+    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta", st["dbeta"])
 
 
 def _sample_rows(w, rng, per_seq=4, n_seq=12):
@@ -205,9 +213,10 @@ def test_mtgr_medium_sampled_rows():
         extra += [s0 + S - 1, s0 + S, s0 + S + R, int(w.offsets[b + 1]) - 1]
     rows = np.unique(np.concatenate([rows, np.array(extra, np.int64)]))
     y, o, _, _ = oracle.layer_fwd(w, rows)
+    st = storage_fwd(w, rows)
     rt = torch.as_tensor(rows).cuda()
-    assert_bf16(out["y"][rt], y, "y")
-    assert_bf16(out["o_pre"][rt], o, "o_pre")
+    assert_bf16(out["y"][rt], y, "y", st["y"])
+    assert_bf16(out["o_pre"][rt], o, "o_pre", st["o_pre"])
 
 
 def test_mfalcon_ranking_sampled_candidates():
@@ -216,9 +225,10 @@ def test_mfalcon_ranking_sampled_candidates():
     rng = np.random.default_rng(3)
     rows = np.unique(rng.integers(0, w.T, size=96)).astype(np.int64)
     y, o = oracle.mfalcon_layer(w, rows)
+    st = storage_mfalcon(w, rows)
     rt = torch.as_tensor(rows).cuda()
-    assert_bf16(out["y"][rt], y, "y")
-    assert_bf16(out["o_pre"][rt], o, "o_pre")
+    assert_bf16(out["y"][rt], y, "y", st["y"])
+    assert_bf16(out["o_pre"][rt], o, "o_pre", st["o_pre"])
 
 
 def _sub_workload(w, b):
@@ -238,17 +248,19 @@ def test_large_layer_sampled_forward_and_per_sequence_backward():
     rng = np.random.default_rng(4)
     rows = _sample_rows(w, rng, per_seq=3, n_seq=10)
     y, o, _, _ = oracle.layer_fwd(w, rows)
+    st = storage_fwd(w, rows)
     rt = torch.as_tensor(rows).cuda()
-    assert_bf16(out["y"][rt], y, "y")
-    assert_bf16(out["o_pre"][rt], o, "o_pre")
+    assert_bf16(out["y"][rt], y, "y", st["y"])
+    assert_bf16(out["o_pre"][rt], o, "o_pre", st["o_pre"])
     # full backward of two whole sequences (the shortest and one near 1000 tokens)
     L = w.lengths
     picks = [int(np.argmin(L)), int(np.argmin(np.abs(L - 1000)))]
     for b in picks:
         ws, s0, s1 = _sub_workload(w, b)
         ref = oracle.layer_bwd(ws)
+        st = storage_bwd(ws)
         for k in ("dq", "dk", "dv", "du"):
-            assert_bf16(out[k][s0:s1], ref[k], f"{k}[seq {b}]")
+            assert_bf16(out[k][s0:s1], ref[k], f"{k}[seq {b}]", st[k])
 
 
 # ----------------------------------------------------------------------------
