@@ -334,6 +334,7 @@ def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, cl
         "attn_bwd_dkv_simt_kernel": ("alu", 6 * d * P, "TFLOP/s"),
         "attn_bwd_dq_simt_kernel": ("alu", 2 * d * P, "TFLOP/s"),
         "attn_bwd_tc_kernel": ("tensor", f_bwd, "TFLOP/s"),
+        "dq_convert_kernel": ("hbm", 6 * w.D * w.T, "GB/s"),
         "ln_fwd_kernel": ("hbm", (6 * w.D + 8) * w.T, "GB/s"),
         "ln_bwd_kernel": ("hbm", (10 * w.D + 8) * w.T, "GB/s"),
     }

@@ -1,0 +1,657 @@
+// attn_bwd_tc.cu -- fused jagged HSTU pointwise attention backward on tcgen05 (sm_100a).
+//
+// The derivative of Y = (1/alpha) sum_j mask * SiLU(z_ij) v_j with
+// z_ij = q_i.k_j + rab_pos[pidx] + rab_time[tb] (Meta HSTU blog, sections 3,
+// 3.1 and 3.2; the pages give no backward formulas):
+//   dA_ij = dy_i . v_j / alpha,  dz_ij = mask * dA_ij * SiLU'(z_ij),
+//   SiLU'(z) = sig + SiLU(z) (1 - sig),  sig = sigmoid(z) = (1 + tanh(z/2)) / 2,
+//   dV_j = sum_i (mask * SiLU(z_ij) / alpha) dy_i,  dK_j = sum_i dz_ij q_i,
+//   dQ_i = sum_j dz_ij k_j,  d_rab_pos[p] / d_rab_time[t] = sum of dz over the pairs using p / t.
+// A = SiLU(z) is recomputed from Q and K, never read from memory.
+//
+// One work item = (sequence, head, 128-key tile); the CTA loops over the
+// 128-query tiles that see the key tile.  Per query tile, five UMMAs:
+//   S^T  = K Q^T   -> TMEM [0,128)        (SS, both K-major)
+//   dP^T = V dY^T  -> TMEM [128,256)      (SS, both K-major)
+//   elementwise warps: bias, mask, sigmoid, A^T (bf16) -> TMEM over S^T,
+//                      dZ^T (bf16) -> shared memory (128-byte swizzle)
+//   dV  += A^T dY  -> TMEM [256,256+D)    (TS: A^T from TMEM, dY MN-major)
+//   dK  += dZ^T Q  -> TMEM [256+D,256+2D) (SS: dZ^T K-major, Q MN-major)
+//   dQ   = dZ K    -> TMEM [128,128+D)    (SS: dZ^T read MN-major, K MN-major),
+//          drained by the elementwise warps into an fp32 buffer with vector reductions.
+// Warps 0-7 elementwise (warp w owns TMEM lanes 32*(w%4)..+31 = key rows, and
+// query columns [64*(w/4), +64)), warp 8 producer (TMA), warp 9 MMA issuer.
+// rab gradients: shared-memory accumulators (run-length per thread for the time
+// bucket, one atomic per element for the position index, or a warp sum when the
+// bias is uniform over the warp's block), flushed to global memory at the end.
+// Every wait is bounded; a timeout sets the status word and the CTA exits cleanly.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hstu {
+namespace {
+
+using namespace ptx;
+
+template <int D>
+struct BwdSmem {
+    static constexpr uint32_t kTile = 128u * D * 2u;            // one 128-row bf16 tile
+    static constexpr uint32_t k = 0;
+    static constexpr uint32_t v = k + kTile;
+    static constexpr uint32_t q0 = v + kTile;
+    static constexpr uint32_t q1 = q0 + kTile;
+    static constexpr uint32_t dy = q1 + kTile;
+    static constexpr uint32_t dz = dy + kTile;                   // 128 keys x 128 queries bf16
+    static constexpr uint32_t rp = dz + 128u * 128u * 2u;        // float[2*kMaxPos]
+    static constexpr uint32_t rt = rp + 2u * kMaxPos * 4u;       // float[64]
+    static constexpr uint32_t grp = rt + kMaxTBuckets * 4u;      // float[2*kMaxPos]
+    static constexpr uint32_t grt = grp + 2u * kMaxPos * 4u;     // float[64]
+    static constexpr uint32_t qts = grt + kMaxTBuckets * 4u;     // int64[8 warps][64]
+    static constexpr uint32_t item = qts + 8u * 64u * 8u;        // int4[2]
+    static constexpr uint32_t bars = item + 2u * 16u;            // uint64[24]
+    static constexpr uint32_t tmem = bars + 24u * 8u;
+    static constexpr uint32_t abort_flag = tmem + 4u;
+    static constexpr uint32_t bytes = abort_flag + 4u;
+    static constexpr uint32_t alloc = bytes + 1024u;
+};
+
+enum {
+    kKVFull = 0, kKVEmpty, kQFull0, kQFull1, kQEmpty0, kQEmpty1, kDYFull, kDYEmpty, kSFull, kPFull,
+    kDQFull, kDQDrained, kDZEmpty, kAccFull, kAccEmpty, kItFull0, kItFull1, kItEmpty0, kItEmpty1,
+    kDrain, kNumBars
+};
+
+constexpr int kThreads = 320;
+constexpr int kEwThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCol = 0;
+constexpr uint32_t kPCol = 128;
+constexpr uint32_t kVCol = 256;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr uint32_t kPanel = 128u * 128u;                         // 128 rows x 128 B
+
+struct KvItem {
+    int b, n0, h, n_end;   // keys [n0, n_end) of sequence b, head h
+    int off0, L, S, R;
+};
+
+template <int KIND>
+__device__ __forceinline__ KvItem load_kv_item(const BwdParams& p, int4 it) {
+    KvItem s;
+    s.b = it.x; s.n0 = it.y; s.h = it.z; s.n_end = it.w;
+    s.off0 = p.off[s.b];
+    s.L = p.off[s.b + 1] - s.off0;
+    if (KIND == HSTU_KIND_MTGR) {
+        s.S = p.n_static[s.b];
+        s.R = p.n_rt[s.b];
+    } else {
+        s.S = s.L;
+        s.R = 0;
+    }
+    return s;
+}
+
+// does query tile t see any key of this item?
+template <int KIND>
+__device__ __forceinline__ int q_class(const KvItem& s, int t) {
+    const int qa = t * kTileM;
+    const int qb = min(qa + kTileM - 1, s.L - 1);
+    return tile_class(KIND, qa, qb, s.n0, s.n_end - 1, s.S, s.R);
+}
+
+__device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicOr(&p.ctrl->status, kStatusTimeout);
+}
+
+template <int KIND, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dy,
+                   const BwdParams p) {
+    using L = BwdSmem<D>;
+    constexpr int kPanels = D / 64;
+    constexpr uint32_t kKCol = kVCol + D;
+    constexpr uint32_t kIdSS = idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T
+    constexpr uint32_t kIdTS = idesc_bf16_f32(128, D, 0, 1);      // dV: A tmem, B MN-major
+    constexpr uint32_t kIdKM = idesc_bf16_f32(128, D, 0, 1);      // dK: A K-major, B MN-major
+    constexpr uint32_t kIdMM = idesc_bf16_f32(128, D, 1, 1);      // dQ: A MN-major, B MN-major
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    float* s_rp = reinterpret_cast<float*>(sm + L::rp);
+    float* s_rt = reinterpret_cast<float*>(sm + L::rt);
+    float* s_grp = reinterpret_cast<float*>(sm + L::grp);
+    float* s_grt = reinterpret_cast<float*>(sm + L::grt);
+    int64_t* s_qts = reinterpret_cast<int64_t*>(sm + L::qts);
+    int4* s_item = reinterpret_cast<int4*>(sm + L::item);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::tmem);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::abort_flag);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int np = 2 * p.P - 1;
+    for (int i = tid; i < np; i += kThreads) {
+        s_rp[i] = p.rab_pos[i];
+        s_grp[i] = 0.f;
+    }
+    for (int i = tid; i < p.nb; i += kThreads) {
+        s_rt[i] = p.rab_time[i];
+        s_grt[i] = 0.f;
+    }
+    if (tid == 0) {
+        const uint32_t counts[kNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, kEwThreads, 1, kEwThreads, 1, 1,
+                                           kEwThreads, 1, 1, kEwThreads + 1, kEwThreads + 1, 1};
+        for (int i = 0; i < kNumBars; i++) mbar_init(&bars[i], counts[i]);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_dy);
+    }
+    if (warp == 9) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 8) {
+        // ============================================================ producer
+        int it_use = 0, kv_use = 0, q_use = 0, dy_use = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = it_use & 1;
+            if (lane == 0) {
+                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort);
+                if (ok) {
+                    const int idx = atomicAdd(&p.ctrl->counter, 1);
+                    s_item[slot] = idx < p.ctrl->n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
+                    mbar_arrive(&bars[kItFull0 + slot]);
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+            if (!ok) break;
+            int4 it = s_item[slot];
+            it.x = __shfl_sync(kFull, it.x, 0);
+            it.y = __shfl_sync(kFull, it.y, 0);
+            it.z = __shfl_sync(kFull, it.z, 0);
+            it.w = __shfl_sync(kFull, it.w, 0);
+            it_use++;
+            if (it.x < 0) break;
+            if (lane == 0) {
+                const KvItem s = load_kv_item<KIND>(p, it);
+                ok = mbar_wait(&bars[kKVEmpty], (kv_use & 1) ^ 1, s_abort);
+                if (ok) {
+                    mbar_arrive_expect_tx(&bars[kKVFull], 2 * L::kTile);
+                    for (int pn = 0; pn < kPanels; pn++) {
+                        tma_load_2d(sm + L::k + pn * kPanel, &tm_k, &bars[kKVFull], s.h * D + pn * 64,
+                                    s.off0 + s.n0);
+                        tma_load_2d(sm + L::v + pn * kPanel, &tm_v, &bars[kKVFull], s.h * D + pn * 64,
+                                    s.off0 + s.n0);
+                    }
+                    kv_use++;
+                }
+                const int n_qt = (s.L + kTileM - 1) / kTileM;
+                for (int t = 0; ok && t < n_qt; t++) {
+                    if (q_class<KIND>(s, t) == 0) continue;
+                    const int st = q_use & 1;
+                    ok = mbar_wait(&bars[kQEmpty0 + st], ((q_use >> 1) & 1) ^ 1, s_abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars[kQFull0 + st], L::kTile);
+                    for (int pn = 0; pn < kPanels; pn++)
+                        tma_load_2d(sm + (st ? L::q1 : L::q0) + pn * kPanel, &tm_q, &bars[kQFull0 + st],
+                                    s.h * D + pn * 64, s.off0 + t * kTileM);
+                    q_use++;
+                    ok = mbar_wait(&bars[kDYEmpty], (dy_use & 1) ^ 1, s_abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars[kDYFull], L::kTile);
+                    for (int pn = 0; pn < kPanels; pn++)
+                        tma_load_2d(sm + L::dy + pn * kPanel, &tm_dy, &bars[kDYFull], s.h * D + pn * 64,
+                                    s.off0 + t * kTileM);
+                    dy_use++;
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+        }
+        if (lane == 0) {
+            if (!ok && !*s_abort) flag_timeout(p, s_abort);
+            if (*s_abort) {
+                volatile int dummy = 0;
+                if (kv_use) mbar_wait(&bars[kKVFull], (kv_use - 1) & 1, &dummy);
+                if (q_use) {
+                    const int st = (q_use - 1) & 1;
+                    mbar_wait(&bars[kQFull0 + st], ((q_use - 1) >> 1) & 1, &dummy);
+                }
+                if (q_use > 1) {
+                    const int st = (q_use - 2) & 1;
+                    mbar_wait(&bars[kQFull0 + st], ((q_use - 2) >> 1) & 1, &dummy);
+                }
+                if (dy_use) mbar_wait(&bars[kDYFull], (dy_use - 1) & 1, &dummy);
+            }
+        }
+    } else if (warp == 9) {
+        // ============================================================ MMA issuer
+        int it_use = 0, kv_use = 0, q_use = 0, dy_use = 0, p_use = 0, dq_use = 0, acc_use = 0;
+        bool ok = true;
+        const uint32_t aK = smem_u32(sm + L::k), aV = smem_u32(sm + L::v);
+        const uint32_t aQ0 = smem_u32(sm + L::q0), aQ1 = smem_u32(sm + L::q1);
+        const uint32_t aDY = smem_u32(sm + L::dy), aDZ = smem_u32(sm + L::dz);
+        while (ok) {
+            const int slot = it_use & 1;
+            int4 it = make_int4(-1, 0, 0, 0);
+            if (lane == 0) {
+                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+                if (ok) it = s_item[slot];
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+            if (!ok) break;
+            it.x = __shfl_sync(kFull, it.x, 0);
+            it_use++;
+            if (it.x < 0) break;
+            if (lane == 0) {
+                const KvItem s = load_kv_item<KIND>(p, it);
+                const int n_qt = (s.L + kTileM - 1) / kTileM;
+                int last = -1;
+                for (int t = 0; t < n_qt; t++)
+                    if (q_class<KIND>(s, t) != 0) last = t;
+                ok = mbar_wait(&bars[kKVFull], kv_use & 1, s_abort);
+                kv_use++;
+                int n_done = 0;
+                for (int t = 0; ok && t <= last; t++) {
+                    if (q_class<KIND>(s, t) == 0) continue;
+                    const int st = q_use & 1;
+                    const uint32_t aQ = st ? aQ1 : aQ0;
+                    ok = mbar_wait(&bars[kQFull0 + st], (q_use >> 1) & 1, s_abort);
+                    if (!ok) break;
+                    q_use++;
+                    tc_fence_after();
+                    // S^T = K Q^T
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; kk++) {
+                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                        mma_ss(tmem + kSCol, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(aQ + off, 16, 1024),
+                               kIdSS, kk > 0 ? 1u : 0u);
+                    }
+                    ok = mbar_wait(&bars[kDYFull], dy_use & 1, s_abort);
+                    if (!ok) break;
+                    dy_use++;
+                    // dQ of the previous tile lives in the dP^T columns until drained
+                    ok = mbar_wait(&bars[kDQDrained], (dq_use & 1) ^ 1, s_abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // dP^T = V dY^T
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; kk++) {
+                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                        mma_ss(tmem + kPCol, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(aDY + off, 16, 1024),
+                               kIdSS, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bars[kSFull]);
+                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort);
+                    if (!ok) break;
+                    p_use++;
+                    if (n_done == 0) {
+                        ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    // dV += A^T dY   (A^T from TMEM: queries 64g..64g+63 at columns 64g..64g+31)
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++) {
+                        const uint32_t acol = kSCol + 64 * (kk >> 2) + 8 * (kk & 3);
+                        mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY + kk * 2048, kPanel, 1024), kIdTS,
+                               (n_done > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&bars[kDYEmpty]);
+                    // dK += dZ^T Q
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++) {
+                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                        mma_ss(tmem + kKCol, sdesc_sw128(aDZ + off, 16, 1024),
+                               sdesc_sw128(aQ + kk * 2048, kPanel, 1024), kIdKM, (n_done > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&bars[kQEmpty0 + st]);
+                    // dQ = dZ K   (dZ^T read MN-major, K read MN-major)
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++) {
+                        mma_ss(tmem + kPCol, sdesc_sw128(aDZ + kk * 2048, kPanel, 1024),
+                               sdesc_sw128(aK + kk * 2048, kPanel, 1024), kIdMM, kk > 0 ? 1u : 0u);
+                    }
+                    dq_use++;
+                    tc_commit(&bars[kDZEmpty]);
+                    tc_commit(&bars[kDQFull]);
+                    if (t == last) tc_commit(&bars[kKVEmpty]);
+                    n_done++;
+                }
+                if (ok && n_done == 0) {
+                    tc_commit(&bars[kKVEmpty]);
+                    ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
+                }
+                if (ok) {
+                    acc_use++;
+                    tc_commit(&bars[kAccFull]);
+                    mbar_arrive(&bars[kItEmpty0 + slot]);
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+        }
+        if (lane == 0) {
+            if (!ok && !*s_abort) flag_timeout(p, s_abort);
+            volatile int dummy = 0;
+            tc_commit(&bars[kDrain]);
+            mbar_wait(&bars[kDrain], 0, &dummy);
+        }
+    } else {
+        // ============================================================ elementwise (warps 0-7)
+        const int wq = warp & 3;                 // lane quarter: key rows 32*wq .. +31
+        const int g = warp >> 2;                 // query half: columns 64*g .. +63
+        const int r = wq * 32 + lane;            // key row within the tile (TMEM lane)
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        const uint32_t aDZ = smem_u32(sm + L::dz);
+        int64_t* w_qts = s_qts + warp * 64;
+        int it_use = 0, s_use = 0, dz_use = 0, dq_use = 0, acc_use = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = it_use & 1;
+            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+            if (!__all_sync(kFull, ok)) { ok = false; break; }
+            const int4 it = s_item[slot];
+            it_use++;
+            if (it.x < 0) break;
+            const KvItem s = load_kv_item<KIND>(p, it);
+            const int j = s.n0 + r;
+            const bool key_ok = j < s.n_end;
+            const int jc = min(j, s.n_end - 1);
+            const int64_t ts_j = p.ts[s.off0 + jc];
+            const int pos_j = token_pos(KIND, jc, s.S, s.R);
+            int64_t kmin = key_ok ? ts_j : INT64_MAX, kmax = key_ok ? ts_j : INT64_MIN;
+            int pk_lo = key_ok ? pos_j : INT32_MAX, pk_hi = key_ok ? pos_j : INT32_MIN;
+            int warp_keys = key_ok ? 1 : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                kmin = min(kmin, (int64_t)__shfl_xor_sync(kFull, (long long)kmin, o));
+                kmax = max(kmax, (int64_t)__shfl_xor_sync(kFull, (long long)kmax, o));
+                pk_lo = min(pk_lo, __shfl_xor_sync(kFull, pk_lo, o));
+                pk_hi = max(pk_hi, __shfl_xor_sync(kFull, pk_hi, o));
+                warp_keys += __shfl_xor_sync(kFull, warp_keys, o);
+            }
+            const int n_qt = (s.L + kTileM - 1) / kTileM;
+            int n_done = 0;
+            for (int t = 0; t < n_qt; t++) {
+                const int cls = q_class<KIND>(s, t);
+                if (cls == 0) continue;
+                const int i0 = t * kTileM + 64 * g;       // first query of this warp's columns
+                __syncwarp();
+                int64_t qmin = INT64_MAX, qmax = INT64_MIN;
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    const int ii = lane + 32 * e;
+                    const int i = i0 + ii;
+                    const int64_t ti = i < s.L ? p.ts[s.off0 + i] : 0;
+                    w_qts[ii] = ti;
+                    if (i < s.L) {
+                        qmin = min(qmin, ti);
+                        qmax = max(qmax, ti);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
+                    qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
+                }
+                __syncwarp();
+                // uniform bias and full visibility over this warp's 32 keys x 64 queries?
+                bool fast = false;
+                int pidx_u = 0, tb_u = 0;
+                float cbias = 0.f;
+                if (warp_keys == 32 && i0 + 64 <= s.L) {
+                    const int ka = s.n0 + 32 * wq;
+                    fast = tile_class(KIND, i0, i0 + 63, ka, ka + 31, s.S, s.R) == 2;
+                    if (fast) {
+                        const int pq_lo = token_pos(KIND, i0, s.S, s.R);
+                        const int pq_hi = token_pos(KIND, i0 + 63, s.S, s.R);
+                        const int dmax = pk_hi - pq_lo, dmin = pk_lo - pq_hi;
+                        pidx_u = -1;
+                        if (dmax <= -(p.P - 1)) pidx_u = 0;
+                        else if (dmin >= p.P - 1) pidx_u = 2 * p.P - 2;
+                        uint64_t lo;
+                        if (qmin > kmax) lo = abs_diff_u64(qmin, kmax);
+                        else if (kmin > qmax) lo = abs_diff_u64(kmin, qmax);
+                        else lo = 0;
+                        const uint64_t hi = max(abs_diff_u64(qmax, kmin), abs_diff_u64(kmax, qmin));
+                        tb_u = time_bucket_of_delta(lo, p.nb);
+                        fast = pidx_u >= 0 && tb_u == time_bucket_of_delta(hi, p.nb);
+                        if (fast) cbias = s_rp[pidx_u] + s_rt[tb_u];
+                    }
+                }
+                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
+                if (ok) ok = mbar_wait(&bars[kDZEmpty], (dz_use & 1) ^ 1, s_abort);
+                if (!__all_sync(kFull, ok)) { ok = false; break; }
+                s_use++;
+                dz_use++;
+                tc_fence_after();
+                float fast_sum = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 2; c++) {
+                    uint32_t sv[32], dp[32];
+                    tmem_ld32(tmem + lane_base + kSCol + 64 * g + 32 * c, sv);
+                    tmem_ld32(tmem + lane_base + kPCol + 64 * g + 32 * c, dp);
+                    tmem_ld_wait(sv);
+                    tmem_ld_wait(dp);
+                    uint32_t pa[16], pz[16];
+                    if (fast) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float av[2], zv[2];
+#pragma unroll
+                            for (int f = 0; f < 2; f++) {
+                                const float z = __uint_as_float(sv[e + f]) + cbias;
+                                const float h = 0.5f * z;
+                                const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
+                                const float a = z * sg;
+                                const float gd = fmaf(a, 1.f - sg, sg);
+                                av[f] = a * p.inv_alpha;
+                                zv[f] = __uint_as_float(dp[e + f]) * p.inv_alpha * gd;
+                                fast_sum += zv[f];
+                            }
+                            pa[e >> 1] = pack_bf16x2(av[0], av[1]);
+                            pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
+                        }
+                    } else {
+                        int cur_tb = -1;
+                        float acc_tb = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float av[2], zv[2];
+#pragma unroll
+                            for (int f = 0; f < 2; f++) {
+                                const int ii = 32 * c + e + f;
+                                const int i = i0 + ii;
+                                const int64_t ts_i = w_qts[ii];
+                                const bool vis = key_ok && i < s.L && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
+                                const int pidx = pos_index(token_pos(KIND, min(i, s.L - 1), s.S, s.R), pos_j, p.P);
+                                const int tb = time_bucket(ts_i, ts_j, p.nb);
+                                const float z = __uint_as_float(sv[e + f]) + s_rp[pidx] + s_rt[tb];
+                                const float h = 0.5f * z;
+                                const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
+                                const float a = z * sg;
+                                const float gd = fmaf(a, 1.f - sg, sg);
+                                av[f] = vis ? a * p.inv_alpha : 0.f;
+                                const float dz = vis ? __uint_as_float(dp[e + f]) * p.inv_alpha * gd : 0.f;
+                                zv[f] = dz;
+                                if (vis) atomicAdd(&s_grp[pidx], dz);
+                                if (tb != cur_tb) {
+                                    if (cur_tb >= 0 && acc_tb != 0.f) atomicAdd(&s_grt[cur_tb], acc_tb);
+                                    cur_tb = tb;
+                                    acc_tb = 0.f;
+                                }
+                                acc_tb += dz;
+                            }
+                            pa[e >> 1] = pack_bf16x2(av[0], av[1]);
+                            pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
+                        }
+                        if (cur_tb >= 0 && acc_tb != 0.f) atomicAdd(&s_grt[cur_tb], acc_tb);
+                    }
+                    // A^T back into TMEM over the S^T columns this warp group has read
+                    tmem_st16(tmem + lane_base + kSCol + 64 * g + 16 * c, pa);
+                    // dZ^T into shared memory: row r, queries 64g+32c.. (128-byte swizzle)
+                    const uint32_t row_addr = aDZ + g * kPanel + r * 128;
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const uint32_t ch = (uint32_t)((4 * c + e) ^ (r & 7));
+                        st_shared_v4(row_addr + ch * 16, pz[4 * e], pz[4 * e + 1], pz[4 * e + 2], pz[4 * e + 3]);
+                    }
+                }
+                if (fast) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) fast_sum += __shfl_xor_sync(kFull, fast_sum, o);
+                    if (lane == 0 && fast_sum != 0.f) {
+                        atomicAdd(&s_grp[pidx_u], fast_sum);
+                        atomicAdd(&s_grt[tb_u], fast_sum);
+                    }
+                }
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars[kPFull]);
+                // drain dQ of this query tile (rows = queries, this group's half of the columns)
+                ok = mbar_wait(&bars[kDQFull], dq_use & 1, s_abort);
+                if (!__all_sync(kFull, ok)) { ok = false; break; }
+                dq_use++;
+                tc_fence_after();
+                const int qi = t * kTileM + r;            // query row held in this TMEM lane
+#pragma unroll 1
+                for (int c = 0; c < D / 64; c++) {
+                    uint32_t v[32];
+                    const int col = g * (D / 2) + 32 * c;
+                    tmem_ld32(tmem + lane_base + kPCol + col, v);
+                    tmem_ld_wait(v);
+                    if (qi < s.L) {
+                        float* dst = p.dq_acc + (size_t)(s.off0 + qi) * p.ld + (size_t)s.h * D + col;
+#pragma unroll
+                        for (int e = 0; e < 8; e++)
+                            red_add_v4(dst + 4 * e, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                       __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars[kDQDrained]);
+                n_done++;
+            }
+            if (!ok) break;
+            // ---------------- epilogue: dV, dK rows of this key tile
+            ok = mbar_wait(&bars[kAccFull], acc_use & 1, s_abort);
+            if (!__all_sync(kFull, ok)) { ok = false; break; }
+            acc_use++;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 64; c++) {
+                const int col = g * (D / 2) + 32 * c;
+                uint32_t vv[32], kv[32];
+                tmem_ld32(tmem + lane_base + kVCol + col, vv);
+                tmem_ld32(tmem + lane_base + kKCol + col, kv);
+                tmem_ld_wait(vv);
+                tmem_ld_wait(kv);
+                if (key_ok) {
+                    uint4 wv[4], wk[4];
+                    uint32_t* pv = reinterpret_cast<uint32_t*>(wv);
+                    uint32_t* pk = reinterpret_cast<uint32_t*>(wk);
+#pragma unroll
+                    for (int e = 0; e < 16; e++) {
+                        pv[e] = n_done ? pack_bf16x2(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1])) : 0u;
+                        pk[e] = n_done ? pack_bf16x2(__uint_as_float(kv[2 * e]), __uint_as_float(kv[2 * e + 1])) : 0u;
+                    }
+                    const size_t o = (size_t)(s.off0 + j) * p.ld + (size_t)s.h * D + col;
+                    uint4* dv = reinterpret_cast<uint4*>(p.dv + o);
+                    uint4* dk = reinterpret_cast<uint4*>(p.dk + o);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        dv[e] = wv[e];
+                        dk[e] = wk[e];
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[kAccEmpty]);
+            mbar_arrive(&bars[kItEmpty0 + slot]);
+        }
+        if (!ok && lane == 0 && !*s_abort) flag_timeout(p, s_abort);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    // rab gradients of this CTA
+    for (int i = tid; i < np; i += kThreads)
+        if (s_grp[i] != 0.f) atomicAdd(&p.d_rab_pos[i], s_grp[i]);
+    for (int i = tid; i < p.nb; i += kThreads)
+        if (s_grt[i] != 0.f) atomicAdd(&p.d_rab_time[i], s_grt[i]);
+}
+
+template <int KIND, int D>
+cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdy, const BwdParams& p, int grid, cudaStream_t s) {
+    constexpr uint32_t smem = BwdSmem<D>::alloc;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<KIND, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    prof_begin(kProfAttnBwdTc, s);
+    attn_bwd_tc_kernel<KIND, D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdy, p);
+    prof_end(kProfAttnBwdTc, s);
+    return cudaGetLastError();
+}
+
+__global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, long long n4) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float4 v = src[i];
+        uint2 o;
+        o.x = pack_bf16x2(v.x, v.y);
+        o.y = pack_bf16x2(v.z, v.w);
+        dst[i] = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const CUtensorMap& tdy, const BwdParams& p,
+                               int grid, cudaStream_t s) {
+#define HSTU_BWD_CASE(K, DD) \
+    if (kind == K && d == DD) return launch_one<K, DD>(tq, tk, tv, tdy, p, grid, s);
+    HSTU_BWD_CASE(HSTU_KIND_CAUSAL, 128)
+    HSTU_BWD_CASE(HSTU_KIND_CAUSAL, 64)
+    HSTU_BWD_CASE(HSTU_KIND_MTGR, 128)
+    HSTU_BWD_CASE(HSTU_KIND_MTGR, 64)
+#undef HSTU_BWD_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t s) {
+    const long long n4 = n / 4;   // n is a multiple of 8 (H*d with d in {64, 128})
+    const int threads = 256;
+    long long blocks = (n4 + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    prof_begin(kProfDqConvert, s);
+    f32_to_bf16_kernel<<<(unsigned)blocks, threads, 0, s>>>(reinterpret_cast<const float4*>(src),
+                                                             reinterpret_cast<uint2*>(dst), n4);
+    prof_end(kProfDqConvert, s);
+    return cudaGetLastError();
+}
+
+}  // namespace hstu

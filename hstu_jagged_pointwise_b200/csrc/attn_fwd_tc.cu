@@ -523,14 +523,19 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 template <int KIND, int D>
 int ctas_per_sm_one() {
+    // Shared memory decides: each CTA holds ~110 KB (plus the 1 KB the driver
+    // reserves per CTA) and 256 TMEM columns, so at most two fit on an SM.
     constexpr uint32_t smem = FwdSmem<D>::alloc;
     cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          smem);
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_fwd_tc_kernel<KIND, D>, kThreads,
-                                                      smem) != cudaSuccess)
+    cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         100);
+    int dev = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
         return 1;
-    return n < 1 ? 1 : (n > 2 ? 2 : n);   // two CTAs fill the SM's 512 TMEM columns
+    const int n = per_sm / (int)(smem + 1024);
+    return n < 1 ? 1 : (n > 2 ? 2 : n);
 }
 
 }  // namespace

@@ -117,7 +117,7 @@ int check_mask(const hstu_mask_spec* m, int* kind) {
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-    size_t items = 0, perm = 0, seq_base = 0, dy = 0, part = 0, total = 0;
+    size_t items = 0, perm = 0, seq_base = 0, dy = 0, part = 0, dq_acc = 0, total = 0;
     long long max_items = 0;
     int n_part = 0;
 };
@@ -139,6 +139,10 @@ Layout attn_layout(const hstu_dims& d, int is_bwd) {
         L.n_part = ln_bwd_partials(d.T);
         L.part = off;
         off = align_up(off + (size_t)L.n_part * 2 * D * 4, 256);
+        if (d.dtype == HSTU_BF16) {
+            L.dq_acc = off;                      // fp32 dQ accumulated across key tiles
+            off = align_up(off + (size_t)d.T * D * 4, 256);
+        }
     }
     L.total = off;
     return L;
@@ -353,7 +357,7 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
         return HSTU_ERR_INVALID_ARG;
     Control* ctrl = at<Control>(workspace, 0);
 
-    // 1. validation
+    // 1. validation + work list of (sequence, head, key tile)
     SchedParams sp;
     memset(&sp, 0, sizeof(sp));
     sp.kind = kind;
@@ -365,6 +369,7 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     sp.n_rt = mask->n_realtime;
     sp.max_q_len = sp.max_kv_len = d.max_seq_len;
     sp.b_m = 1;
+    sp.ascending = 1;        // backward items are key tiles: the first one is seen by most queries
     sp.ctrl = ctrl;
     sp.items = at<int4>(workspace, L.items);
     sp.perm = at<int>(workspace, L.perm);
@@ -396,14 +401,49 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     if (st != HSTU_OK) return st;
 
     // 3. attention backward
-    SimtParams p = simt_params(d, kind, *mask, seq_offsets, timestamps, rab_pos, rab_time, q, k, v, ctrl);
-    p.dy = lp.dy;
-    p.dq = dq;
-    p.dk = dk;
-    p.dv = dv;
-    p.d_rab_pos = d_rab_pos;
-    p.d_rab_time = d_rab_time;
-    return cuda_status(launch_attn_bwd_simt(d.dtype == HSTU_F32, d.d_qk, p, s));
+    if (d.dtype == HSTU_F32) {
+        SimtParams p = simt_params(d, kind, *mask, seq_offsets, timestamps, rab_pos, rab_time, q, k, v,
+                                   ctrl);
+        p.dy = lp.dy;
+        p.dq = dq;
+        p.dk = dk;
+        p.dv = dv;
+        p.d_rab_pos = d_rab_pos;
+        p.d_rab_time = d_rab_time;
+        return cuda_status(launch_attn_bwd_simt(1, d.d_qk, p, s));
+    }
+    const DevInfo* di = dev_info();
+    if (!di) return HSTU_ERR_CUDA;
+    CUtensorMap tq, tk, tv, tdy;
+    if (!make_tmap(&tq, q, d.T, D) || !make_tmap(&tk, k, d.T, D) || !make_tmap(&tv, v, d.T, D) ||
+        !make_tmap(&tdy, lp.dy, d.T, D))
+        return HSTU_ERR_CUDA;
+    float* dq_acc = at<float>(workspace, L.dq_acc);
+    st = cuda_status(cudaMemsetAsync(dq_acc, 0, (size_t)d.T * D * sizeof(float), s));
+    if (st != HSTU_OK) return st;
+    BwdParams bp;
+    memset(&bp, 0, sizeof(bp));
+    bp.off = seq_offsets;
+    bp.ts = timestamps;
+    bp.n_static = mask->n_static;
+    bp.n_rt = mask->n_realtime;
+    bp.rab_pos = rab_pos;
+    bp.rab_time = rab_time;
+    bp.items = sp.items;
+    bp.ctrl = ctrl;
+    bp.dq_acc = dq_acc;
+    bp.dk = static_cast<__nv_bfloat16*>(dk);
+    bp.dv = static_cast<__nv_bfloat16*>(dv);
+    bp.d_rab_pos = d_rab_pos;
+    bp.d_rab_time = d_rab_time;
+    bp.H = d.H;
+    bp.P = d.n_pos;
+    bp.nb = d.n_tbuckets;
+    bp.ld = D;
+    bp.inv_alpha = 1.0f / d.alpha;
+    st = cuda_status(launch_attn_bwd_tc(kind, d.d_qk, tq, tk, tv, tdy, bp, di->sms, s));
+    if (st != HSTU_OK) return st;
+    return cuda_status(launch_f32_to_bf16(dq_acc, static_cast<__nv_bfloat16*>(dq), (long long)d.T * D, s));
 }
 
 size_t hstu_mfalcon_workspace_bytes(const hstu_mfalcon_dims* dims, int32_t b_m) {

@@ -43,6 +43,7 @@ struct SchedParams {
     const int32_t* n_static;
     const int32_t* n_rt;
     int max_q_len, max_kv_len, b_m;
+    int ascending;   // causal/MTGR tile order inside a group: 1 = first tile first (backward key tiles)
     Control* ctrl;
     int4* items;
     int* perm;       // [B]
@@ -65,6 +66,25 @@ struct FwdParams {
     const __nv_bfloat16* self_q;   // M-FALCON candidate q/k/v for the self term
     const __nv_bfloat16* self_k;
     const __nv_bfloat16* self_v;
+    int H, P, nb, ld;
+    float inv_alpha;
+};
+
+// tcgen05 backward: one work item = (sequence, head, 128-key tile).
+struct BwdParams {
+    const int32_t* off;
+    const int64_t* ts;
+    const int32_t* n_static;
+    const int32_t* n_rt;
+    const float* rab_pos;
+    const float* rab_time;
+    const int4* items;
+    Control* ctrl;
+    float* dq_acc;            // [T, H*d] fp32, zeroed before the launch
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* d_rab_pos;
+    float* d_rab_time;
     int H, P, nb, ld;
     float inv_alpha;
 };
@@ -116,7 +136,8 @@ struct LnParams {
 // ---- opt-in per-kernel timing (profile.cu)
 enum ProfKind {
     kProfSchedule = 0, kProfAttnFwdTc, kProfAttnFwdSimt, kProfLnFwd, kProfLnBwd, kProfLnBwdReduce,
-    kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfKinds
+    kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfDqConvert,
+    kProfKinds
 };
 void prof_begin(int kind, cudaStream_t s);
 void prof_end(int kind, cudaStream_t s);
@@ -128,6 +149,10 @@ cudaError_t launch_attn_fwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
 int attn_fwd_tc_ctas_per_sm(int kind, int d);
 cudaError_t launch_attn_fwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
+cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const CUtensorMap& tdy, const BwdParams& p,
+                               int grid, cudaStream_t s);
+cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t s);
 cudaError_t launch_ln_fwd(int dtype_f32, const LnParams& p, cudaStream_t s);
 cudaError_t launch_ln_bwd(int dtype_f32, const LnParams& p, cudaStream_t s);
 int ln_bwd_partials(long long T);

@@ -28,7 +28,7 @@ __device__ int n_q_tiles(const SchedParams& p, int Lq) {
 // rows [row0, row_end) of query tile k (tile order inside a (sequence, head) group)
 __device__ void tile_rows(const SchedParams& p, int Lq, int nt, int k, int* row0, int* row_end) {
     if (p.kind != HSTU_KIND_MFALCON) {
-        const int t = nt - 1 - k;                        // heaviest (last) tile first
+        const int t = p.ascending ? k : nt - 1 - k;      // heaviest tile first
         *row0 = t * kTileM;
         *row_end = min(*row0 + kTileM, Lq);
         return;

@@ -340,7 +340,7 @@ def large_layer(seed: int = 0, total: int = 262144, with_grad: bool = True) -> W
     rng = np.random.Generator(np.random.PCG64(seed))
     lengths = lognormal_lengths(rng, total)
     return make_causal(lengths, H=8, d=128, dtype=torch.bfloat16, seed=seed + 404,
-                       with_grad=with_grad, name="large_layer_T262144_H8_d128")
+                       with_grad=with_grad, name=f"large_layer_T{total}_H8_d128")
 
 
 CONFIGS = {0: tiny_fp32, 1: training_sl, 2: mtgr_medium, 3: mfalcon_ranking, 4: large_layer}
