@@ -25,6 +25,7 @@
 // bucket, one atomic per element for the position index, or a warp sum when the
 // bias is uniform over the warp's block), flushed to global memory at the end.
 // Every wait is bounded; a timeout sets the status word and the CTA exits cleanly.
+#include "ew_bias.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -46,8 +47,12 @@ struct BwdSmem {
     static constexpr uint32_t rt = rp + 2u * kMaxPos * 4u;       // float[64]
     static constexpr uint32_t grp = rt + kMaxTBuckets * 4u;      // float[2*kMaxPos]
     static constexpr uint32_t grt = grp + 2u * kMaxPos * 4u;     // float[64]
-    static constexpr uint32_t qts = grt + kMaxTBuckets * 4u;     // int64[8 warps][64]
-    static constexpr uint32_t item = qts + 8u * 64u * 8u;        // int4[2]
+    static constexpr uint32_t rth = grt + kMaxTBuckets * 4u;     // float[64]: rab_time / 2
+    static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][64]
+    static constexpr uint32_t qrel = qts + 8u * 64u * 8u;        // int32[8 warps][64]
+    static constexpr uint32_t diag = qrel + 8u * 64u * 4u;       // float[8 warps][96]
+    static constexpr uint32_t gdiag = diag + 8u * 96u * 4u;      // float[8 warps][96]
+    static constexpr uint32_t item = gdiag + 8u * 96u * 4u;      // int4[2]
     static constexpr uint32_t bars = item + 2u * 16u;            // uint64[24]
     static constexpr uint32_t tmem = bars + 24u * 8u;
     static constexpr uint32_t abort_flag = tmem + 4u;
@@ -104,6 +109,70 @@ __device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* a
     atomicOr(&p.ctrl->status, kStatusTimeout);
 }
 
+// One 32-column chunk of a dense block: keys in lanes, queries along the chunk.
+// dg / gg point at this lane's diagonal-row entry for the chunk's first query
+// (entries for later queries sit at decreasing addresses); qr holds the
+// chunk's 32-bit query times relative to the block's smallest key time.
+template <int PM, int TM>
+__device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* dg,
+                                          float* gg, const int32_t* qr, int32_t a_j, uint32_t thr, float c0,
+                                          float c1, const float* rth, int nbm1, float inv_alpha, float& acc,
+                                          float& acc_hi, float* s_grt, uint32_t (&pa)[16], uint32_t (&pz)[16]) {
+    int32_t q[32];
+    if (TM != kTimeUniform) {
+        const int4* q4 = reinterpret_cast<const int4*>(qr);
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+            const int4 v = q4[e];
+            q[4 * e] = v.x; q[4 * e + 1] = v.y; q[4 * e + 2] = v.z; q[4 * e + 3] = v.w;
+        }
+    }
+    int cur_t = -1;
+    float acc_t = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float av[2], zv[2];
+#pragma unroll
+        for (int f = 0; f < 2; f++) {
+            const int k = e + f;
+            float hb = PM == kPosUniform ? c0 : dg[-k];
+            bool hi_b = false;
+            int tb = 0;
+            if (TM == kTimeTwo) {
+                const uint32_t x = (uint32_t)abs(q[k] - a_j);
+                hi_b = x >= thr;
+                if (PM == kPosUniform) hb = hi_b ? c1 : c0;
+                else hb += hi_b ? c1 : c0;
+            } else if (TM == kTimeBits) {
+                const uint32_t x = (uint32_t)abs(q[k] - a_j);
+                tb = time_bucket_u32(x, nbm1);
+                hb += rth[tb];
+            }
+            const float h = fmaf(__uint_as_float(sv[k]), 0.5f, hb);
+            const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
+            const float a = 2.f * h * sg;
+            const float gd = fmaf(a, 1.f - sg, sg);
+            av[f] = a * inv_alpha;
+            const float dz = __uint_as_float(dp[k]) * inv_alpha * gd;
+            zv[f] = dz;
+            acc += dz;
+            if (TM == kTimeTwo) acc_hi += hi_b ? dz : 0.f;
+            if (TM == kTimeBits) {
+                if (tb != cur_t) {
+                    if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+                    cur_t = tb;
+                    acc_t = 0.f;
+                }
+                acc_t += dz;
+            }
+            if (PM == kPosDiag) atomicAdd(gg - k, dz);
+        }
+        pa[e >> 1] = pack_bf16x2(av[0], av[1]);
+        pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
+    }
+    if (TM == kTimeBits && cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+}
+
 template <int KIND, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -139,6 +208,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int i = tid; i < p.nb; i += kThreads) {
         s_rt[i] = p.rab_time[i];
         s_grt[i] = 0.f;
+        reinterpret_cast<float*>(sm + L::rth)[i] = 0.5f * p.rab_time[i];
     }
     if (tid == 0) {
         const uint32_t counts[kNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, kEwThreads, 1, kEwThreads, 1, 1,
@@ -356,6 +426,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const uint32_t aDZ = smem_u32(sm + L::dz);
         int64_t* w_qts = s_qts + warp * 64;
+        int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * 64;
+        float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * 96;
+        float* w_gdiag = reinterpret_cast<float*>(sm + L::gdiag) + warp * 96;
+        float* s_rth = reinterpret_cast<float*>(sm + L::rth);   // rab_time / 2
+        const int nbm1 = p.nb - 1;
         int it_use = 0, s_use = 0, dz_use = 0, dq_use = 0, acc_use = 0;
         bool ok = true;
         while (ok) {
@@ -371,15 +446,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int jc = min(j, s.n_end - 1);
             const int64_t ts_j = p.ts[s.off0 + jc];
             const int pos_j = token_pos(KIND, jc, s.S, s.R);
+            const int ka = s.n0 + 32 * wq;           // first key of this warp
             int64_t kmin = key_ok ? ts_j : INT64_MAX, kmax = key_ok ? ts_j : INT64_MIN;
-            int pk_lo = key_ok ? pos_j : INT32_MAX, pk_hi = key_ok ? pos_j : INT32_MIN;
             int warp_keys = key_ok ? 1 : 0;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 kmin = min(kmin, (int64_t)__shfl_xor_sync(kFull, (long long)kmin, o));
                 kmax = max(kmax, (int64_t)__shfl_xor_sync(kFull, (long long)kmax, o));
-                pk_lo = min(pk_lo, __shfl_xor_sync(kFull, pk_lo, o));
-                pk_hi = max(pk_hi, __shfl_xor_sync(kFull, pk_hi, o));
                 warp_keys += __shfl_xor_sync(kFull, warp_keys, o);
             }
             const int n_qt = (s.L + kTileM - 1) / kTileM;
@@ -406,98 +479,124 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
                     qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
                 }
-                __syncwarp();
-                // uniform bias and full visibility over this warp's 32 keys x 64 queries?
-                bool fast = false;
-                int pidx_u = 0, tb_u = 0;
-                float cbias = 0.f;
-                if (warp_keys == 32 && i0 + 64 <= s.L) {
-                    const int ka = s.n0 + 32 * wq;
-                    fast = tile_class(KIND, i0, i0 + 63, ka, ka + 31, s.S, s.R) == 2;
-                    if (fast) {
-                        const int pq_lo = token_pos(KIND, i0, s.S, s.R);
-                        const int pq_hi = token_pos(KIND, i0 + 63, s.S, s.R);
-                        const int dmax = pk_hi - pq_lo, dmin = pk_lo - pq_hi;
-                        pidx_u = -1;
-                        if (dmax <= -(p.P - 1)) pidx_u = 0;
-                        else if (dmin >= p.P - 1) pidx_u = 2 * p.P - 2;
-                        uint64_t lo;
-                        if (qmin > kmax) lo = abs_diff_u64(qmin, kmax);
-                        else if (kmin > qmax) lo = abs_diff_u64(kmin, qmax);
-                        else lo = 0;
-                        const uint64_t hi = max(abs_diff_u64(qmax, kmin), abs_diff_u64(kmax, qmin));
-                        tb_u = time_bucket_of_delta(lo, p.nb);
-                        fast = pidx_u >= 0 && tb_u == time_bucket_of_delta(hi, p.nb);
-                        if (fast) cbias = s_rp[pidx_u] + s_rt[tb_u];
+                // ---- classify this warp's block: 32 keys x 64 queries
+                int wcls = 0;
+                if (warp_keys > 0 && i0 < s.L)
+                    wcls = tile_class(KIND, i0, min(i0 + 63, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
+                int pm = -1, tm = -1;            // -1 = element-by-element rules
+                float c0 = 0.f, c1 = 0.f;
+                int pidx_u = 0;
+                TimeClass tc;
+                tc.tb_lo = tc.tb_hi = 0;
+                tc.thr = 0;
+                const bool dense = wcls != 0 && warp_keys == 32 && i0 + 64 <= s.L &&
+                                   (KIND == HSTU_KIND_CAUSAL || wcls == 2);
+                if (dense) {
+                    tc = classify_time(kmin, kmax, qmin, qmax, p.nb);
+                    if (tc.mode >= 0) {
+                        tm = tc.mode;
+                        const int dmax = ka + 31 - i0, dmin = ka - (i0 + 63);   // j - i over the block
+                        if (wcls == 2 && dmax <= -(p.P - 1)) { pm = kPosUniform; pidx_u = 0; }
+                        else if (wcls == 2 && dmin >= p.P - 1) { pm = kPosUniform; pidx_u = 2 * p.P - 2; }
+                        else pm = kPosDiag;
+                        if (pm == kPosDiag) {
+                            // diagonal row: delta = j - i = dmin + k, k in [0, 95)
+                            const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
+                            for (int k = lane; k < 95; k += 32) {
+                                const int dl = dmin + k;
+                                const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
+                                w_diag[k] = masked ? kMaskedHalfBias
+                                                   : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
+                                w_gdiag[k] = 0.f;
+                            }
+                        }
+                        const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
+                        if (tm == kTimeUniform) c0 = ph + s_rth[tc.tb_lo];
+                        else if (tm == kTimeTwo) { c0 = ph + s_rth[tc.tb_lo]; c1 = ph + s_rth[tc.tb_hi]; }
+                        else c0 = ph;
+                        if (tm != kTimeUniform) {
+                            const int32_t qa = (int32_t)(w_qts[lane] - kmin);
+                            const int32_t qb = (int32_t)(w_qts[lane + 32] - kmin);
+                            w_qrel[lane] = qa;
+                            w_qrel[lane + 32] = qb;
+                        }
                     }
                 }
+                __syncwarp();
                 ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
                 if (ok) ok = mbar_wait(&bars[kDZEmpty], (dz_use & 1) ^ 1, s_abort);
                 if (!__all_sync(kFull, ok)) { ok = false; break; }
                 s_use++;
                 dz_use++;
                 tc_fence_after();
-                float fast_sum = 0.f;
+                const int32_t a_j = (int32_t)(ts_j - kmin);
+                float acc = 0.f, acc_hi = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 2; c++) {
-                    uint32_t sv[32], dp[32];
-                    tmem_ld32(tmem + lane_base + kSCol + 64 * g + 32 * c, sv);
-                    tmem_ld32(tmem + lane_base + kPCol + 64 * g + 32 * c, dp);
-                    tmem_ld_wait(sv);
-                    tmem_ld_wait(dp);
                     uint32_t pa[16], pz[16];
-                    if (fast) {
+                    if (wcls == 0) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float av[2], zv[2];
-#pragma unroll
-                            for (int f = 0; f < 2; f++) {
-                                const float z = __uint_as_float(sv[e + f]) + cbias;
-                                const float h = 0.5f * z;
-                                const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
-                                const float a = z * sg;
-                                const float gd = fmaf(a, 1.f - sg, sg);
-                                av[f] = a * p.inv_alpha;
-                                zv[f] = __uint_as_float(dp[e + f]) * p.inv_alpha * gd;
-                                fast_sum += zv[f];
-                            }
-                            pa[e >> 1] = pack_bf16x2(av[0], av[1]);
-                            pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
-                        }
+                        for (int e = 0; e < 16; e++) pa[e] = pz[e] = 0u;
                     } else {
-                        int cur_tb = -1;
-                        float acc_tb = 0.f;
+                        uint32_t sv[32], dp[32];
+                        tmem_ld32(tmem + lane_base + kSCol + 64 * g + 32 * c, sv);
+                        tmem_ld32(tmem + lane_base + kPCol + 64 * g + 32 * c, dp);
+                        tmem_ld_wait(sv);
+                        tmem_ld_wait(dp);
+                        const float* dg = w_diag + lane + 63 - 32 * c;
+                        float* gg = w_gdiag + lane + 63 - 32 * c;
+                        const int32_t* qr = w_qrel + 32 * c;
+#define HSTU_BWD_SPEC(PM_, TM_) \
+    bwd_block<PM_, TM_>(sv, dp, dg, gg, qr, a_j, tc.thr, c0, c1, s_rth, nbm1, p.inv_alpha, acc, acc_hi, s_grt, pa, pz)
+                        if (pm == kPosUniform && tm == kTimeUniform) HSTU_BWD_SPEC(kPosUniform, kTimeUniform);
+                        else if (pm == kPosUniform && tm == kTimeTwo) HSTU_BWD_SPEC(kPosUniform, kTimeTwo);
+                        else if (pm == kPosUniform && tm == kTimeBits) HSTU_BWD_SPEC(kPosUniform, kTimeBits);
+                        else if (pm == kPosDiag && tm == kTimeUniform) HSTU_BWD_SPEC(kPosDiag, kTimeUniform);
+                        else if (pm == kPosDiag && tm == kTimeTwo) HSTU_BWD_SPEC(kPosDiag, kTimeTwo);
+                        else if (pm == kPosDiag && tm == kTimeBits) HSTU_BWD_SPEC(kPosDiag, kTimeBits);
+#undef HSTU_BWD_SPEC
+                        else {
+                            // element by element (MTGR candidates, ragged edges, int64-wide times)
+                            int cur_p = -1, cur_t = -1;
+                            float acc_p = 0.f, acc_t = 0.f;
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float av[2], zv[2];
+                            for (int e = 0; e < 32; e += 2) {
+                                float av[2], zv[2];
 #pragma unroll
-                            for (int f = 0; f < 2; f++) {
-                                const int ii = 32 * c + e + f;
-                                const int i = i0 + ii;
-                                const int64_t ts_i = w_qts[ii];
-                                const bool vis = key_ok && i < s.L && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
-                                const int pidx = pos_index(token_pos(KIND, min(i, s.L - 1), s.S, s.R), pos_j, p.P);
-                                const int tb = time_bucket(ts_i, ts_j, p.nb);
-                                const float z = __uint_as_float(sv[e + f]) + s_rp[pidx] + s_rt[tb];
-                                const float h = 0.5f * z;
-                                const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
-                                const float a = z * sg;
-                                const float gd = fmaf(a, 1.f - sg, sg);
-                                av[f] = vis ? a * p.inv_alpha : 0.f;
-                                const float dz = vis ? __uint_as_float(dp[e + f]) * p.inv_alpha * gd : 0.f;
-                                zv[f] = dz;
-                                if (vis) atomicAdd(&s_grp[pidx], dz);
-                                if (tb != cur_tb) {
-                                    if (cur_tb >= 0 && acc_tb != 0.f) atomicAdd(&s_grt[cur_tb], acc_tb);
-                                    cur_tb = tb;
-                                    acc_tb = 0.f;
+                                for (int f = 0; f < 2; f++) {
+                                    const int ii = 32 * c + e + f;
+                                    const int i = i0 + ii;
+                                    const int64_t ts_i = w_qts[ii];
+                                    const bool vis = key_ok && i < s.L && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
+                                    const int pidx = pos_index(token_pos(KIND, min(i, s.L - 1), s.S, s.R), pos_j, p.P);
+                                    const int tb = time_bucket(ts_i, ts_j, p.nb);
+                                    const float h = fmaf(__uint_as_float(sv[e + f]), 0.5f,
+                                                         0.5f * s_rp[pidx] + s_rth[tb]);
+                                    const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
+                                    const float a = 2.f * h * sg;
+                                    const float gd = fmaf(a, 1.f - sg, sg);
+                                    av[f] = vis ? a * p.inv_alpha : 0.f;
+                                    const float dz = vis ? __uint_as_float(dp[e + f]) * p.inv_alpha * gd : 0.f;
+                                    zv[f] = dz;
+                                    if (pidx != cur_p) {
+                                        if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
+                                        cur_p = pidx;
+                                        acc_p = 0.f;
+                                    }
+                                    acc_p += dz;
+                                    if (tb != cur_t) {
+                                        if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+                                        cur_t = tb;
+                                        acc_t = 0.f;
+                                    }
+                                    acc_t += dz;
                                 }
-                                acc_tb += dz;
+                                pa[e >> 1] = pack_bf16x2(av[0], av[1]);
+                                pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
                             }
-                            pa[e >> 1] = pack_bf16x2(av[0], av[1]);
-                            pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
+                            if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
+                            if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
                         }
-                        if (cur_tb >= 0 && acc_tb != 0.f) atomicAdd(&s_grt[cur_tb], acc_tb);
                     }
                     // A^T back into TMEM over the S^T columns this warp group has read
                     tmem_st16(tmem + lane_base + kSCol + 64 * g + 16 * c, pa);
@@ -509,12 +608,29 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         st_shared_v4(row_addr + ch * 16, pz[4 * e], pz[4 * e + 1], pz[4 * e + 2], pz[4 * e + 3]);
                     }
                 }
-                if (fast) {
+                // ---- rab gradients of the dense block
+                if (pm >= 0) {
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) fast_sum += __shfl_xor_sync(kFull, fast_sum, o);
-                    if (lane == 0 && fast_sum != 0.f) {
-                        atomicAdd(&s_grp[pidx_u], fast_sum);
-                        atomicAdd(&s_grt[tb_u], fast_sum);
+                    for (int o = 16; o > 0; o >>= 1) {
+                        acc += __shfl_xor_sync(kFull, acc, o);
+                        acc_hi += __shfl_xor_sync(kFull, acc_hi, o);
+                    }
+                    if (lane == 0) {
+                        if (pm == kPosUniform) atomicAdd(&s_grp[pidx_u], acc);
+                        if (tm == kTimeUniform) atomicAdd(&s_grt[tc.tb_lo], acc);
+                        if (tm == kTimeTwo) {
+                            atomicAdd(&s_grt[tc.tb_hi], acc_hi);
+                            atomicAdd(&s_grt[tc.tb_lo], acc - acc_hi);
+                        }
+                    }
+                    if (pm == kPosDiag) {
+                        __syncwarp();
+                        const int dmin = ka - (i0 + 63);
+                        for (int k = lane; k < 95; k += 32) {
+                            const float v = w_gdiag[k];
+                            if (v != 0.f)
+                                atomicAdd(&s_grp[min(max(dmin + k, -(p.P - 1)), p.P - 1) + p.P - 1], v);
+                        }
                     }
                 }
                 tmem_st_wait();

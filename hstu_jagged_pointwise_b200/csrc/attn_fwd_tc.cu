@@ -17,6 +17,7 @@
 // TMEM columns: S/P at [0, 128), O at [128, 128 + D).
 // Every wait is bounded; on timeout the CTA records a status bit, drains its
 // copies and MMAs, frees TMEM and exits.
+#include "ew_bias.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -31,15 +32,17 @@ struct FwdSmem {
     static constexpr uint32_t q = 0;
     static constexpr uint32_t k = q + kTileBytes;
     static constexpr uint32_t v = k + kTileBytes;
-    static constexpr uint32_t rp = v + kTileBytes;              // float[2*kMaxPos]
-    static constexpr uint32_t rt = rp + 2u * kMaxPos * 4u;      // float[64]
-    static constexpr uint32_t cts = rt + kMaxTBuckets * 4u;     // int64[4 warps][128]
-    static constexpr uint32_t item = cts + 4u * 128u * 8u;      // int4[2]
-    static constexpr uint32_t bars = item + 2u * 16u;           // uint64[16]
-    static constexpr uint32_t tmem = bars + 16u * 8u;           // uint32
-    static constexpr uint32_t abort_flag = tmem + 4u;           // int
-    static constexpr uint32_t bytes = abort_flag + 4u;
-    static constexpr uint32_t alloc = bytes + 1024u;            // slack for 1024-B alignment
+    static constexpr uint32_t rt = v + kTileBytes;                 // float[64]
+    static constexpr uint32_t rth = rt + kMaxTBuckets * 4u;        // float[64]: rab_time / 2
+    static constexpr uint32_t cts = rth + kMaxTBuckets * 4u;       // int64[4 warps][128]
+    static constexpr uint32_t diag = cts + 4u * 128u * 8u;         // float[4 warps][160]
+    static constexpr uint32_t item = diag + 4u * 160u * 4u;        // int4[2]
+    static constexpr uint32_t bars = item + 2u * 16u;              // uint64[16]
+    static constexpr uint32_t tmem = bars + 16u * 8u;              // uint32
+    static constexpr uint32_t abort_flag = tmem + 4u;              // int
+    static constexpr uint32_t rp = abort_flag + 12u;               // float[2P-1], sized at launch
+    // bytes to request for a given P (1024 B of slack for the alignment of the base)
+    static constexpr uint32_t alloc(int P) { return rp + 8u * (uint32_t)P + 1024u; }
 };
 
 enum {
@@ -100,6 +103,43 @@ __device__ __forceinline__ void flag_timeout(const FwdParams& p, volatile int* a
     atomicOr(&p.ctrl->status, kStatusTimeout);
 }
 
+// One 32-column chunk of a dense block: rows in lanes, keys along the chunk.
+// dg points at this lane's diagonal-row entry for the chunk's first key;
+// cr holds the chunk's 32-bit key times relative to the tile's smallest one.
+template <int PM, int TM>
+__device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* dg, const int32_t* cr, int32_t a_i,
+                                          uint32_t thr, float c0, float c1, const float* rth, int nbm1,
+                                          uint32_t (&pk)[16]) {
+    int32_t b[32];
+    if (TM != kTimeUniform) {
+        const int4* b4 = reinterpret_cast<const int4*>(cr);
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+            const int4 x = b4[e];
+            b[4 * e] = x.x; b[4 * e + 1] = x.y; b[4 * e + 2] = x.z; b[4 * e + 3] = x.w;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float pv[2];
+#pragma unroll
+        for (int f = 0; f < 2; f++) {
+            const int k = e + f;
+            float hb = PM == kPosUniform ? c0 : dg[k];
+            if (TM == kTimeTwo) {
+                const bool hi_b = (uint32_t)abs(b[k] - a_i) >= thr;
+                if (PM == kPosUniform) hb = hi_b ? c1 : c0;
+                else hb += hi_b ? c1 : c0;
+            } else if (TM == kTimeBits) {
+                hb += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
+            }
+            const float h = fmaf(__uint_as_float(v[k]), 0.5f, hb);
+            pv[f] = fmaf(h, tanh_approx(h), h);
+        }
+        pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+    }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int KIND, int D>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -119,7 +159,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint8_t* sV = sm + L::v;
     float* s_rp = reinterpret_cast<float*>(sm + L::rp);
     float* s_rt = reinterpret_cast<float*>(sm + L::rt);
+    float* s_rth = reinterpret_cast<float*>(sm + L::rth);
     int64_t* s_cts = reinterpret_cast<int64_t*>(sm + L::cts);
+    float* s_diag = reinterpret_cast<float*>(sm + L::diag);
     int4* s_item = reinterpret_cast<int4*>(sm + L::item);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::tmem);
@@ -128,7 +170,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     for (int i = tid; i < 2 * p.P - 1; i += kThreads) s_rp[i] = p.rab_pos[i];
-    for (int i = tid; i < p.nb; i += kThreads) s_rt[i] = p.rab_time[i];
+    for (int i = tid; i < p.nb; i += kThreads) {
+        s_rt[i] = p.rab_time[i];
+        s_rth[i] = 0.5f * p.rab_time[i];
+    }
     if (tid == 0) {
         mbar_init(&bars[kQFull], 1);
         mbar_init(&bars[kQEmpty], 1);
@@ -312,7 +357,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int it_use = 0, s_use = 0, o_use = 0;
         const int r = tid;                                  // TMEM lane = tile row
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        int64_t* w_cts = s_cts + warp * 128;
+        int64_t* w_cts = s_cts + warp * 128;                // this warp's column times (int64)
+        int32_t* w_crel = reinterpret_cast<int32_t*>(w_cts); // or 32-bit relative times
+        float* w_diag = s_diag + warp * 160;
+        const int nbm1 = p.nb - 1;
         const float rp_self = s_rp[p.P - 1];
         const float rt_zero = s_rt[0];
         bool ok = true;
@@ -329,6 +377,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int ic = min(i, s.row_end - 1);           // clamped row for lookups
             const int64_t ts_i = p.q_ts[s.q0 + ic];
             const int pos_i = row_pos<KIND>(s, ic);
+            const int r0 = s.row0 + 32 * warp;              // first row of this warp
             // this warp's row range (positions and timestamps)
             int64_t rmin = row_ok ? ts_i : INT64_MAX, rmax = row_ok ? ts_i : INT64_MIN;
             int pr_lo = row_ok ? pos_i : INT32_MAX, pr_hi = row_ok ? pos_i : INT32_MIN;
@@ -346,18 +395,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int cls = kv_class<KIND>(s, t);
                 if (cls == 0) continue;
                 const int n0 = t * kTileN;
-                // column timestamps of this tile (each warp keeps its own copy)
+                // column timestamps of this tile
                 __syncwarp();
+                int64_t tj[4];
                 int64_t cmin = INT64_MAX, cmax = INT64_MIN;
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
-                    const int jj = lane + 32 * e;
-                    const int j = n0 + jj;
-                    const int64_t tj = j < s.Lk ? p.kv_ts[s.kv0 + j] : 0;
-                    w_cts[jj] = tj;
+                    const int j = n0 + lane + 32 * e;
+                    tj[e] = j < s.Lk ? p.kv_ts[s.kv0 + j] : 0;
                     if (j < s.Lk) {
-                        cmin = min(cmin, tj);
-                        cmax = max(cmax, tj);
+                        cmin = min(cmin, tj[e]);
+                        cmax = max(cmax, tj[e]);
                     }
                 }
 #pragma unroll
@@ -365,26 +413,61 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     cmin = min(cmin, (int64_t)__shfl_xor_sync(kFull, (long long)cmin, o));
                     cmax = max(cmax, (int64_t)__shfl_xor_sync(kFull, (long long)cmax, o));
                 }
-                __syncwarp();
-                // uniform-bias test for this warp's 32 rows x 128 columns
-                const int jl = min(n0 + kTileN, s.Lk) - 1;
-                bool fast = warp_rows && cls == 2 && n0 + kTileN <= s.Lk;
-                float cbias = 0.f;
-                if (fast) {
-                    const int dmax = col_pos<KIND>(s, jl) - pr_lo;
+                // ---- classify this warp's block: 32 rows x 128 columns
+                int pm = -1, tm = -1;
+                float c0 = 0.f, c1 = 0.f;
+                TimeClass tc;
+                tc.tb_lo = tc.tb_hi = 0;
+                tc.thr = 0;
+                int wcls = 0;
+                if (warp_rows)
+                    wcls = KIND == HSTU_KIND_MFALCON
+                               ? 2
+                               : tile_class(KIND, r0, min(r0 + 31, s.row_end - 1), n0,
+                                            min(n0 + kTileN - 1, s.Lk - 1), s.S, s.R);
+                const bool dense = wcls != 0 && n0 + kTileN <= s.Lk &&
+                                   (KIND == HSTU_KIND_CAUSAL || wcls == 2);
+                if (dense) {
+                    tc = classify_time(rmin, rmax, cmin, cmax, p.nb);
+                    const int dmax = col_pos<KIND>(s, n0 + kTileN - 1) - pr_lo;
                     const int dmin = col_pos<KIND>(s, n0) - pr_hi;
-                    int pidx = -1;
-                    if (dmax <= -(p.P - 1)) pidx = 0;
-                    else if (dmin >= p.P - 1) pidx = 2 * p.P - 2;
-                    uint64_t lo;
-                    if (rmin > cmax) lo = abs_diff_u64(rmin, cmax);
-                    else if (cmin > rmax) lo = abs_diff_u64(cmin, rmax);
-                    else lo = 0;
-                    const uint64_t hi = max(abs_diff_u64(rmax, cmin), abs_diff_u64(cmax, rmin));
-                    const int tlo = time_bucket_of_delta(lo, p.nb), thi = time_bucket_of_delta(hi, p.nb);
-                    fast = pidx >= 0 && tlo == thi;
-                    if (fast) cbias = s_rp[pidx] + s_rt[tlo];
+                    int pidx_u = -1;
+                    if (wcls == 2 && dmax <= -(p.P - 1)) pidx_u = 0;
+                    else if (wcls == 2 && dmin >= p.P - 1) pidx_u = 2 * p.P - 2;
+                    if (pidx_u >= 0) pm = kPosUniform;
+                    else if (KIND != HSTU_KIND_MFALCON) pm = kPosDiag;
+                    if (pm >= 0 && tc.mode >= 0) {
+                        tm = tc.mode;
+                        if (pm == kPosDiag) {
+                            // diagonal row: delta = j - i = (n0 - r0 - 31) + k, k in [0, 159)
+                            const int d0 = n0 - r0 - 31;
+                            const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
+                            for (int k = lane; k < 159; k += 32) {
+                                const int dl = d0 + k;
+                                const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
+                                w_diag[k] = masked ? kMaskedHalfBias
+                                                   : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
+                            }
+                        }
+                        const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
+                        if (tm == kTimeUniform) c0 = ph + s_rth[tc.tb_lo];
+                        else if (tm == kTimeTwo) { c0 = ph + s_rth[tc.tb_lo]; c1 = ph + s_rth[tc.tb_hi]; }
+                        else c0 = ph;
+                    } else {
+                        pm = -1;
+                    }
                 }
+                if (pm >= 0) {
+                    if (tm != kTimeUniform) {
+#pragma unroll
+                        for (int e = 0; e < 4; e++) w_crel[lane + 32 * e] = (int32_t)(tj[e] - cmin);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; e++) w_cts[lane + 32 * e] = tj[e];
+                }
+                __syncwarp();
+                const int32_t a_i = (int32_t)(ts_i - cmin);
                 ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
                 if (!__all_sync(kFull, ok)) { ok = false; break; }
                 s_use++;
@@ -395,14 +478,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
                     tmem_ld_wait(v);
                     uint32_t pk[16];
-                    if (fast) {
-#pragma unroll
-                        for (int e = 0; e < 16; e++) {
-                            const float p0 = silu_fast(__uint_as_float(v[2 * e]) + cbias);
-                            const float p1 = silu_fast(__uint_as_float(v[2 * e + 1]) + cbias);
-                            pk[e] = pack_bf16x2(p0, p1);
-                        }
-                    } else {
+                    const float* dg = w_diag + 31 - lane + 32 * c;
+                    const int32_t* cr = w_crel + 32 * c;
+#define HSTU_FWD_SPEC(PM_, TM_) fwd_block<PM_, TM_>(v, dg, cr, a_i, tc.thr, c0, c1, s_rth, nbm1, pk)
+                    if (pm == kPosUniform && tm == kTimeUniform) HSTU_FWD_SPEC(kPosUniform, kTimeUniform);
+                    else if (pm == kPosUniform && tm == kTimeTwo) HSTU_FWD_SPEC(kPosUniform, kTimeTwo);
+                    else if (pm == kPosUniform && tm == kTimeBits) HSTU_FWD_SPEC(kPosUniform, kTimeBits);
+                    else if (pm == kPosDiag && tm == kTimeUniform) HSTU_FWD_SPEC(kPosDiag, kTimeUniform);
+                    else if (pm == kPosDiag && tm == kTimeTwo) HSTU_FWD_SPEC(kPosDiag, kTimeTwo);
+                    else if (pm == kPosDiag && tm == kTimeBits) HSTU_FWD_SPEC(kPosDiag, kTimeBits);
+#undef HSTU_FWD_SPEC
+                    else {
+                        // element by element: MTGR candidates, ragged key tiles, int64-wide time spans
                         float pv[32];
 #pragma unroll
                         for (int e = 0; e < 32; e++) {
@@ -414,8 +501,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 vis = vis && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
                             const int pidx = pos_index(pos_i, col_pos<KIND>(s, j), p.P);
                             const int tb = time_bucket(ts_i, ts_j, p.nb);
-                            const float z = __uint_as_float(v[e]) + s_rp[pidx] + s_rt[tb];
-                            pv[e] = vis ? silu_fast(z) : 0.f;
+                            const float h = fmaf(__uint_as_float(v[e]), 0.5f, 0.5f * s_rp[pidx] + s_rth[tb]);
+                            pv[e] = vis ? fmaf(h, tanh_approx(h), h) : 0.f;
                         }
 #pragma unroll
                         for (int e = 0; e < 16; e++) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
@@ -507,11 +594,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 template <int KIND, int D>
 cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t s) {
-    constexpr uint32_t smem = FwdSmem<D>::alloc;
+    const uint32_t smem = FwdSmem<D>::alloc(p.P);
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             FwdSmem<D>::alloc(kMaxPos));
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -525,7 +613,7 @@ template <int KIND, int D>
 int ctas_per_sm_one() {
     // Shared memory decides: each CTA holds ~110 KB (plus the 1 KB the driver
     // reserves per CTA) and 256 TMEM columns, so at most two fit on an SM.
-    constexpr uint32_t smem = FwdSmem<D>::alloc;
+    constexpr uint32_t smem = FwdSmem<D>::alloc(kMaxPos);
     cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          smem);
     cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributePreferredSharedMemoryCarveout,
