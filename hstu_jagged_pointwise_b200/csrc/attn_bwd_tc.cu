@@ -51,8 +51,7 @@ struct BwdSmem {
     static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][64]
     static constexpr uint32_t qrel = qts + 8u * 64u * 8u;        // int32[8 warps][64]
     static constexpr uint32_t diag = qrel + 8u * 64u * 4u;       // float[8 warps][96]
-    static constexpr uint32_t gdiag = diag + 8u * 96u * 4u;      // float[8 warps][96]
-    static constexpr uint32_t item = gdiag + 8u * 96u * 4u;      // int4[2]
+    static constexpr uint32_t item = diag + 8u * 96u * 4u;       // int4[2]
     static constexpr uint32_t bars = item + 2u * 16u;            // uint64[24]
     static constexpr uint32_t tmem = bars + 24u * 8u;
     static constexpr uint32_t abort_flag = tmem + 4u;
@@ -115,9 +114,11 @@ __device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* a
 // chunk's 32-bit query times relative to the block's smallest key time.
 template <int PM, int TM>
 __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* dg,
-                                          float* gg, const int32_t* qr, int32_t a_j, uint32_t thr, float c0,
-                                          float c1, const float* rth, int nbm1, float inv_alpha, float& acc,
-                                          float& acc_hi, float* s_grt, uint32_t (&pa)[16], uint32_t (&pz)[16]) {
+                                          float& dlo, float& dhi, const int32_t* qr, int32_t a_j, uint32_t thr,
+                                          float c0, float c1, const float* rth, int nbm1, float inv_alpha,
+                                          float& acc, float& acc_hi, float* s_grt, uint32_t (&pa)[16],
+                                          uint32_t (&pz)[16]) {
+    const int lane = threadIdx.x & 31;
     int32_t q[32];
     if (TM != kTimeUniform) {
         const int4* q4 = reinterpret_cast<const int4*>(qr);
@@ -165,7 +166,13 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
                 }
                 acc_t += dz;
             }
-            if (PM == kPosDiag) atomicAdd(gg - k, dz);
+            if (PM == kPosDiag) {
+                // diagonal m = key lane - query k: lane L collects m = L (dlo) and
+                // m = L - 32 (dhi), both of which sit in lane (L + k) mod 32 at step k
+                const float vd = __shfl_sync(0xffffffffu, dz, (lane + k) & 31);
+                if (lane + k < 32) dlo += vd;
+                else dhi += vd;
+            }
         }
         pa[e >> 1] = pack_bf16x2(av[0], av[1]);
         pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
@@ -269,8 +276,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     kv_use++;
                 }
                 const int n_qt = (s.L + kTileM - 1) / kTileM;
+                int t_pf = 0;                              // next tile to prefetch into L2
                 for (int t = 0; ok && t < n_qt; t++) {
                     if (q_class<KIND>(s, t) == 0) continue;
+                    // keep the query tile after this one on its way into L2
+                    if (t_pf <= t) t_pf = t + 1;
+                    while (t_pf < n_qt && q_class<KIND>(s, t_pf) == 0) t_pf++;
+                    if (t_pf < n_qt) {
+                        for (int pn = 0; pn < kPanels; pn++) {
+                            tma_prefetch_2d(&tm_q, s.h * D + pn * 64, s.off0 + t_pf * kTileM);
+                            tma_prefetch_2d(&tm_dy, s.h * D + pn * 64, s.off0 + t_pf * kTileM);
+                        }
+                        t_pf++;
+                    }
                     const int st = q_use & 1;
                     ok = mbar_wait(&bars[kQEmpty0 + st], ((q_use >> 1) & 1) ^ 1, s_abort);
                     if (!ok) break;
@@ -428,7 +446,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int64_t* w_qts = s_qts + warp * 64;
         int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * 64;
         float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * 96;
-        float* w_gdiag = reinterpret_cast<float*>(sm + L::gdiag) + warp * 96;
         float* s_rth = reinterpret_cast<float*>(sm + L::rth);   // rab_time / 2
         const int nbm1 = p.nb - 1;
         int it_use = 0, s_use = 0, dz_use = 0, dq_use = 0, acc_use = 0;
@@ -507,7 +524,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
                                 w_diag[k] = masked ? kMaskedHalfBias
                                                    : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
-                                w_gdiag[k] = 0.f;
                             }
                         }
                         const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
@@ -531,9 +547,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tc_fence_after();
                 const int32_t a_j = (int32_t)(ts_j - kmin);
                 float acc = 0.f, acc_hi = 0.f;
+                // per-diagonal dz sums (delta = key - query = dmin + idx):
+                // d0 -> idx lane + 63, d1 -> idx lane + 31, d2 -> idx lane - 1
+                float d0 = 0.f, d1 = 0.f, d2 = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 2; c++) {
                     uint32_t pa[16], pz[16];
+                    float dlo = 0.f, dhi = 0.f;        // this chunk's diagonal sums
                     if (wcls == 0) {
 #pragma unroll
                         for (int e = 0; e < 16; e++) pa[e] = pz[e] = 0u;
@@ -544,10 +564,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_ld_wait(sv);
                         tmem_ld_wait(dp);
                         const float* dg = w_diag + lane + 63 - 32 * c;
-                        float* gg = w_gdiag + lane + 63 - 32 * c;
                         const int32_t* qr = w_qrel + 32 * c;
 #define HSTU_BWD_SPEC(PM_, TM_) \
-    bwd_block<PM_, TM_>(sv, dp, dg, gg, qr, a_j, tc.thr, c0, c1, s_rth, nbm1, p.inv_alpha, acc, acc_hi, s_grt, pa, pz)
+    bwd_block<PM_, TM_>(sv, dp, dg, dlo, dhi, qr, a_j, tc.thr, c0, c1, s_rth, nbm1, p.inv_alpha, acc, acc_hi, s_grt, pa, pz)
                         if (pm == kPosUniform && tm == kTimeUniform) HSTU_BWD_SPEC(kPosUniform, kTimeUniform);
                         else if (pm == kPosUniform && tm == kTimeTwo) HSTU_BWD_SPEC(kPosUniform, kTimeTwo);
                         else if (pm == kPosUniform && tm == kTimeBits) HSTU_BWD_SPEC(kPosUniform, kTimeBits);
@@ -578,12 +597,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                     av[f] = vis ? a * p.inv_alpha : 0.f;
                                     const float dz = vis ? __uint_as_float(dp[e + f]) * p.inv_alpha * gd : 0.f;
                                     zv[f] = dz;
-                                    if (pidx != cur_p) {
-                                        if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
-                                        cur_p = pidx;
-                                        acc_p = 0.f;
+                                    if (KIND == HSTU_KIND_CAUSAL) {
+                                        const int k = e + f;
+                                        const float vd = __shfl_sync(kFull, dz, (lane + k) & 31);
+                                        if (lane + k < 32) dlo += vd;
+                                        else dhi += vd;
+                                    } else {
+                                        if (pidx != cur_p) {
+                                            if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
+                                            cur_p = pidx;
+                                            acc_p = 0.f;
+                                        }
+                                        acc_p += dz;
                                     }
-                                    acc_p += dz;
                                     if (tb != cur_t) {
                                         if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
                                         cur_t = tb;
@@ -597,6 +623,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
                             if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
                         }
+                    }
+                    if (c == 0) {
+                        d0 += dlo;
+                        d1 += dhi;
+                    } else {
+                        d1 += dlo;
+                        d2 += dhi;
                     }
                     // A^T back into TMEM over the S^T columns this warp group has read
                     tmem_st16(tmem + lane_base + kSCol + 64 * g + 16 * c, pa);
@@ -623,15 +656,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             atomicAdd(&s_grt[tc.tb_lo], acc - acc_hi);
                         }
                     }
-                    if (pm == kPosDiag) {
-                        __syncwarp();
-                        const int dmin = ka - (i0 + 63);
-                        for (int k = lane; k < 95; k += 32) {
-                            const float v = w_gdiag[k];
-                            if (v != 0.f)
-                                atomicAdd(&s_grp[min(max(dmin + k, -(p.P - 1)), p.P - 1) + p.P - 1], v);
-                        }
-                    }
+                }
+                if (pm == kPosDiag || (pm < 0 && wcls != 0 && KIND == HSTU_KIND_CAUSAL)) {
+                    const int dmin = ka - (i0 + 63);
+                    const int np1 = p.P - 1;
+                    if (d0 != 0.f) atomicAdd(&s_grp[min(max(dmin + lane + 63, -np1), np1) + np1], d0);
+                    if (d1 != 0.f) atomicAdd(&s_grp[min(max(dmin + lane + 31, -np1), np1) + np1], d1);
+                    if (lane > 0 && d2 != 0.f) atomicAdd(&s_grp[min(max(dmin + lane - 1, -np1), np1) + np1], d2);
                 }
                 tmem_st_wait();
                 fence_proxy_async_smem();

@@ -242,8 +242,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     q_use++;
                 }
                 const int n_kt = (s.Lk + kTileN - 1) / kTileN;
+                int t_pf = 0;                              // next key tile to prefetch into L2
                 for (int t = 0; ok && t < n_kt; t++) {
                     if (kv_class<KIND>(s, t) == 0) continue;
+                    if (t_pf <= t) t_pf = t + 1;
+                    while (t_pf < n_kt && kv_class<KIND>(s, t_pf) == 0) t_pf++;
+                    if (t_pf < n_kt) {
+                        for (int pn = 0; pn < kPanels; pn++) {
+                            tma_prefetch_2d(&tm_k, s.h * D + pn * 64, s.kv0 + t_pf * kTileN);
+                            tma_prefetch_2d(&tm_v, s.h * D + pn * 64, s.kv0 + t_pf * kTileN);
+                        }
+                        t_pf++;
+                    }
                     const int y = s.kv0 + t * kTileN;
                     ok = mbar_wait(&bars[kKEmpty], (k_use & 1) ^ 1, s_abort);
                     if (!ok) break;
