@@ -21,9 +21,10 @@
 //          drained by the elementwise warps into an fp32 buffer with vector reductions.
 // Warps 0-7 elementwise (warp w owns TMEM lanes 32*(w%4)..+31 = key rows, and
 // query columns [64*(w/4), +64)), warp 8 producer (TMA), warp 9 MMA issuer.
-// rab gradients: shared-memory accumulators (run-length per thread for the time
-// bucket, one atomic per element for the position index, or a warp sum when the
-// bias is uniform over the warp's block), flushed to global memory at the end.
+// rab gradients: register sums per warp block (uniform bias), per-diagonal sums
+// gathered with warp shuffles (position), run-length sums per thread (time),
+// sent with fire-and-forget global reductions into this CTA's own partial row;
+// a small kernel sums the rows in a fixed order.
 // Every wait is bounded; a timeout sets the status word and the CTA exits cleanly.
 #include "ew_bias.cuh"
 #include "internal.h"
@@ -45,9 +46,7 @@ struct BwdSmem {
     static constexpr uint32_t dz = dy + kTile;                   // 128 keys x 128 queries bf16
     static constexpr uint32_t rp = dz + 128u * 128u * 2u;        // float[2*kMaxPos]
     static constexpr uint32_t rt = rp + 2u * kMaxPos * 4u;       // float[64]
-    static constexpr uint32_t grp = rt + kMaxTBuckets * 4u;      // float[2*kMaxPos]
-    static constexpr uint32_t grt = grp + 2u * kMaxPos * 4u;     // float[64]
-    static constexpr uint32_t rth = grt + kMaxTBuckets * 4u;     // float[64]: rab_time / 2
+    static constexpr uint32_t rth = rt + kMaxTBuckets * 4u;      // float[64]: rab_time / 2
     static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][64]
     static constexpr uint32_t qrel = qts + 8u * 64u * 8u;        // int32[8 warps][64]
     static constexpr uint32_t diag = qrel + 8u * 64u * 4u;       // float[8 warps][96]
@@ -116,7 +115,7 @@ template <int PM, int TM>
 __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* dg,
                                           float& dlo, float& dhi, const int32_t* qr, int32_t a_j, uint32_t thr,
                                           float c0, float c1, const float* rth, int nbm1, float inv_alpha,
-                                          float& acc, float& acc_hi, float* s_grt, uint32_t (&pa)[16],
+                                          float& acc, float& acc_hi, float* g_rt, uint32_t (&pa)[16],
                                           uint32_t (&pz)[16]) {
     const int lane = threadIdx.x & 31;
     int32_t q[32];
@@ -160,7 +159,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
             if (TM == kTimeTwo) acc_hi += hi_b ? dz : 0.f;
             if (TM == kTimeBits) {
                 if (tb != cur_t) {
-                    if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+                    if (cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
                     cur_t = tb;
                     acc_t = 0.f;
                 }
@@ -177,7 +176,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
         pa[e >> 1] = pack_bf16x2(av[0], av[1]);
         pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
     }
-    if (TM == kTimeBits && cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+    if (TM == kTimeBits && cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
 }
 
 template <int KIND, int D>
@@ -198,8 +197,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint8_t* sm = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     float* s_rp = reinterpret_cast<float*>(sm + L::rp);
     float* s_rt = reinterpret_cast<float*>(sm + L::rt);
-    float* s_grp = reinterpret_cast<float*>(sm + L::grp);
-    float* s_grt = reinterpret_cast<float*>(sm + L::grt);
+    // this CTA's rab-gradient partial sums (global, zeroed by the host, summed by rab_reduce)
+    float* g_rp = p.rab_part + (size_t)blockIdx.x * (2 * p.P - 1 + p.nb);
+    float* g_rt = g_rp + (2 * p.P - 1);
     int64_t* s_qts = reinterpret_cast<int64_t*>(sm + L::qts);
     int4* s_item = reinterpret_cast<int4*>(sm + L::item);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
@@ -208,13 +208,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int np = 2 * p.P - 1;
-    for (int i = tid; i < np; i += kThreads) {
-        s_rp[i] = p.rab_pos[i];
-        s_grp[i] = 0.f;
-    }
+    for (int i = tid; i < np; i += kThreads) s_rp[i] = p.rab_pos[i];
     for (int i = tid; i < p.nb; i += kThreads) {
         s_rt[i] = p.rab_time[i];
-        s_grt[i] = 0.f;
         reinterpret_cast<float*>(sm + L::rth)[i] = 0.5f * p.rab_time[i];
     }
     if (tid == 0) {
@@ -566,7 +562,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         const float* dg = w_diag + lane + 63 - 32 * c;
                         const int32_t* qr = w_qrel + 32 * c;
 #define HSTU_BWD_SPEC(PM_, TM_) \
-    bwd_block<PM_, TM_>(sv, dp, dg, dlo, dhi, qr, a_j, tc.thr, c0, c1, s_rth, nbm1, p.inv_alpha, acc, acc_hi, s_grt, pa, pz)
+    bwd_block<PM_, TM_>(sv, dp, dg, dlo, dhi, qr, a_j, tc.thr, c0, c1, s_rth, nbm1, p.inv_alpha, acc, acc_hi, g_rt, pa, pz)
                         if (pm == kPosUniform && tm == kTimeUniform) HSTU_BWD_SPEC(kPosUniform, kTimeUniform);
                         else if (pm == kPosUniform && tm == kTimeTwo) HSTU_BWD_SPEC(kPosUniform, kTimeTwo);
                         else if (pm == kPosUniform && tm == kTimeBits) HSTU_BWD_SPEC(kPosUniform, kTimeBits);
@@ -604,14 +600,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                         else dhi += vd;
                                     } else {
                                         if (pidx != cur_p) {
-                                            if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
+                                            if (cur_p >= 0 && acc_p != 0.f) red_add_f32(&g_rp[cur_p], acc_p);
                                             cur_p = pidx;
                                             acc_p = 0.f;
                                         }
                                         acc_p += dz;
                                     }
                                     if (tb != cur_t) {
-                                        if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+                                        if (cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
                                         cur_t = tb;
                                         acc_t = 0.f;
                                     }
@@ -620,8 +616,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 pa[e >> 1] = pack_bf16x2(av[0], av[1]);
                                 pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
                             }
-                            if (cur_p >= 0 && acc_p != 0.f) atomicAdd(&s_grp[cur_p], acc_p);
-                            if (cur_t >= 0 && acc_t != 0.f) atomicAdd(&s_grt[cur_t], acc_t);
+                            if (cur_p >= 0 && acc_p != 0.f) red_add_f32(&g_rp[cur_p], acc_p);
+                            if (cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
                         }
                     }
                     if (c == 0) {
@@ -649,20 +645,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         acc_hi += __shfl_xor_sync(kFull, acc_hi, o);
                     }
                     if (lane == 0) {
-                        if (pm == kPosUniform) atomicAdd(&s_grp[pidx_u], acc);
-                        if (tm == kTimeUniform) atomicAdd(&s_grt[tc.tb_lo], acc);
+                        if (pm == kPosUniform) red_add_f32(&g_rp[pidx_u], acc);
+                        if (tm == kTimeUniform) red_add_f32(&g_rt[tc.tb_lo], acc);
                         if (tm == kTimeTwo) {
-                            atomicAdd(&s_grt[tc.tb_hi], acc_hi);
-                            atomicAdd(&s_grt[tc.tb_lo], acc - acc_hi);
+                            red_add_f32(&g_rt[tc.tb_hi], acc_hi);
+                            red_add_f32(&g_rt[tc.tb_lo], acc - acc_hi);
                         }
                     }
                 }
                 if (pm == kPosDiag || (pm < 0 && wcls != 0 && KIND == HSTU_KIND_CAUSAL)) {
                     const int dmin = ka - (i0 + 63);
                     const int np1 = p.P - 1;
-                    if (d0 != 0.f) atomicAdd(&s_grp[min(max(dmin + lane + 63, -np1), np1) + np1], d0);
-                    if (d1 != 0.f) atomicAdd(&s_grp[min(max(dmin + lane + 31, -np1), np1) + np1], d1);
-                    if (lane > 0 && d2 != 0.f) atomicAdd(&s_grp[min(max(dmin + lane - 1, -np1), np1) + np1], d2);
+                    if (d0 != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + 63, -np1), np1) + np1], d0);
+                    if (d1 != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + 31, -np1), np1) + np1], d1);
+                    if (lane > 0 && d2 != 0.f) red_add_f32(&g_rp[min(max(dmin + lane - 1, -np1), np1) + np1], d2);
                 }
                 tmem_st_wait();
                 fence_proxy_async_smem();
@@ -738,11 +734,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    // rab gradients of this CTA
-    for (int i = tid; i < np; i += kThreads)
-        if (s_grp[i] != 0.f) atomicAdd(&p.d_rab_pos[i], s_grp[i]);
-    for (int i = tid; i < p.nb; i += kThreads)
-        if (s_grt[i] != 0.f) atomicAdd(&p.d_rab_time[i], s_grt[i]);
 }
 
 template <int KIND, int D>
@@ -773,7 +764,28 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
     }
 }
 
+// d_rab[i] = sum over CTAs of part[cta][i], in CTA order.
+__global__ void rab_reduce_kernel(const float* __restrict__ part, int n_part, int P, int nb,
+                                  float* __restrict__ d_rab_pos, float* __restrict__ d_rab_time) {
+    const int w = 2 * P - 1 + nb;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= w) return;
+    float s = 0.f;
+    for (int c = 0; c < n_part; c++) s += part[(size_t)c * w + i];
+    if (i < 2 * P - 1) d_rab_pos[i] = s;
+    else d_rab_time[i - (2 * P - 1)] = s;
+}
+
 }  // namespace
+
+cudaError_t launch_rab_reduce(const float* part, int n_part, int P, int nb, float* d_rab_pos,
+                              float* d_rab_time, cudaStream_t s) {
+    const int w = 2 * P - 1 + nb;
+    prof_begin(kProfRabReduce, s);
+    rab_reduce_kernel<<<(w + 127) / 128, 128, 0, s>>>(part, n_part, P, nb, d_rab_pos, d_rab_time);
+    prof_end(kProfRabReduce, s);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdy, const BwdParams& p,

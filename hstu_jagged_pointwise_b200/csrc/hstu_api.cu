@@ -117,7 +117,7 @@ int check_mask(const hstu_mask_spec* m, int* kind) {
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-    size_t items = 0, perm = 0, seq_base = 0, dy = 0, part = 0, dq_acc = 0, total = 0;
+    size_t items = 0, perm = 0, seq_base = 0, dy = 0, part = 0, dq_acc = 0, rab_part = 0, total = 0;
     long long max_items = 0;
     int n_part = 0;
 };
@@ -142,6 +142,8 @@ Layout attn_layout(const hstu_dims& d, int is_bwd) {
         if (d.dtype == HSTU_BF16) {
             L.dq_acc = off;                      // fp32 dQ accumulated across key tiles
             off = align_up(off + (size_t)d.T * D * 4, 256);
+            L.rab_part = off;                    // per-CTA rab gradient partial sums
+            off = align_up(off + (size_t)kMaxBwdCtas * (2 * d.n_pos - 1 + d.n_tbuckets) * 4, 256);
         }
     }
     L.total = off;
@@ -421,6 +423,11 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     float* dq_acc = at<float>(workspace, L.dq_acc);
     st = cuda_status(cudaMemsetAsync(dq_acc, 0, (size_t)d.T * D * sizeof(float), s));
     if (st != HSTU_OK) return st;
+    const int grid = di->sms < kMaxBwdCtas ? di->sms : kMaxBwdCtas;
+    const int rab_w = 2 * d.n_pos - 1 + d.n_tbuckets;
+    float* rab_part = at<float>(workspace, L.rab_part);
+    st = cuda_status(cudaMemsetAsync(rab_part, 0, (size_t)grid * rab_w * sizeof(float), s));
+    if (st != HSTU_OK) return st;
     BwdParams bp;
     memset(&bp, 0, sizeof(bp));
     bp.off = seq_offsets;
@@ -434,14 +441,15 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     bp.dq_acc = dq_acc;
     bp.dk = static_cast<__nv_bfloat16*>(dk);
     bp.dv = static_cast<__nv_bfloat16*>(dv);
-    bp.d_rab_pos = d_rab_pos;
-    bp.d_rab_time = d_rab_time;
+    bp.rab_part = rab_part;
     bp.H = d.H;
     bp.P = d.n_pos;
     bp.nb = d.n_tbuckets;
     bp.ld = D;
     bp.inv_alpha = 1.0f / d.alpha;
-    st = cuda_status(launch_attn_bwd_tc(kind, d.d_qk, tq, tk, tv, tdy, bp, di->sms, s));
+    st = cuda_status(launch_attn_bwd_tc(kind, d.d_qk, tq, tk, tv, tdy, bp, grid, s));
+    if (st != HSTU_OK) return st;
+    st = cuda_status(launch_rab_reduce(rab_part, grid, d.n_pos, d.n_tbuckets, d_rab_pos, d_rab_time, s));
     if (st != HSTU_OK) return st;
     return cuda_status(launch_f32_to_bf16(dq_acc, static_cast<__nv_bfloat16*>(dq), (long long)d.T * D, s));
 }

@@ -83,11 +83,12 @@ struct BwdParams {
     float* dq_acc;            // [T, H*d] fp32, zeroed before the launch
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
-    float* d_rab_pos;
-    float* d_rab_time;
+    float* rab_part;          // [grid][2P-1 + nb] per-CTA rab gradient partial sums, zeroed
     int H, P, nb, ld;
     float inv_alpha;
 };
+
+constexpr int kMaxBwdCtas = 1024;   // bound on the backward's persistent grid (workspace sizing)
 
 // Generic (CUDA-core, fp32 arithmetic) attention kernels' parameters.
 struct SimtParams {
@@ -137,7 +138,7 @@ struct LnParams {
 enum ProfKind {
     kProfSchedule = 0, kProfAttnFwdTc, kProfAttnFwdSimt, kProfLnFwd, kProfLnBwd, kProfLnBwdReduce,
     kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfDqConvert,
-    kProfKinds
+    kProfRabReduce, kProfKinds
 };
 void prof_begin(int kind, cudaStream_t s);
 void prof_end(int kind, cudaStream_t s);
@@ -153,6 +154,8 @@ cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
                                const CUtensorMap& tv, const CUtensorMap& tdy, const BwdParams& p,
                                int grid, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t s);
+cudaError_t launch_rab_reduce(const float* part, int n_part, int P, int nb, float* d_rab_pos,
+                              float* d_rab_time, cudaStream_t s);
 cudaError_t launch_ln_fwd(int dtype_f32, const LnParams& p, cudaStream_t s);
 cudaError_t launch_ln_bwd(int dtype_f32, const LnParams& p, cudaStream_t s);
 int ln_bwd_partials(long long T);
