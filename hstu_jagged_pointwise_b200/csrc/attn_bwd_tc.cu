@@ -127,56 +127,66 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
             q[4 * e] = v.x; q[4 * e + 1] = v.y; q[4 * e + 2] = v.z; q[4 * e + 3] = v.w;
         }
     }
-    int cur_t = -1;
-    float acc_t = 0.f;
+    // pass 1: independent per-element chains (no cross-lane operations)
+    float zf[32];
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        float av[2], zv[2];
+        float av[2];
 #pragma unroll
         for (int f = 0; f < 2; f++) {
             const int k = e + f;
             float hb = PM == kPosUniform ? c0 : dg[-k];
-            bool hi_b = false;
-            int tb = 0;
             if (TM == kTimeTwo) {
-                const uint32_t x = (uint32_t)abs(q[k] - a_j);
-                hi_b = x >= thr;
+                const bool hi_b = (uint32_t)abs(q[k] - a_j) >= thr;
                 if (PM == kPosUniform) hb = hi_b ? c1 : c0;
                 else hb += hi_b ? c1 : c0;
             } else if (TM == kTimeBits) {
-                const uint32_t x = (uint32_t)abs(q[k] - a_j);
-                tb = time_bucket_u32(x, nbm1);
-                hb += rth[tb];
+                hb += rth[time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1)];
             }
             const float h = fmaf(__uint_as_float(sv[k]), 0.5f, hb);
             const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
             const float a = 2.f * h * sg;
             const float gd = fmaf(a, 1.f - sg, sg);
             av[f] = a * inv_alpha;
-            const float dz = __uint_as_float(dp[k]) * inv_alpha * gd;
-            zv[f] = dz;
-            acc += dz;
-            if (TM == kTimeTwo) acc_hi += hi_b ? dz : 0.f;
-            if (TM == kTimeBits) {
-                if (tb != cur_t) {
-                    if (cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
-                    cur_t = tb;
-                    acc_t = 0.f;
-                }
-                acc_t += dz;
-            }
-            if (PM == kPosDiag) {
-                // diagonal m = key lane - query k: lane L collects m = L (dlo) and
-                // m = L - 32 (dhi), both of which sit in lane (L + k) mod 32 at step k
-                const float vd = __shfl_sync(0xffffffffu, dz, (lane + k) & 31);
-                if (lane + k < 32) dlo += vd;
-                else dhi += vd;
-            }
+            zf[k] = __uint_as_float(dp[k]) * inv_alpha * gd;
         }
         pa[e >> 1] = pack_bf16x2(av[0], av[1]);
-        pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
+        pz[e >> 1] = pack_bf16x2(zf[e], zf[e + 1]);
     }
-    if (TM == kTimeBits && cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
+    // pass 2: gradient bookkeeping on finished values
+#pragma unroll
+    for (int k = 0; k < 32; k++) acc += zf[k];
+    if (TM == kTimeTwo) {
+#pragma unroll
+        for (int k = 0; k < 32; k++) acc_hi += (uint32_t)abs(q[k] - a_j) >= thr ? zf[k] : 0.f;
+    }
+    if (TM == kTimeBits) {
+        // the bucket changes rarely along a row: run-length sums, flushed on change
+        int cur_t = time_bucket_u32((uint32_t)abs(q[0] - a_j), nbm1);
+        float acc_t = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; k++) {
+            const int tb = time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1);
+            if (tb != cur_t) {
+                red_add_f32(&g_rt[cur_t], acc_t);
+                cur_t = tb;
+                acc_t = 0.f;
+            }
+            acc_t += zf[k];
+        }
+        red_add_f32(&g_rt[cur_t], acc_t);
+    }
+    if (PM == kPosDiag) {
+        // diagonal m = key lane - query k: lane L collects m = L (dlo) and m = L - 32
+        // (dhi), both held by lane (L + k) mod 32 at step k
+#pragma unroll
+        for (int k = 0; k < 32; k++) {
+            const float vd = __shfl_sync(0xffffffffu, zf[k], (lane + k) & 31);
+            const bool lo = lane + k < 32;
+            dlo += lo ? vd : 0.f;
+            dhi += lo ? 0.f : vd;
+        }
+    }
 }
 
 template <int KIND, int D>
@@ -574,9 +584,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             // element by element (MTGR candidates, ragged edges, int64-wide times)
                             int cur_p = -1, cur_t = -1;
                             float acc_p = 0.f, acc_t = 0.f;
+                            float zf[32];
 #pragma unroll
                             for (int e = 0; e < 32; e += 2) {
-                                float av[2], zv[2];
+                                float av[2];
 #pragma unroll
                                 for (int f = 0; f < 2; f++) {
                                     const int ii = 32 * c + e + f;
@@ -592,13 +603,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                     const float gd = fmaf(a, 1.f - sg, sg);
                                     av[f] = vis ? a * p.inv_alpha : 0.f;
                                     const float dz = vis ? __uint_as_float(dp[e + f]) * p.inv_alpha * gd : 0.f;
-                                    zv[f] = dz;
-                                    if (KIND == HSTU_KIND_CAUSAL) {
-                                        const int k = e + f;
-                                        const float vd = __shfl_sync(kFull, dz, (lane + k) & 31);
-                                        if (lane + k < 32) dlo += vd;
-                                        else dhi += vd;
-                                    } else {
+                                    zf[e + f] = dz;
+                                    if (KIND != HSTU_KIND_CAUSAL) {
                                         if (pidx != cur_p) {
                                             if (cur_p >= 0 && acc_p != 0.f) red_add_f32(&g_rp[cur_p], acc_p);
                                             cur_p = pidx;
@@ -614,10 +620,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                     acc_t += dz;
                                 }
                                 pa[e >> 1] = pack_bf16x2(av[0], av[1]);
-                                pz[e >> 1] = pack_bf16x2(zv[0], zv[1]);
+                                pz[e >> 1] = pack_bf16x2(zf[e], zf[e + 1]);
                             }
                             if (cur_p >= 0 && acc_p != 0.f) red_add_f32(&g_rp[cur_p], acc_p);
                             if (cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
+                            if (KIND == HSTU_KIND_CAUSAL) {
+#pragma unroll
+                                for (int k = 0; k < 32; k++) {
+                                    const float vd = __shfl_sync(kFull, zf[k], (lane + k) & 31);
+                                    const bool lo = lane + k < 32;
+                                    dlo += lo ? vd : 0.f;
+                                    dhi += lo ? 0.f : vd;
+                                }
+                            }
                         }
                     }
                     if (c == 0) {
