@@ -10,17 +10,25 @@
 // A = SiLU(z) is recomputed from Q and K, never read from memory.
 //
 // One work item = (sequence, head, 128-key tile); the CTA loops over the
-// 128-query tiles that see the key tile.  Per query tile, five UMMAs:
-//   S^T  = K Q^T   -> TMEM [0,128)        (SS, both K-major)
-//   dP^T = V dY^T  -> TMEM [128,256)      (SS, both K-major)
-//   elementwise warps: bias, mask, sigmoid, A^T (bf16) -> TMEM over S^T,
-//                      dZ^T (bf16) -> shared memory (128-byte swizzle)
-//   dV  += A^T dY  -> TMEM [256,256+D)    (TS: A^T from TMEM, dY MN-major)
-//   dK  += dZ^T Q  -> TMEM [256+D,256+2D) (SS: dZ^T K-major, Q MN-major)
-//   dQ   = dZ K    -> TMEM [128,128+D)    (SS: dZ^T read MN-major, K MN-major),
-//          drained by the elementwise warps into an fp32 buffer with vector reductions.
-// Warps 0-7 elementwise (warp w owns TMEM lanes 32*(w%4)..+31 = key rows, and
-// query columns [64*(w/4), +64)), warp 8 producer (TMA), warp 9 MMA issuer.
+// 128-query tiles that see the key tile, each handled as two 64-query halves so
+// that the elementwise warps work on one half while the tensor core runs the
+// other half's products.  Per half h (TMEM columns; keys are TMEM lanes):
+//   S^T_h  = K Q_h^T    -> [64h, 64h+64)       (SS, both K-major, N = 64)
+//   dP^T_h = V dY_h^T   -> [128+64h, +64)      (SS, both K-major, N = 64)
+//   elementwise warps: bias, mask, sigmoid; A^T_h (bf16) back into the S^T_h
+//                      columns, dZ^T_h (bf16) into shared memory (128-byte swizzle)
+//   dV += A^T_h dY_h    -> [256, 256+D)        (TS: A^T from TMEM, dY MN-major)
+//   dK += dZ^T_h Q_h    -> [256+D, 256+2D)     (SS: dZ^T K-major, Q MN-major)
+//   dQ^T_h = K^T dZ^T_h -> [128+64h, +64)      (SS: K read MN-major, dZ^T MN-major;
+//          lanes = head dims), drained by the elementwise warps.
+// dY arrives pre-scaled by 1/(2 alpha) (the LayerNorm backward writes it so), which
+// turns the elementwise step into, with h = z/2 and t = tanh(h):
+//   SiLU(z) = h (1 + t),   2 SiLU'(z) = 1 + t + h (1 - t^2),
+//   dz = dP' * 2 SiLU'(z) with dP' = V dY'^T,   dV = 2 A_raw^T dY' (the 2 in the epilogue).
+// dQ^T leaves TMEM through registers and a per-warp shared-memory slab; a TMA
+// tensor reduce-add sends each slab to the fp32 accumulation buffer.
+// Warps 0-7 elementwise (warp w owns TMEM lanes 32*(w%4)..+31 and 32 of the
+// half's 64 columns, [32*(w/4), +32)), warp 8 producer (TMA), warp 9 MMA issuer.
 // rab gradients: register sums per warp block (uniform bias), per-diagonal sums
 // gathered with warp shuffles (position), run-length sums per thread (time),
 // sent with fire-and-forget global reductions into this CTA's own partial row;
@@ -38,30 +46,34 @@ using namespace ptx;
 template <int D>
 struct BwdSmem {
     static constexpr uint32_t kTile = 128u * D * 2u;            // one 128-row bf16 tile
+    static constexpr uint32_t kHalf = 64u * D * 2u;             // one 64-row bf16 tile
     static constexpr uint32_t k = 0;
     static constexpr uint32_t v = k + kTile;
-    static constexpr uint32_t q0 = v + kTile;
+    static constexpr uint32_t q0 = v + kTile;                    // Q double buffer (full tiles)
     static constexpr uint32_t q1 = q0 + kTile;
-    static constexpr uint32_t dy = q1 + kTile;
-    static constexpr uint32_t dz = dy + kTile;                   // 128 keys x 128 queries bf16
-    static constexpr uint32_t rp = dz + 128u * 128u * 2u;        // float[2*kMaxPos]
-    static constexpr uint32_t rt = rp + 2u * kMaxPos * 4u;       // float[64]
+    static constexpr uint32_t dy0 = q1 + kTile;                  // dY halves (rows 0-63, 64-127)
+    static constexpr uint32_t dy1 = dy0 + kHalf;
+    static constexpr uint32_t dz0 = dy1 + kHalf;                 // dZ^T halves: 128 keys x 64 queries
+    static constexpr uint32_t dz1 = dz0 + 128u * 64u * 2u;
+    static constexpr uint32_t stg = dz1 + 128u * 64u * 2u;       // float[8 warps][512]: dQ slabs
+    static constexpr uint32_t rt = stg + 8u * 512u * 4u;         // float[64]
     static constexpr uint32_t rth = rt + kMaxTBuckets * 4u;      // float[64]: rab_time / 2
-    static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][64]
-    static constexpr uint32_t qrel = qts + 8u * 64u * 8u;        // int32[8 warps][64]
-    static constexpr uint32_t diag = qrel + 8u * 64u * 4u;       // float[8 warps][96]
-    static constexpr uint32_t item = diag + 8u * 96u * 4u;       // int4[2]
-    static constexpr uint32_t bars = item + 2u * 16u;            // uint64[24]
-    static constexpr uint32_t tmem = bars + 24u * 8u;
+    static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][32]
+    static constexpr uint32_t qrel = qts + 8u * 32u * 8u;        // int32[8 warps][32]
+    static constexpr uint32_t diag = qrel + 8u * 32u * 4u;       // float[8 warps][64]
+    static constexpr uint32_t item = diag + 8u * 64u * 4u;       // int4[2]
+    static constexpr uint32_t bars = item + 2u * 16u;            // uint64[32]
+    static constexpr uint32_t tmem = bars + 32u * 8u;
     static constexpr uint32_t abort_flag = tmem + 4u;
-    static constexpr uint32_t bytes = abort_flag + 4u;
-    static constexpr uint32_t alloc = bytes + 1024u;
+    static constexpr uint32_t rp = abort_flag + 12u;             // float[2P-1], sized at launch
+    static constexpr uint32_t alloc(int P) { return rp + 8u * (uint32_t)P + 1024u; }
 };
 
 enum {
-    kKVFull = 0, kKVEmpty, kQFull0, kQFull1, kQEmpty0, kQEmpty1, kDYFull, kDYEmpty, kSFull, kPFull,
-    kDQFull, kDQDrained, kDZEmpty, kAccFull, kAccEmpty, kItFull0, kItFull1, kItEmpty0, kItEmpty1,
-    kDrain, kNumBars
+    kKVFull = 0, kKVEmpty, kQFull0, kQFull1, kQEmpty0, kQEmpty1, kDYFull0, kDYFull1, kDYEmpty0,
+    kDYEmpty1, kSFull0, kSFull1, kPFull0, kPFull1, kDQFull0, kDQFull1, kDQDrained0, kDQDrained1,
+    kDZEmpty0, kDZEmpty1, kAccFull, kAccEmpty, kItFull0, kItFull1, kItEmpty0, kItEmpty1, kDrain,
+    kNumBars
 };
 
 constexpr int kThreads = 320;
@@ -72,6 +84,7 @@ constexpr uint32_t kPCol = 128;
 constexpr uint32_t kVCol = 256;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kPanel = 128u * 128u;                         // 128 rows x 128 B
+constexpr uint32_t kHalfPanel = 64u * 128u;                      // 64 rows x 128 B
 
 struct KvItem {
     int b, n0, h, n_end;   // keys [n0, n_end) of sequence b, head h
@@ -107,14 +120,14 @@ __device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* a
     atomicOr(&p.ctrl->status, kStatusTimeout);
 }
 
-// One 32-column chunk of a dense block: keys in lanes, queries along the chunk.
-// dg / gg point at this lane's diagonal-row entry for the chunk's first query
-// (entries for later queries sit at decreasing addresses); qr holds the
-// chunk's 32-bit query times relative to the block's smallest key time.
+// One dense 32 x 32 block: keys in lanes, queries along the chunk.  dg points
+// at this lane's diagonal-row entry for the block's first query (later queries
+// sit at decreasing addresses); qr holds the block's 32-bit query times
+// relative to the warp's smallest key time.
 template <int PM, int TM>
 __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* dg,
                                           float& dlo, float& dhi, const int32_t* qr, int32_t a_j, uint32_t thr,
-                                          float c0, float c1, const float* rth, int nbm1, float inv_alpha,
+                                          float c0, float c1, const float* rth, int nbm1,
                                           float& acc, float& acc_hi, float* g_rt, uint32_t (&pa)[16],
                                           uint32_t (&pz)[16]) {
     const int lane = threadIdx.x & 31;
@@ -144,11 +157,10 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
                 hb += rth[time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1)];
             }
             const float h = fmaf(__uint_as_float(sv[k]), 0.5f, hb);
-            const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
-            const float a = 2.f * h * sg;
-            const float gd = fmaf(a, 1.f - sg, sg);
-            av[f] = a * inv_alpha;
-            zf[k] = __uint_as_float(dp[k]) * inv_alpha * gd;
+            const float th = tanh_approx(h);
+            av[f] = fmaf(h, th, h);                                        // SiLU(z)
+            const float g2 = fmaf(h, fmaf(-th, th, 1.f), th + 1.f);        // 2 SiLU'(z)
+            zf[k] = __uint_as_float(dp[k]) * g2;
         }
         pa[e >> 1] = pack_bf16x2(av[0], av[1]);
         pz[e >> 1] = pack_bf16x2(zf[e], zf[e + 1]);
@@ -193,40 +205,47 @@ template <int KIND, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dy,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using L = BwdSmem<D>;
     constexpr int kPanels = D / 64;
+    constexpr int kDqDims = D == 128 ? 32 : 16;     // dQ slab: head dims per warp
+    constexpr int kDqRows = 512 / kDqDims;          // dQ slab: queries (2 KB per warp)
     constexpr uint32_t kKCol = kVCol + D;
-    constexpr uint32_t kIdSS = idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T
-    constexpr uint32_t kIdTS = idesc_bf16_f32(128, D, 0, 1);      // dV: A tmem, B MN-major
-    constexpr uint32_t kIdKM = idesc_bf16_f32(128, D, 0, 1);      // dK: A K-major, B MN-major
-    constexpr uint32_t kIdMM = idesc_bf16_f32(128, D, 1, 1);      // dQ: A MN-major, B MN-major
+    constexpr uint32_t kIdSP = idesc_bf16_f32(128, 64, 0, 0);     // S^T_h, dP^T_h
+    constexpr uint32_t kIdV = idesc_bf16_f32(128, D, 0, 1);       // dV: A tmem, B MN-major
+    constexpr uint32_t kIdK = idesc_bf16_f32(128, D, 0, 1);       // dK: A K-major, B MN-major
+    constexpr uint32_t kIdQ = idesc_bf16_f32(D, 64, 1, 1);        // dQ^T_h: A, B MN-major
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* sm = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     float* s_rp = reinterpret_cast<float*>(sm + L::rp);
     float* s_rt = reinterpret_cast<float*>(sm + L::rt);
-    // this CTA's rab-gradient partial sums (global, zeroed by the host, summed by rab_reduce)
-    float* g_rp = p.rab_part + (size_t)blockIdx.x * (2 * p.P - 1 + p.nb);
-    float* g_rt = g_rp + (2 * p.P - 1);
+    float* s_rth = reinterpret_cast<float*>(sm + L::rth);
     int64_t* s_qts = reinterpret_cast<int64_t*>(sm + L::qts);
     int4* s_item = reinterpret_cast<int4*>(sm + L::item);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::tmem);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::abort_flag);
+    // this CTA's rab-gradient partial sums (global, zeroed by the host, summed by rab_reduce)
+    float* g_rp = p.rab_part + (size_t)blockIdx.x * (2 * p.P - 1 + p.nb);
+    float* g_rt = g_rp + (2 * p.P - 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int np = 2 * p.P - 1;
     for (int i = tid; i < np; i += kThreads) s_rp[i] = p.rab_pos[i];
     for (int i = tid; i < p.nb; i += kThreads) {
         s_rt[i] = p.rab_time[i];
-        reinterpret_cast<float*>(sm + L::rth)[i] = 0.5f * p.rab_time[i];
+        s_rth[i] = 0.5f * p.rab_time[i];
     }
     if (tid == 0) {
-        const uint32_t counts[kNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, kEwThreads, 1, kEwThreads, 1, 1,
-                                           kEwThreads, 1, 1, kEwThreads + 1, kEwThreads + 1, 1};
-        for (int i = 0; i < kNumBars; i++) mbar_init(&bars[i], counts[i]);
+        for (int i = 0; i < kNumBars; i++) {
+            uint32_t c = 1;
+            if (i == kPFull0 || i == kPFull1 || i == kDQDrained0 || i == kDQDrained1 || i == kAccEmpty)
+                c = kEwThreads;
+            if (i == kItEmpty0 || i == kItEmpty1) c = kEwThreads + 1;
+            mbar_init(&bars[i], c);
+        }
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -235,6 +254,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_dy);
+        prefetch_tmap(&tm_dq);
     }
     if (warp == 9) {
         tmem_alloc(s_tmem, kTmemCols);
@@ -247,7 +267,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (warp == 8) {
         // ============================================================ producer
-        int it_use = 0, kv_use = 0, q_use = 0, dy_use = 0;
+        int it_use = 0, kv_use = 0, q_use = 0, dy_use[2] = {0, 0};
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
@@ -282,16 +302,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     kv_use++;
                 }
                 const int n_qt = (s.L + kTileM - 1) / kTileM;
-                int t_pf = 0;                              // next tile to prefetch into L2
+                int t_pf = 0;                              // next query tile to prefetch into L2
                 for (int t = 0; ok && t < n_qt; t++) {
                     if (q_class<KIND>(s, t) == 0) continue;
-                    // keep the query tile after this one on its way into L2
                     if (t_pf <= t) t_pf = t + 1;
                     while (t_pf < n_qt && q_class<KIND>(s, t_pf) == 0) t_pf++;
                     if (t_pf < n_qt) {
                         for (int pn = 0; pn < kPanels; pn++) {
                             tma_prefetch_2d(&tm_q, s.h * D + pn * 64, s.off0 + t_pf * kTileM);
                             tma_prefetch_2d(&tm_dy, s.h * D + pn * 64, s.off0 + t_pf * kTileM);
+                            tma_prefetch_2d(&tm_dy, s.h * D + pn * 64, s.off0 + t_pf * kTileM + 64);
                         }
                         t_pf++;
                     }
@@ -303,13 +323,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tma_load_2d(sm + (st ? L::q1 : L::q0) + pn * kPanel, &tm_q, &bars[kQFull0 + st],
                                     s.h * D + pn * 64, s.off0 + t * kTileM);
                     q_use++;
-                    ok = mbar_wait(&bars[kDYEmpty], (dy_use & 1) ^ 1, s_abort);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&bars[kDYFull], L::kTile);
-                    for (int pn = 0; pn < kPanels; pn++)
-                        tma_load_2d(sm + L::dy + pn * kPanel, &tm_dy, &bars[kDYFull], s.h * D + pn * 64,
-                                    s.off0 + t * kTileM);
-                    dy_use++;
+                    for (int hh = 0; ok && hh < 2; hh++) {
+                        ok = mbar_wait(&bars[kDYEmpty0 + hh], (dy_use[hh] & 1) ^ 1, s_abort);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&bars[kDYFull0 + hh], L::kHalf);
+                        for (int pn = 0; pn < kPanels; pn++)
+                            tma_load_2d(sm + (hh ? L::dy1 : L::dy0) + pn * kHalfPanel, &tm_dy,
+                                        &bars[kDYFull0 + hh], s.h * D + pn * 64, s.off0 + t * kTileM + 64 * hh);
+                        dy_use[hh]++;
+                    }
                 }
             }
             ok = __shfl_sync(kFull, ok, 0);
@@ -317,26 +339,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (lane == 0) {
             if (!ok && !*s_abort) flag_timeout(p, s_abort);
             if (*s_abort) {
+                // drain the copies this warp issued (at most the latest one per buffer)
                 volatile int dummy = 0;
                 if (kv_use) mbar_wait(&bars[kKVFull], (kv_use - 1) & 1, &dummy);
-                if (q_use) {
-                    const int st = (q_use - 1) & 1;
-                    mbar_wait(&bars[kQFull0 + st], ((q_use - 1) >> 1) & 1, &dummy);
-                }
-                if (q_use > 1) {
-                    const int st = (q_use - 2) & 1;
-                    mbar_wait(&bars[kQFull0 + st], ((q_use - 2) >> 1) & 1, &dummy);
-                }
-                if (dy_use) mbar_wait(&bars[kDYFull], (dy_use - 1) & 1, &dummy);
+                for (int u = q_use - 2; u < q_use; u++)
+                    if (u >= 0) mbar_wait(&bars[kQFull0 + (u & 1)], (u >> 1) & 1, &dummy);
+                for (int hh = 0; hh < 2; hh++)
+                    if (dy_use[hh]) mbar_wait(&bars[kDYFull0 + hh], (dy_use[hh] - 1) & 1, &dummy);
             }
         }
     } else if (warp == 9) {
         // ============================================================ MMA issuer
-        int it_use = 0, kv_use = 0, q_use = 0, dy_use = 0, p_use = 0, dq_use = 0, acc_use = 0;
+        int it_use = 0, kv_use = 0, q_use = 0, acc_use = 0;
+        int dy_use[2] = {0, 0}, p_use[2] = {0, 0}, dq_use[2] = {0, 0};
         bool ok = true;
         const uint32_t aK = smem_u32(sm + L::k), aV = smem_u32(sm + L::v);
         const uint32_t aQ0 = smem_u32(sm + L::q0), aQ1 = smem_u32(sm + L::q1);
-        const uint32_t aDY = smem_u32(sm + L::dy), aDZ = smem_u32(sm + L::dz);
+        const uint32_t aDY[2] = {smem_u32(sm + L::dy0), smem_u32(sm + L::dy1)};
+        const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
         while (ok) {
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
@@ -366,61 +386,67 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (!ok) break;
                     q_use++;
                     tc_fence_after();
-                    // S^T = K Q^T
+                    // ---- S^T_h and dP^T_h for both halves
+                    for (int hh = 0; ok && hh < 2; hh++) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; kk++) {
-                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                        mma_ss(tmem + kSCol, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(aQ + off, 16, 1024),
-                               kIdSS, kk > 0 ? 1u : 0u);
-                    }
-                    ok = mbar_wait(&bars[kDYFull], dy_use & 1, s_abort);
-                    if (!ok) break;
-                    dy_use++;
-                    // dQ of the previous tile lives in the dP^T columns until drained
-                    ok = mbar_wait(&bars[kDQDrained], (dq_use & 1) ^ 1, s_abort);
-                    if (!ok) break;
-                    tc_fence_after();
-                    // dP^T = V dY^T
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; kk++) {
-                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                        mma_ss(tmem + kPCol, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(aDY + off, 16, 1024),
-                               kIdSS, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(&bars[kSFull]);
-                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort);
-                    if (!ok) break;
-                    p_use++;
-                    if (n_done == 0) {
-                        ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
+                        for (int kk = 0; kk < D / 16; kk++) {
+                            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                            mma_ss(tmem + kSCol + 64 * hh, sdesc_sw128(aK + off, 16, 1024),
+                                   sdesc_sw128(aQ + off + hh * kHalfPanel, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+                        }
+                        ok = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort);
+                        if (ok) ok = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort);
                         if (!ok) break;
-                    }
-                    tc_fence_after();
-                    // dV += A^T dY   (A^T from TMEM: queries 64g..64g+63 at columns 64g..64g+31)
+                        dy_use[hh]++;
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-                        const uint32_t acol = kSCol + 64 * (kk >> 2) + 8 * (kk & 3);
-                        mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY + kk * 2048, kPanel, 1024), kIdTS,
-                               (n_done > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; kk++) {
+                            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                            const uint32_t offh = (kk >> 2) * kHalfPanel + (kk & 3) * 32;
+                            mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aV + off, 16, 1024),
+                                   sdesc_sw128(aDY[hh] + offh, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+                        }
+                        tc_commit(&bars[kSFull0 + hh]);
                     }
-                    tc_commit(&bars[kDYEmpty]);
-                    // dK += dZ^T Q
+                    // ---- products that need the elementwise results, half by half
+                    for (int hh = 0; ok && hh < 2; hh++) {
+                        ok = mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort);
+                        if (!ok) break;
+                        p_use[hh]++;
+                        if (n_done == 0 && hh == 0) {
+                            ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
+                            if (!ok) break;
+                        }
+                        tc_fence_after();
+                        const bool first = n_done == 0 && hh == 0;
+                        // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys); first,
+                        // so that its drain overlaps the two products below
 #pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                        mma_ss(tmem + kKCol, sdesc_sw128(aDZ + off, 16, 1024),
-                               sdesc_sw128(aQ + kk * 2048, kPanel, 1024), kIdKM, (n_done > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 8; kk++) {
+                            mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aK + kk * 2048, kPanel, 1024),
+                                   sdesc_sw128(aDZ[hh] + kk * 2048, 16, 1024), kIdQ, kk > 0 ? 1u : 0u);
+                        }
+                        dq_use[hh]++;
+                        tc_commit(&bars[kDQFull0 + hh]);
+                        // dV += A^T_h dY'_h   (A^T_h: queries 32g.. at columns 64h + 32g .. +15)
+#pragma unroll
+                        for (int kk = 0; kk < 4; kk++) {
+                            const uint32_t acol = kSCol + 64 * hh + 32 * (kk >> 1) + 8 * (kk & 1);
+                            mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY[hh] + kk * 2048, kHalfPanel, 1024),
+                                   kIdV, (!first || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&bars[kDYEmpty0 + hh]);
+                        // dK += dZ^T_h Q_h
+#pragma unroll
+                        for (int kk = 0; kk < 4; kk++) {
+                            mma_ss(tmem + kKCol, sdesc_sw128(aDZ[hh] + kk * 32, 16, 1024),
+                                   sdesc_sw128(aQ + hh * kHalfPanel + kk * 2048, kPanel, 1024), kIdK,
+                                   (!first || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&bars[kDZEmpty0 + hh]);
                     }
+                    if (!ok) break;
                     tc_commit(&bars[kQEmpty0 + st]);
-                    // dQ = dZ K   (dZ^T read MN-major, K read MN-major)
-#pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-                        mma_ss(tmem + kPCol, sdesc_sw128(aDZ + kk * 2048, kPanel, 1024),
-                               sdesc_sw128(aK + kk * 2048, kPanel, 1024), kIdMM, kk > 0 ? 1u : 0u);
-                    }
-                    dq_use++;
-                    tc_commit(&bars[kDZEmpty]);
-                    tc_commit(&bars[kDQFull]);
                     if (t == last) tc_commit(&bars[kKVEmpty]);
                     n_done++;
                 }
@@ -445,16 +471,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     } else {
         // ============================================================ elementwise (warps 0-7)
         const int wq = warp & 3;                 // lane quarter: key rows 32*wq .. +31
-        const int g = warp >> 2;                 // query half: columns 64*g .. +63
+        const int g = warp >> 2;                 // column group: queries 32*g .. +31 of each half
         const int r = wq * 32 + lane;            // key row within the tile (TMEM lane)
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        const uint32_t aDZ = smem_u32(sm + L::dz);
-        int64_t* w_qts = s_qts + warp * 64;
-        int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * 64;
-        float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * 96;
-        float* s_rth = reinterpret_cast<float*>(sm + L::rth);   // rab_time / 2
+        const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
+        int64_t* w_qts = s_qts + warp * 32;
+        float* w_stg = reinterpret_cast<float*>(sm + L::stg) + warp * 512;
+        int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * 32;
+        float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * 64;
         const int nbm1 = p.nb - 1;
-        int it_use = 0, s_use = 0, dz_use = 0, dq_use = 0, acc_use = 0;
+        int it_use = 0, acc_use = 0;
+        int s_use[2] = {0, 0}, dz_use[2] = {0, 0}, dq_use[2] = {0, 0};
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
@@ -478,101 +505,82 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 kmax = max(kmax, (int64_t)__shfl_xor_sync(kFull, (long long)kmax, o));
                 warp_keys += __shfl_xor_sync(kFull, warp_keys, o);
             }
+            const int32_t a_j = (int32_t)(ts_j - kmin);
             const int n_qt = (s.L + kTileM - 1) / kTileM;
             int n_done = 0;
-            for (int t = 0; t < n_qt; t++) {
-                const int cls = q_class<KIND>(s, t);
-                if (cls == 0) continue;
-                const int i0 = t * kTileM + 64 * g;       // first query of this warp's columns
-                __syncwarp();
-                int64_t qmin = INT64_MAX, qmax = INT64_MIN;
+            for (int t = 0; ok && t < n_qt; t++) {
+                if (q_class<KIND>(s, t) == 0) continue;
+                for (int hh = 0; hh < 2; hh++) {
+                    const int i0 = t * kTileM + 64 * hh + 32 * g;   // first query of this warp's block
+                    __syncwarp();
+                    const int iq = i0 + lane;
+                    const int64_t tq = iq < s.L ? p.ts[s.off0 + iq] : 0;
+                    w_qts[lane] = tq;
+                    int64_t qmin = iq < s.L ? tq : INT64_MAX, qmax = iq < s.L ? tq : INT64_MIN;
 #pragma unroll
-                for (int e = 0; e < 2; e++) {
-                    const int ii = lane + 32 * e;
-                    const int i = i0 + ii;
-                    const int64_t ti = i < s.L ? p.ts[s.off0 + i] : 0;
-                    w_qts[ii] = ti;
-                    if (i < s.L) {
-                        qmin = min(qmin, ti);
-                        qmax = max(qmax, ti);
+                    for (int o = 16; o > 0; o >>= 1) {
+                        qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
+                        qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
                     }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
-                    qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
-                }
-                // ---- classify this warp's block: 32 keys x 64 queries
-                int wcls = 0;
-                if (warp_keys > 0 && i0 < s.L)
-                    wcls = tile_class(KIND, i0, min(i0 + 63, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
-                int pm = -1, tm = -1;            // -1 = element-by-element rules
-                float c0 = 0.f, c1 = 0.f;
-                int pidx_u = 0;
-                TimeClass tc;
-                tc.tb_lo = tc.tb_hi = 0;
-                tc.thr = 0;
-                const bool dense = wcls != 0 && warp_keys == 32 && i0 + 64 <= s.L &&
-                                   (KIND == HSTU_KIND_CAUSAL || wcls == 2);
-                if (dense) {
-                    tc = classify_time(kmin, kmax, qmin, qmax, p.nb);
-                    if (tc.mode >= 0) {
-                        tm = tc.mode;
-                        const int dmax = ka + 31 - i0, dmin = ka - (i0 + 63);   // j - i over the block
-                        if (wcls == 2 && dmax <= -(p.P - 1)) { pm = kPosUniform; pidx_u = 0; }
-                        else if (wcls == 2 && dmin >= p.P - 1) { pm = kPosUniform; pidx_u = 2 * p.P - 2; }
-                        else pm = kPosDiag;
-                        if (pm == kPosDiag) {
-                            // diagonal row: delta = j - i = dmin + k, k in [0, 95)
-                            const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
-                            for (int k = lane; k < 95; k += 32) {
-                                const int dl = dmin + k;
-                                const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
-                                w_diag[k] = masked ? kMaskedHalfBias
-                                                   : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
+                    // ---- classify this warp's block: 32 keys x 32 queries
+                    int wcls = 0;
+                    if (warp_keys > 0 && i0 < s.L)
+                        wcls = tile_class(KIND, i0, min(i0 + 31, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
+                    int pm = -1, tm = -1;                // -1 = element-by-element rules
+                    float c0 = 0.f, c1 = 0.f;
+                    int pidx_u = 0;
+                    TimeClass tc;
+                    tc.tb_lo = tc.tb_hi = 0;
+                    tc.thr = 0;
+                    const bool dense = wcls != 0 && warp_keys == 32 && i0 + 32 <= s.L &&
+                                       (KIND == HSTU_KIND_CAUSAL || wcls == 2);
+                    const int dmin = ka - (i0 + 31);     // smallest key - query of the block
+                    if (dense) {
+                        tc = classify_time(kmin, kmax, qmin, qmax, p.nb);
+                        if (tc.mode >= 0) {
+                            tm = tc.mode;
+                            const int dmax = ka + 31 - i0;
+                            if (wcls == 2 && dmax <= -(p.P - 1)) { pm = kPosUniform; pidx_u = 0; }
+                            else if (wcls == 2 && dmin >= p.P - 1) { pm = kPosUniform; pidx_u = 2 * p.P - 2; }
+                            else pm = kPosDiag;
+                            if (pm == kPosDiag) {
+                                // diagonal row: key - query = dmin + k, k in [0, 63)
+                                const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
+                                for (int k = lane; k < 63; k += 32) {
+                                    const int dl = dmin + k;
+                                    const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
+                                    w_diag[k] = masked ? kMaskedHalfBias
+                                                       : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
+                                }
                             }
-                        }
-                        const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
-                        if (tm == kTimeUniform) c0 = ph + s_rth[tc.tb_lo];
-                        else if (tm == kTimeTwo) { c0 = ph + s_rth[tc.tb_lo]; c1 = ph + s_rth[tc.tb_hi]; }
-                        else c0 = ph;
-                        if (tm != kTimeUniform) {
-                            const int32_t qa = (int32_t)(w_qts[lane] - kmin);
-                            const int32_t qb = (int32_t)(w_qts[lane + 32] - kmin);
-                            w_qrel[lane] = qa;
-                            w_qrel[lane + 32] = qb;
+                            const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
+                            if (tm == kTimeUniform) c0 = ph + s_rth[tc.tb_lo];
+                            else if (tm == kTimeTwo) { c0 = ph + s_rth[tc.tb_lo]; c1 = ph + s_rth[tc.tb_hi]; }
+                            else c0 = ph;
+                            if (tm != kTimeUniform) w_qrel[lane] = (int32_t)(tq - kmin);
                         }
                     }
-                }
-                __syncwarp();
-                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
-                if (ok) ok = mbar_wait(&bars[kDZEmpty], (dz_use & 1) ^ 1, s_abort);
-                if (!__all_sync(kFull, ok)) { ok = false; break; }
-                s_use++;
-                dz_use++;
-                tc_fence_after();
-                const int32_t a_j = (int32_t)(ts_j - kmin);
-                float acc = 0.f, acc_hi = 0.f;
-                // per-diagonal dz sums (delta = key - query = dmin + idx):
-                // d0 -> idx lane + 63, d1 -> idx lane + 31, d2 -> idx lane - 1
-                float d0 = 0.f, d1 = 0.f, d2 = 0.f;
-#pragma unroll 1
-                for (int c = 0; c < 2; c++) {
+                    __syncwarp();
+                    ok = mbar_wait(&bars[kSFull0 + hh], s_use[hh] & 1, s_abort);
+                    if (ok) ok = mbar_wait(&bars[kDZEmpty0 + hh], (dz_use[hh] & 1) ^ 1, s_abort);
+                    if (!__all_sync(kFull, ok)) { ok = false; break; }
+                    s_use[hh]++;
+                    dz_use[hh]++;
+                    tc_fence_after();
+                    float acc = 0.f, acc_hi = 0.f, dlo = 0.f, dhi = 0.f;
                     uint32_t pa[16], pz[16];
-                    float dlo = 0.f, dhi = 0.f;        // this chunk's diagonal sums
                     if (wcls == 0) {
 #pragma unroll
                         for (int e = 0; e < 16; e++) pa[e] = pz[e] = 0u;
                     } else {
                         uint32_t sv[32], dp[32];
-                        tmem_ld32(tmem + lane_base + kSCol + 64 * g + 32 * c, sv);
-                        tmem_ld32(tmem + lane_base + kPCol + 64 * g + 32 * c, dp);
+                        tmem_ld32(tmem + lane_base + kSCol + 64 * hh + 32 * g, sv);
+                        tmem_ld32(tmem + lane_base + kPCol + 64 * hh + 32 * g, dp);
                         tmem_ld_wait(sv);
                         tmem_ld_wait(dp);
-                        const float* dg = w_diag + lane + 63 - 32 * c;
-                        const int32_t* qr = w_qrel + 32 * c;
+                        const float* dg = w_diag + lane + 31;
 #define HSTU_BWD_SPEC(PM_, TM_) \
-    bwd_block<PM_, TM_>(sv, dp, dg, dlo, dhi, qr, a_j, tc.thr, c0, c1, s_rth, nbm1, p.inv_alpha, acc, acc_hi, g_rt, pa, pz)
+    bwd_block<PM_, TM_>(sv, dp, dg, dlo, dhi, w_qrel, a_j, tc.thr, c0, c1, s_rth, nbm1, acc, acc_hi, g_rt, pa, pz)
                         if (pm == kPosUniform && tm == kTimeUniform) HSTU_BWD_SPEC(kPosUniform, kTimeUniform);
                         else if (pm == kPosUniform && tm == kTimeTwo) HSTU_BWD_SPEC(kPosUniform, kTimeTwo);
                         else if (pm == kPosUniform && tm == kTimeBits) HSTU_BWD_SPEC(kPosUniform, kTimeBits);
@@ -590,20 +598,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 float av[2];
 #pragma unroll
                                 for (int f = 0; f < 2; f++) {
-                                    const int ii = 32 * c + e + f;
-                                    const int i = i0 + ii;
-                                    const int64_t ts_i = w_qts[ii];
+                                    const int k = e + f;
+                                    const int i = i0 + k;
+                                    const int64_t ts_i = w_qts[k];
                                     const bool vis = key_ok && i < s.L && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
                                     const int pidx = pos_index(token_pos(KIND, min(i, s.L - 1), s.S, s.R), pos_j, p.P);
                                     const int tb = time_bucket(ts_i, ts_j, p.nb);
-                                    const float h = fmaf(__uint_as_float(sv[e + f]), 0.5f,
-                                                         0.5f * s_rp[pidx] + s_rth[tb]);
-                                    const float sg = fmaf(0.5f, tanh_approx(h), 0.5f);
-                                    const float a = 2.f * h * sg;
-                                    const float gd = fmaf(a, 1.f - sg, sg);
-                                    av[f] = vis ? a * p.inv_alpha : 0.f;
-                                    const float dz = vis ? __uint_as_float(dp[e + f]) * p.inv_alpha * gd : 0.f;
-                                    zf[e + f] = dz;
+                                    const float h = fmaf(__uint_as_float(sv[k]), 0.5f, 0.5f * s_rp[pidx] + s_rth[tb]);
+                                    const float th = tanh_approx(h);
+                                    av[f] = vis ? fmaf(h, th, h) : 0.f;
+                                    const float g2 = fmaf(h, fmaf(-th, th, 1.f), th + 1.f);
+                                    const float dz = vis ? __uint_as_float(dp[k]) * g2 : 0.f;
+                                    zf[k] = dz;
                                     if (KIND != HSTU_KIND_CAUSAL) {
                                         if (pidx != cur_p) {
                                             if (cur_p >= 0 && acc_p != 0.f) red_add_f32(&g_rp[cur_p], acc_p);
@@ -635,72 +641,77 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                         }
                     }
-                    if (c == 0) {
-                        d0 += dlo;
-                        d1 += dhi;
-                    } else {
-                        d1 += dlo;
-                        d2 += dhi;
-                    }
-                    // A^T back into TMEM over the S^T columns this warp group has read
-                    tmem_st16(tmem + lane_base + kSCol + 64 * g + 16 * c, pa);
-                    // dZ^T into shared memory: row r, queries 64g+32c.. (128-byte swizzle)
-                    const uint32_t row_addr = aDZ + g * kPanel + r * 128;
+                    // A^T_h back into TMEM inside the S^T_h columns this warp has read
+                    tmem_st16(tmem + lane_base + kSCol + 64 * hh + 32 * g, pa);
+                    // dZ^T_h into shared memory: row r, queries 32g.. (128-byte swizzle)
+                    const uint32_t row_addr = aDZ[hh] + r * 128;
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        const uint32_t ch = (uint32_t)((4 * c + e) ^ (r & 7));
+                        const uint32_t ch = (uint32_t)((4 * g + e) ^ (r & 7));
                         st_shared_v4(row_addr + ch * 16, pz[4 * e], pz[4 * e + 1], pz[4 * e + 2], pz[4 * e + 3]);
                     }
-                }
-                // ---- rab gradients of the dense block
-                if (pm >= 0) {
+                    // ---- rab gradients of the block
+                    if (pm >= 0) {
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        acc += __shfl_xor_sync(kFull, acc, o);
-                        acc_hi += __shfl_xor_sync(kFull, acc_hi, o);
+                        for (int o = 16; o > 0; o >>= 1) {
+                            acc += __shfl_xor_sync(kFull, acc, o);
+                            acc_hi += __shfl_xor_sync(kFull, acc_hi, o);
+                        }
+                        if (lane == 0) {
+                            if (pm == kPosUniform) red_add_f32(&g_rp[pidx_u], acc);
+                            if (tm == kTimeUniform) red_add_f32(&g_rt[tc.tb_lo], acc);
+                            if (tm == kTimeTwo) {
+                                red_add_f32(&g_rt[tc.tb_hi], acc_hi);
+                                red_add_f32(&g_rt[tc.tb_lo], acc - acc_hi);
+                            }
+                        }
                     }
-                    if (lane == 0) {
-                        if (pm == kPosUniform) red_add_f32(&g_rp[pidx_u], acc);
-                        if (tm == kTimeUniform) red_add_f32(&g_rt[tc.tb_lo], acc);
-                        if (tm == kTimeTwo) {
-                            red_add_f32(&g_rt[tc.tb_hi], acc_hi);
-                            red_add_f32(&g_rt[tc.tb_lo], acc - acc_hi);
+                    if (pm == kPosDiag || (pm < 0 && wcls != 0 && KIND == HSTU_KIND_CAUSAL)) {
+                        const int np1 = p.P - 1;
+                        // dlo: key - query = dmin + lane + 31;  dhi: dmin + lane - 1
+                        if (dlo != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + 31, -np1), np1) + np1], dlo);
+                        if (lane > 0 && dhi != 0.f)
+                            red_add_f32(&g_rp[min(max(dmin + lane - 1, -np1), np1) + np1], dhi);
+                    }
+                    tmem_st_wait();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(&bars[kPFull0 + hh]);
+                }
+                if (!ok) break;
+                // ---- drain dQ^T of both halves (lanes = head dims, columns = queries)
+                for (int hh = 0; hh < 2; hh++) {
+                    ok = mbar_wait(&bars[kDQFull0 + hh], dq_use[hh] & 1, s_abort);
+                    if (!__all_sync(kFull, ok)) { ok = false; break; }
+                    dq_use[hh]++;
+                    tc_fence_after();
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + kPCol + 64 * hh + 32 * g, v);
+                    tmem_ld_wait(v);
+                    tc_fence_before();
+                    mbar_arrive(&bars[kDQDrained0 + hh]);      // the columns are free again
+                    // Slabs of kDqRows queries x kDqDims head dims, row-major, one TMA
+                    // reduce-add each.  M = 128 puts head dim 32*wq + lane in this lane; M = 64
+                    // puts head dims 16*wq .. +15 in the first 16 lanes of the lane quarter.
+                    // Queries past the sequence end carry exact zeros (their dZ is zero).
+                    const int qi = t * kTileM + 64 * hh + 32 * g;  // first query of the columns
+#pragma unroll
+                    for (int ps = 0; ps < 32 / kDqRows; ps++) {
+                        if (qi + ps * kDqRows >= s.L) break;
+                        if (lane == 0) bulk_wait_read_all();   // the previous slab has been read
+                        __syncwarp();
+                        if (D == 128 || lane < 16) {
+#pragma unroll
+                            for (int e = 0; e < kDqRows; e++) w_stg[e * kDqDims + lane] = __uint_as_float(v[ps * kDqRows + e]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_reduce_add_2d(&tm_dq, w_stg, s.h * D + wq * kDqDims, s.off0 + qi + ps * kDqRows);
+                            bulk_commit_group();
                         }
                     }
                 }
-                if (pm == kPosDiag || (pm < 0 && wcls != 0 && KIND == HSTU_KIND_CAUSAL)) {
-                    const int dmin = ka - (i0 + 63);
-                    const int np1 = p.P - 1;
-                    if (d0 != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + 63, -np1), np1) + np1], d0);
-                    if (d1 != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + 31, -np1), np1) + np1], d1);
-                    if (lane > 0 && d2 != 0.f) red_add_f32(&g_rp[min(max(dmin + lane - 1, -np1), np1) + np1], d2);
-                }
-                tmem_st_wait();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bars[kPFull]);
-                // drain dQ of this query tile (rows = queries, this group's half of the columns)
-                ok = mbar_wait(&bars[kDQFull], dq_use & 1, s_abort);
-                if (!__all_sync(kFull, ok)) { ok = false; break; }
-                dq_use++;
-                tc_fence_after();
-                const int qi = t * kTileM + r;            // query row held in this TMEM lane
-#pragma unroll 1
-                for (int c = 0; c < D / 64; c++) {
-                    uint32_t v[32];
-                    const int col = g * (D / 2) + 32 * c;
-                    tmem_ld32(tmem + lane_base + kPCol + col, v);
-                    tmem_ld_wait(v);
-                    if (qi < s.L) {
-                        float* dst = p.dq_acc + (size_t)(s.off0 + qi) * p.ld + (size_t)s.h * D + col;
-#pragma unroll
-                        for (int e = 0; e < 8; e++)
-                            red_add_v4(dst + 4 * e, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                       __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&bars[kDQDrained]);
                 n_done++;
             }
             if (!ok) break;
@@ -723,7 +734,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     uint32_t* pk = reinterpret_cast<uint32_t*>(wk);
 #pragma unroll
                     for (int e = 0; e < 16; e++) {
-                        pv[e] = n_done ? pack_bf16x2(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1])) : 0u;
+                        pv[e] = n_done ? pack_bf16x2(2.f * __uint_as_float(vv[2 * e]), 2.f * __uint_as_float(vv[2 * e + 1])) : 0u;
                         pk[e] = n_done ? pack_bf16x2(__uint_as_float(kv[2 * e]), __uint_as_float(kv[2 * e + 1])) : 0u;
                     }
                     const size_t o = (size_t)(s.off0 + j) * p.ld + (size_t)s.h * D + col;
@@ -741,6 +752,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_arrive(&bars[kItEmpty0 + slot]);
         }
         if (!ok && lane == 0 && !*s_abort) flag_timeout(p, s_abort);
+        if (lane == 0) bulk_wait_all();              // reduce-adds done before the CTA exits
     }
 
     tc_fence_before();
@@ -753,17 +765,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 template <int KIND, int D>
 cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdy, const BwdParams& p, int grid, cudaStream_t s) {
-    constexpr uint32_t smem = BwdSmem<D>::alloc;
+                       const CUtensorMap& tdy, const CUtensorMap& tdq, const BwdParams& p, int grid,
+                       cudaStream_t s) {
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<KIND, D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             BwdSmem<D>::alloc(kMaxPos));
         if (e != cudaSuccess) return e;
         configured = true;
     }
     prof_begin(kProfAttnBwdTc, s);
-    attn_bwd_tc_kernel<KIND, D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdy, p);
+    attn_bwd_tc_kernel<KIND, D><<<grid, kThreads, BwdSmem<D>::alloc(p.P), s>>>(tq, tk, tv, tdy, tdq, p);
     prof_end(kProfAttnBwdTc, s);
     return cudaGetLastError();
 }
@@ -803,10 +816,10 @@ cudaError_t launch_rab_reduce(const float* part, int n_part, int P, int nb, floa
 }
 
 cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const CUtensorMap& tdy, const BwdParams& p,
-                               int grid, cudaStream_t s) {
+                               const CUtensorMap& tv, const CUtensorMap& tdy, const CUtensorMap& tdq,
+                               const BwdParams& p, int grid, cudaStream_t s) {
 #define HSTU_BWD_CASE(K, DD) \
-    if (kind == K && d == DD) return launch_one<K, DD>(tq, tk, tv, tdy, p, grid, s);
+    if (kind == K && d == DD) return launch_one<K, DD>(tq, tk, tv, tdy, tdq, p, grid, s);
     HSTU_BWD_CASE(HSTU_KIND_CAUSAL, 128)
     HSTU_BWD_CASE(HSTU_KIND_CAUSAL, 64)
     HSTU_BWD_CASE(HSTU_KIND_MTGR, 128)

@@ -61,17 +61,31 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, cols] bf16 row-major; box = 64 columns (128 B, one swizzle row) x 128 rows.
-bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols) {
+// [rows, cols] bf16 row-major; box = 64 columns (128 B, one swizzle row) x box_rows rows.
+bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// [rows, cols] fp32 row-major, no swizzle; box = box_cols x box_rows (box_cols * 4 B a multiple of 16).
+bool make_tmap_f32(CUtensorMap* m, void* base, long long rows, long long cols, int box_cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -394,6 +408,8 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     lp.rstd = const_cast<float*>(ln_rstd);
     lp.g = d_o_pre;
     lp.dy = at<void>(workspace, L.dy);
+    // the tensor-core backward takes dY / (2 alpha): its elementwise step then needs no scaling
+    lp.dy_scale = d.dtype == HSTU_F32 ? 1.0f : 0.5f / d.alpha;
     lp.du = du;
     lp.part = at<float>(workspace, L.part);
     lp.n_part = L.n_part;
@@ -416,11 +432,13 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     }
     const DevInfo* di = dev_info();
     if (!di) return HSTU_ERR_CUDA;
-    CUtensorMap tq, tk, tv, tdy;
-    if (!make_tmap(&tq, q, d.T, D) || !make_tmap(&tk, k, d.T, D) || !make_tmap(&tv, v, d.T, D) ||
-        !make_tmap(&tdy, lp.dy, d.T, D))
-        return HSTU_ERR_CUDA;
+    CUtensorMap tq, tk, tv, tdy, tdq;
     float* dq_acc = at<float>(workspace, L.dq_acc);
+    const int dq_box_cols = d.d_qk == 128 ? 32 : 16;
+    if (!make_tmap(&tq, q, d.T, D) || !make_tmap(&tk, k, d.T, D) || !make_tmap(&tv, v, d.T, D) ||
+        !make_tmap(&tdy, lp.dy, d.T, D, 64) ||
+        !make_tmap_f32(&tdq, dq_acc, d.T, D, dq_box_cols, 512 / dq_box_cols))
+        return HSTU_ERR_CUDA;
     st = cuda_status(cudaMemsetAsync(dq_acc, 0, (size_t)d.T * D * sizeof(float), s));
     if (st != HSTU_OK) return st;
     const int grid = di->sms < kMaxBwdCtas ? di->sms : kMaxBwdCtas;
@@ -446,8 +464,7 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     bp.P = d.n_pos;
     bp.nb = d.n_tbuckets;
     bp.ld = D;
-    bp.inv_alpha = 1.0f / d.alpha;
-    st = cuda_status(launch_attn_bwd_tc(kind, d.d_qk, tq, tk, tv, tdy, bp, grid, s));
+    st = cuda_status(launch_attn_bwd_tc(kind, d.d_qk, tq, tk, tv, tdy, tdq, bp, grid, s));
     if (st != HSTU_OK) return st;
     st = cuda_status(launch_rab_reduce(rab_part, grid, d.n_pos, d.n_tbuckets, d_rab_pos, d_rab_time, s));
     if (st != HSTU_OK) return st;

@@ -80,12 +80,11 @@ struct BwdParams {
     const float* rab_time;
     const int4* items;
     Control* ctrl;
-    float* dq_acc;            // [T, H*d] fp32, zeroed before the launch
+    float* dq_acc;            // [T, H*d] fp32, zeroed before the launch (written via tm_dq)
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     float* rab_part;          // [grid][2P-1 + nb] per-CTA rab gradient partial sums, zeroed
     int H, P, nb, ld;
-    float inv_alpha;
 };
 
 constexpr int kMaxBwdCtas = 1024;   // bound on the backward's persistent grid (workspace sizing)
@@ -127,6 +126,7 @@ struct LnParams {
     // backward
     const void* g;
     void* dy;
+    float dy_scale;  // dY is written times this (1/(2 alpha) for the tensor-core backward)
     void* du;
     float* part;     // [n_blocks][2][D]
     int n_part;
@@ -150,9 +150,11 @@ cudaError_t launch_attn_fwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
 int attn_fwd_tc_ctas_per_sm(int kind, int d);
 cudaError_t launch_attn_fwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
+// tdy maps dY / (2 alpha) (bf16, 64-row boxes); tdq maps the fp32 dQ accumulator with
+// boxes of (32 dims x 16 rows) for d = 128 and (16 dims x 32 rows) for d = 64.
 cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const CUtensorMap& tdy, const BwdParams& p,
-                               int grid, cudaStream_t s);
+                               const CUtensorMap& tv, const CUtensorMap& tdy, const CUtensorMap& tdq,
+                               const BwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t s);
 cudaError_t launch_rab_reduce(const float* part, int n_part, int P, int nb, float* d_rab_pos,
                               float* d_rab_time, cudaStream_t s);

@@ -161,13 +161,14 @@ __global__ void __launch_bounds__(kWarps * 32) ln_bwd_kernel(LnParams p) {
         }
         m1 = warp_sum(m1) / p.D;
         m2 = warp_sum(m2) / p.D;
+        const float rs = rstd * p.dy_scale;
 #pragma unroll
         for (int k = 0; k < NC; k++) {
             const int vi = lane + 32 * k;
             if (vi < nvec) {
                 float dy[V];
 #pragma unroll
-                for (int e = 0; e < V; e++) dy[e] = rstd * (gx[k][e] - m1 - xh[k][e] * m2);
+                for (int e = 0; e < V; e++) dy[e] = rs * (gx[k][e] - m1 - xh[k][e] * m2);
                 Vec<T>::store(p.dy, base + (size_t)vi * V, dy);
             }
         }

@@ -122,12 +122,12 @@ def test_bf16_mtgr_forward_small():
     assert_bf16(out["o_pre"], o, "o_pre", st["o_pre"])
 
 
-@pytest.mark.parametrize("kind", ["causal", "mtgr"])
-def test_bf16_backward_small(kind):
+@pytest.mark.parametrize("kind,d", [("causal", 128), ("mtgr", 128), ("causal", 64), ("mtgr", 64)])
+def test_bf16_backward_small(kind, d):
     if kind == "causal":
-        w = W.make_causal([1, 127, 129, 300], H=2, d=128, seed=9, random_affine=True, with_grad=True)
+        w = W.make_causal([1, 127, 129, 300], H=2, d=d, seed=9, random_affine=True, with_grad=True)
     else:
-        w = W.make_mtgr([24, 2], [100, 190], [10, 0], [20, 70], H=2, d=128, seed=10, random_affine=True,
+        w = W.make_mtgr([24, 2], [100, 190], [10, 0], [20, 70], H=2, d=d, seed=10, random_affine=True,
                         with_grad=True)
     out, _, _ = run_layer(w, backward=True)
     ref = oracle.layer_bwd(w)
