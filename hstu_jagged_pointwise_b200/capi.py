@@ -29,7 +29,10 @@ EXPORTS = (
     "hstu_attn_workspace_bytes", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_mfalcon_workspace_bytes",
     "hstu_mfalcon_score", "hstu_debug_indices", "hstu_check_device_error", "hstu_status_string",
     "hstu_version", "hstu_profile_enable", "hstu_profile_read", "hstu_profile_kind_name",
+    "hstu_attn_fwd_noalloc",
 )
+
+NOALLOC_SCRATCH_BYTES = 4 << 20   # HSTU_NOALLOC_SCRATCH_BYTES
 
 
 class HstuDims(C.Structure):
@@ -69,6 +72,8 @@ def load():
     lib.hstu_attn_workspace_bytes.restype = S
     lib.hstu_attn_fwd.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec)] + [P] * 15 + [S, P]
     lib.hstu_attn_fwd.restype = C.c_int
+    lib.hstu_attn_fwd_noalloc.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec)] + [P] * 15 + [P]
+    lib.hstu_attn_fwd_noalloc.restype = C.c_int
     lib.hstu_attn_bwd.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec)] + [P] * 23 + [S, P]
     lib.hstu_attn_bwd.restype = C.c_int
     lib.hstu_mfalcon_workspace_bytes.argtypes = [C.POINTER(HstuMfalconDims), i32]

@@ -116,6 +116,42 @@ HSTU_API int hstu_attn_fwd(const hstu_dims* dims, const hstu_mask_spec* mask,
                   void* y, void* o_pre, float* ln_mean, float* ln_rstd,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Scratch built into the library for hstu_attn_fwd_noalloc (bytes, per device). */
+#define HSTU_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* hstu_attn_fwd without a caller workspace.  Library plumbing only: the pages
+ * describe no such call; it computes exactly what hstu_attn_fwd computes.
+ *
+ * For callers that must not allocate device memory on the call path, e.g. a
+ * serving loop that reserves all memory at start-up and treats any later
+ * allocation as an error, or a host thread without access to the framework's
+ * allocator.  The work list and status word live in a static device array of
+ * HSTU_NOALLOC_SCRATCH_BYTES inside the library's module; nothing is allocated.
+ *  - Size limit: returns HSTU_ERR_WORKSPACE, launching nothing, when
+ *    hstu_attn_workspace_bytes(dims, mask->kind, 0) exceeds
+ *    HSTU_NOALLOC_SCRATCH_BYTES (4 MiB: H * (ceil(T/128) + B) below about 262000);
+ *    use hstu_attn_fwd with a workspace for larger problems.
+ *  - First call per device: looks up the scratch address (cudaGetSymbolAddress),
+ *    which may load the library's module on that device.  Make the first call on
+ *    each device before any stream capture begins.
+ *  - Each call clears the scratch's control block (status word and work counter)
+ *    on `stream` before the forward's launches.
+ *  - One scratch per device: calls whose work can overlap on the device (other
+ *    streams, other host threads without ordering between them) race on it and
+ *    give undefined results.  Calls on one stream are ordered and safe.
+ *  - device_status: optional DEVICE int32 (NULL to skip) that receives, on
+ *    `stream`, the device status bits after the forward: 0 clean, 1 inputs out of
+ *    bounds (offsets, lengths, MTGR segments), 2 a bounded wait ran out; when
+ *    nonzero the outputs were not written.
+ * Other arguments, layouts and return codes as hstu_attn_fwd. */
+HSTU_API int hstu_attn_fwd_noalloc(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const void* q, const void* k, const void* v, const void* u,
+                  const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta,
+                  void* y, void* o_pre, float* ln_mean, float* ln_rstd,
+                  int32_t* device_status, void* stream);
+
 /* Backward of hstu_attn_fwd for the upstream gradient d_o_pre [T, H*d_v].
  * The A = SiLU(z) matrix is recomputed, never stored.
  * Out: dq, dk [T, H*d_qk]; dv, du [T, H*d_v] (element type dims.dtype);

@@ -18,7 +18,7 @@ def header_functions():
 
 def test_exports_match_header():
     names = header_functions()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     assert set(names) == set(capi.EXPORTS)
     for n in names:
         assert hasattr(capi.LIB, n), n
@@ -111,3 +111,17 @@ def test_debug_indices_rejects_bad_arguments():
                                        None) == capi.HSTU_ERR_INVALID_ARG
     assert capi.LIB.hstu_debug_indices(0, 0, None, None, None, None, 256, 64, None, None, None, None,
                                        None) == capi.HSTU_OK
+
+
+def test_fwd_noalloc_rejects_oversized_problems_on_the_host():
+    """The built-in scratch has a fixed size; larger problems are refused before any launch."""
+    from hstu_jagged_pointwise_b200 import ops
+    import torch
+    dims = ops.make_dims(T=1 << 30, B=1, H=8, d=128, dtype=torch.bfloat16, alpha=1.0, max_seq_len=1 << 18)
+    mask = ops.make_mask("causal")
+    need = capi.LIB.hstu_attn_workspace_bytes(C.byref(dims), capi.HSTU_MASK_CAUSAL, 0)
+    assert need > capi.NOALLOC_SCRATCH_BYTES
+    st = capi.LIB.hstu_attn_fwd_noalloc(C.byref(dims), C.byref(mask), *([None] * 15), None)
+    assert st == capi.HSTU_ERR_WORKSPACE
+    st = capi.LIB.hstu_attn_fwd_noalloc(None, C.byref(mask), *([None] * 15), None)
+    assert st == capi.HSTU_ERR_INVALID_ARG
