@@ -120,19 +120,21 @@ __device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* a
     atomicOr(&p.ctrl->status, kStatusTimeout);
 }
 
-// One dense 32 x 32 block: keys in lanes, queries along the chunk.  dg points
-// at this lane's diagonal-row entry for the block's first query (later queries
-// sit at decreasing addresses); qr holds the block's 32-bit query times
-// relative to the warp's smallest key time.
-template <int PM, int TM>
+// One dense 32 x 32 block: keys in lanes, queries along the chunk.  dg points at
+// this lane's diagonal-row entry for the block's first query (later queries sit at
+// decreasing addresses); the row holds half the position bias, the causal mask and,
+// when the block's time bucket is uniform, half the time bias.  TV: the bucket varies
+// inside the block and is computed per element from qr, the block's 32-bit query
+// times relative to the warp's smallest key time.  Two variants only, so that the
+// elementwise code stays small enough for the instruction cache.
+template <bool TV>
 __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* dg,
-                                          float& dlo, float& dhi, const int32_t* qr, int32_t a_j, uint32_t thr,
-                                          float c0, float c1, const float* rth, int nbm1,
-                                          float& acc, float& acc_hi, float* g_rt, uint32_t (&pa)[16],
-                                          uint32_t (&pz)[16]) {
+                                          bool pos_diag, float& dlo, float& dhi, const int32_t* qr, int32_t a_j,
+                                          const float* rth, int nbm1, float& acc, float* g_rt,
+                                          uint32_t (&pa)[16], uint32_t (&pz)[16]) {
     const int lane = threadIdx.x & 31;
     int32_t q[32];
-    if (TM != kTimeUniform) {
+    if (TV) {
         const int4* q4 = reinterpret_cast<const int4*>(qr);
 #pragma unroll
         for (int e = 0; e < 8; e++) {
@@ -148,14 +150,8 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
 #pragma unroll
         for (int f = 0; f < 2; f++) {
             const int k = e + f;
-            float hb = PM == kPosUniform ? c0 : dg[-k];
-            if (TM == kTimeTwo) {
-                const bool hi_b = (uint32_t)abs(q[k] - a_j) >= thr;
-                if (PM == kPosUniform) hb = hi_b ? c1 : c0;
-                else hb += hi_b ? c1 : c0;
-            } else if (TM == kTimeBits) {
-                hb += rth[time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1)];
-            }
+            float hb = dg[-k];
+            if (TV) hb += rth[time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1)];
             const float h = fmaf(__uint_as_float(sv[k]), 0.5f, hb);
             const float th = tanh_approx(h);
             av[f] = fmaf(h, th, h);                                        // SiLU(z)
@@ -168,11 +164,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
     // pass 2: gradient bookkeeping on finished values
 #pragma unroll
     for (int k = 0; k < 32; k++) acc += zf[k];
-    if (TM == kTimeTwo) {
-#pragma unroll
-        for (int k = 0; k < 32; k++) acc_hi += (uint32_t)abs(q[k] - a_j) >= thr ? zf[k] : 0.f;
-    }
-    if (TM == kTimeBits) {
+    if (TV) {
         // the bucket changes rarely along a row: run-length sums, flushed on change
         int cur_t = time_bucket_u32((uint32_t)abs(q[0] - a_j), nbm1);
         float acc_t = 0.f;
@@ -188,7 +180,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
         }
         red_add_f32(&g_rt[cur_t], acc_t);
     }
-    if (PM == kPosDiag) {
+    if (pos_diag) {
         // diagonal m = key lane - query k: lane L collects m = L (dlo) and m = L - 32
         // (dhi), both held by lane (L + k) mod 32 at step k
 #pragma unroll
@@ -527,7 +519,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (warp_keys > 0 && i0 < s.L)
                         wcls = tile_class(KIND, i0, min(i0 + 31, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
                     int pm = -1, tm = -1;                // -1 = element-by-element rules
-                    float c0 = 0.f, c1 = 0.f;
                     int pidx_u = 0;
                     TimeClass tc;
                     tc.tb_lo = tc.tb_hi = 0;
@@ -543,20 +534,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             if (wcls == 2 && dmax <= -(p.P - 1)) { pm = kPosUniform; pidx_u = 0; }
                             else if (wcls == 2 && dmin >= p.P - 1) { pm = kPosUniform; pidx_u = 2 * p.P - 2; }
                             else pm = kPosDiag;
-                            if (pm == kPosDiag) {
-                                // diagonal row: key - query = dmin + k, k in [0, 63)
-                                const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
-                                for (int k = lane; k < 63; k += 32) {
-                                    const int dl = dmin + k;
-                                    const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
-                                    w_diag[k] = masked ? kMaskedHalfBias
-                                                       : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
-                                }
+                            // diagonal row: key - query = dmin + k, k in [0, 63); constant when
+                            // the position index is clamped across the whole block
+                            const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
+                            for (int k = lane; k < 63; k += 32) {
+                                const int dl = dmin + k;
+                                const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
+                                w_diag[k] = masked ? kMaskedHalfBias
+                                                   : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
                             }
-                            const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
-                            if (tm == kTimeUniform) c0 = ph + s_rth[tc.tb_lo];
-                            else if (tm == kTimeTwo) { c0 = ph + s_rth[tc.tb_lo]; c1 = ph + s_rth[tc.tb_hi]; }
-                            else c0 = ph;
                             if (tm != kTimeUniform) w_qrel[lane] = (int32_t)(tq - kmin);
                         }
                     }
@@ -567,7 +553,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     s_use[hh]++;
                     dz_use[hh]++;
                     tc_fence_after();
-                    float acc = 0.f, acc_hi = 0.f, dlo = 0.f, dhi = 0.f;
+                    float acc = 0.f, dlo = 0.f, dhi = 0.f;
                     uint32_t pa[16], pz[16];
                     if (wcls == 0) {
 #pragma unroll
@@ -579,15 +565,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_ld_wait(sv);
                         tmem_ld_wait(dp);
                         const float* dg = w_diag + lane + 31;
-#define HSTU_BWD_SPEC(PM_, TM_) \
-    bwd_block<PM_, TM_>(sv, dp, dg, dlo, dhi, w_qrel, a_j, tc.thr, c0, c1, s_rth, nbm1, acc, acc_hi, g_rt, pa, pz)
-                        if (pm == kPosUniform && tm == kTimeUniform) HSTU_BWD_SPEC(kPosUniform, kTimeUniform);
-                        else if (pm == kPosUniform && tm == kTimeTwo) HSTU_BWD_SPEC(kPosUniform, kTimeTwo);
-                        else if (pm == kPosUniform && tm == kTimeBits) HSTU_BWD_SPEC(kPosUniform, kTimeBits);
-                        else if (pm == kPosDiag && tm == kTimeUniform) HSTU_BWD_SPEC(kPosDiag, kTimeUniform);
-                        else if (pm == kPosDiag && tm == kTimeTwo) HSTU_BWD_SPEC(kPosDiag, kTimeTwo);
-                        else if (pm == kPosDiag && tm == kTimeBits) HSTU_BWD_SPEC(kPosDiag, kTimeBits);
-#undef HSTU_BWD_SPEC
+                        if (tm == kTimeUniform)
+                            bwd_block<false>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
+                        else if (tm >= 0)
+                            bwd_block<true>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
                         else {
                             // element by element (MTGR candidates, ragged edges, int64-wide times)
                             int cur_p = -1, cur_t = -1;
@@ -651,19 +632,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         st_shared_v4(row_addr + ch * 16, pz[4 * e], pz[4 * e + 1], pz[4 * e + 2], pz[4 * e + 3]);
                     }
                     // ---- rab gradients of the block
-                    if (pm >= 0) {
+                    if (pm == kPosUniform || tm == kTimeUniform) {
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) {
-                            acc += __shfl_xor_sync(kFull, acc, o);
-                            acc_hi += __shfl_xor_sync(kFull, acc_hi, o);
-                        }
+                        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
                         if (lane == 0) {
                             if (pm == kPosUniform) red_add_f32(&g_rp[pidx_u], acc);
                             if (tm == kTimeUniform) red_add_f32(&g_rt[tc.tb_lo], acc);
-                            if (tm == kTimeTwo) {
-                                red_add_f32(&g_rt[tc.tb_hi], acc_hi);
-                                red_add_f32(&g_rt[tc.tb_lo], acc - acc_hi);
-                            }
                         }
                     }
                     if (pm == kPosDiag || (pm < 0 && wcls != 0 && KIND == HSTU_KIND_CAUSAL)) {
