@@ -104,14 +104,18 @@ __device__ __forceinline__ void flag_timeout(const FwdParams& p, volatile int* a
 }
 
 // One 32-column chunk of a dense block: rows in lanes, keys along the chunk.
-// dg points at this lane's diagonal-row entry for the chunk's first key;
-// cr holds the chunk's 32-bit key times relative to the tile's smallest one.
-template <int PM, int TM>
+// BM = kBiasConst: one bias c0 for the whole block; kBiasRow: bias from the
+// diagonal row (dg points at this lane's entry for the chunk's first key);
+// kBiasRowTime: diagonal row plus a per-element time bucket from cr, the chunk's
+// 32-bit key times relative to the tile's smallest one.  Three variants only, so
+// that the elementwise code stays small enough for the instruction cache.
+enum { kBiasConst = 0, kBiasRow = 1, kBiasRowTime = 2 };
+
+template <int BM>
 __device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* dg, const int32_t* cr, int32_t a_i,
-                                          uint32_t thr, float c0, float c1, const float* rth, int nbm1,
-                                          uint32_t (&pk)[16]) {
+                                          float c0, const float* rth, int nbm1, uint32_t (&pk)[16]) {
     int32_t b[32];
-    if (TM != kTimeUniform) {
+    if (BM == kBiasRowTime) {
         const int4* b4 = reinterpret_cast<const int4*>(cr);
 #pragma unroll
         for (int e = 0; e < 8; e++) {
@@ -125,14 +129,8 @@ __device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* 
 #pragma unroll
         for (int f = 0; f < 2; f++) {
             const int k = e + f;
-            float hb = PM == kPosUniform ? c0 : dg[k];
-            if (TM == kTimeTwo) {
-                const bool hi_b = (uint32_t)abs(b[k] - a_i) >= thr;
-                if (PM == kPosUniform) hb = hi_b ? c1 : c0;
-                else hb += hi_b ? c1 : c0;
-            } else if (TM == kTimeBits) {
-                hb += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
-            }
+            float hb = BM == kBiasConst ? c0 : dg[k];
+            if (BM == kBiasRowTime) hb += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
             const float h = fmaf(__uint_as_float(v[k]), 0.5f, hb);
             pv[f] = fmaf(h, tanh_approx(h), h);
         }
@@ -425,7 +423,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 // ---- classify this warp's block: 32 rows x 128 columns
                 int pm = -1, tm = -1;
-                float c0 = 0.f, c1 = 0.f;
+                float c0 = 0.f;
                 TimeClass tc;
                 tc.tb_lo = tc.tb_hi = 0;
                 tc.thr = 0;
@@ -448,21 +446,20 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     else if (KIND != HSTU_KIND_MFALCON) pm = kPosDiag;
                     if (pm >= 0 && tc.mode >= 0) {
                         tm = tc.mode;
-                        if (pm == kPosDiag) {
-                            // diagonal row: delta = j - i = (n0 - r0 - 31) + k, k in [0, 159)
+                        const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
+                        if (pm == kPosUniform && tm == kTimeUniform) {
+                            c0 = 0.5f * s_rp[pidx_u] + tadd;
+                        } else {
+                            // diagonal row: delta = j - i = (n0 - r0 - 31) + k, k in [0, 159);
+                            // constant when the position index is clamped across the block
                             const int d0 = n0 - r0 - 31;
-                            const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
                             for (int k = lane; k < 159; k += 32) {
                                 const int dl = d0 + k;
                                 const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
-                                w_diag[k] = masked ? kMaskedHalfBias
-                                                   : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
+                                const int pi = pm == kPosUniform ? pidx_u : min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1;
+                                w_diag[k] = masked ? kMaskedHalfBias : 0.5f * s_rp[pi] + tadd;
                             }
                         }
-                        const float ph = pm == kPosUniform ? 0.5f * s_rp[pidx_u] : 0.f;
-                        if (tm == kTimeUniform) c0 = ph + s_rth[tc.tb_lo];
-                        else if (tm == kTimeTwo) { c0 = ph + s_rth[tc.tb_lo]; c1 = ph + s_rth[tc.tb_hi]; }
-                        else c0 = ph;
                     } else {
                         pm = -1;
                     }
@@ -490,14 +487,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     uint32_t pk[16];
                     const float* dg = w_diag + 31 - lane + 32 * c;
                     const int32_t* cr = w_crel + 32 * c;
-#define HSTU_FWD_SPEC(PM_, TM_) fwd_block<PM_, TM_>(v, dg, cr, a_i, tc.thr, c0, c1, s_rth, nbm1, pk)
-                    if (pm == kPosUniform && tm == kTimeUniform) HSTU_FWD_SPEC(kPosUniform, kTimeUniform);
-                    else if (pm == kPosUniform && tm == kTimeTwo) HSTU_FWD_SPEC(kPosUniform, kTimeTwo);
-                    else if (pm == kPosUniform && tm == kTimeBits) HSTU_FWD_SPEC(kPosUniform, kTimeBits);
-                    else if (pm == kPosDiag && tm == kTimeUniform) HSTU_FWD_SPEC(kPosDiag, kTimeUniform);
-                    else if (pm == kPosDiag && tm == kTimeTwo) HSTU_FWD_SPEC(kPosDiag, kTimeTwo);
-                    else if (pm == kPosDiag && tm == kTimeBits) HSTU_FWD_SPEC(kPosDiag, kTimeBits);
-#undef HSTU_FWD_SPEC
+                    if (pm == kPosUniform && tm == kTimeUniform) fwd_block<kBiasConst>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                    else if (pm >= 0 && tm == kTimeUniform) fwd_block<kBiasRow>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                    else if (pm >= 0 && tm >= 0) fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else {
                         // element by element: MTGR candidates, ragged key tiles, int64-wide time spans
                         float pv[32];
