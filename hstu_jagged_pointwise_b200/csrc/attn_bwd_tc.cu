@@ -49,14 +49,14 @@ struct BwdSmem {
     static constexpr uint32_t kHalf = 64u * D * 2u;             // one 64-row bf16 tile
     static constexpr uint32_t k = 0;
     static constexpr uint32_t v = k + kTile;
-    static constexpr uint32_t q0 = v + kTile;                    // Q double buffer (full tiles)
-    static constexpr uint32_t q1 = q0 + kTile;
-    static constexpr uint32_t dy0 = q1 + kTile;                  // dY halves (rows 0-63, 64-127)
+    static constexpr uint32_t q0 = v + kTile;                    // Q halves (rows 0-63, 64-127)
+    static constexpr uint32_t q1 = q0 + kHalf;
+    static constexpr uint32_t dy0 = q1 + kHalf;                  // dY halves (rows 0-63, 64-127)
     static constexpr uint32_t dy1 = dy0 + kHalf;
     static constexpr uint32_t dz0 = dy1 + kHalf;                 // dZ^T halves: 128 keys x 64 queries
     static constexpr uint32_t dz1 = dz0 + 128u * 64u * 2u;
-    static constexpr uint32_t stg = dz1 + 128u * 64u * 2u;       // float[8 warps][512]: dQ slabs
-    static constexpr uint32_t rt = stg + 8u * 512u * 4u;         // float[64]
+    static constexpr uint32_t stg = dz1 + 128u * 64u * 2u;       // float[8 warps][1024]: dQ slabs
+    static constexpr uint32_t rt = stg + 8u * 1024u * 4u;        // float[64]
     static constexpr uint32_t rth = rt + kMaxTBuckets * 4u;      // float[64]: rab_time / 2
     static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][32]
     static constexpr uint32_t qrel = qts + 8u * 32u * 8u;        // int32[8 warps][32]
@@ -113,6 +113,14 @@ __device__ __forceinline__ int q_class(const KvItem& s, int t) {
     const int qa = t * kTileM;
     const int qb = min(qa + kTileM - 1, s.L - 1);
     return tile_class(KIND, qa, qb, s.n0, s.n_end - 1, s.S, s.R);
+}
+
+// first query tile after t that sees the item's keys, n_qt when none
+template <int KIND>
+__device__ __forceinline__ int next_visible(const KvItem& s, int t, int n_qt) {
+    for (t++; t < n_qt; t++)
+        if (q_class<KIND>(s, t) != 0) break;
+    return t;
 }
 
 __device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* abort_flag) {
@@ -201,7 +209,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     using L = BwdSmem<D>;
     constexpr int kPanels = D / 64;
     constexpr int kDqDims = D == 128 ? 32 : 16;     // dQ slab: head dims per warp
-    constexpr int kDqRows = 512 / kDqDims;          // dQ slab: queries (2 KB per warp)
+    constexpr int kDqRows = 32;                     // dQ slab: queries (4 KB / 2 KB per warp)
     constexpr uint32_t kKCol = kVCol + D;
     constexpr uint32_t kIdSP = idesc_bf16_f32(128, 64, 0, 0);     // S^T_h, dP^T_h
     constexpr uint32_t kIdV = idesc_bf16_f32(128, D, 0, 1);       // dV: A tmem, B MN-major
@@ -259,7 +267,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (warp == 8) {
         // ============================================================ producer
-        int it_use = 0, kv_use = 0, q_use = 0, dy_use[2] = {0, 0};
+        int it_use = 0, kv_use = 0, q_use[2] = {0, 0}, dy_use[2] = {0, 0};
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
@@ -302,20 +310,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (t_pf < n_qt) {
                         for (int pn = 0; pn < kPanels; pn++) {
                             tma_prefetch_2d(&tm_q, s.h * D + pn * 64, s.off0 + t_pf * kTileM);
+                            tma_prefetch_2d(&tm_q, s.h * D + pn * 64, s.off0 + t_pf * kTileM + 64);
                             tma_prefetch_2d(&tm_dy, s.h * D + pn * 64, s.off0 + t_pf * kTileM);
                             tma_prefetch_2d(&tm_dy, s.h * D + pn * 64, s.off0 + t_pf * kTileM + 64);
                         }
                         t_pf++;
                     }
-                    const int st = q_use & 1;
-                    ok = mbar_wait(&bars[kQEmpty0 + st], ((q_use >> 1) & 1) ^ 1, s_abort);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&bars[kQFull0 + st], L::kTile);
-                    for (int pn = 0; pn < kPanels; pn++)
-                        tma_load_2d(sm + (st ? L::q1 : L::q0) + pn * kPanel, &tm_q, &bars[kQFull0 + st],
-                                    s.h * D + pn * 64, s.off0 + t * kTileM);
-                    q_use++;
                     for (int hh = 0; ok && hh < 2; hh++) {
+                        ok = mbar_wait(&bars[kQEmpty0 + hh], (q_use[hh] & 1) ^ 1, s_abort);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&bars[kQFull0 + hh], L::kHalf);
+                        for (int pn = 0; pn < kPanels; pn++)
+                            tma_load_2d(sm + (hh ? L::q1 : L::q0) + pn * kHalfPanel, &tm_q, &bars[kQFull0 + hh],
+                                        s.h * D + pn * 64, s.off0 + t * kTileM + 64 * hh);
+                        q_use[hh]++;
                         ok = mbar_wait(&bars[kDYEmpty0 + hh], (dy_use[hh] & 1) ^ 1, s_abort);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&bars[kDYFull0 + hh], L::kHalf);
@@ -334,21 +342,93 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // drain the copies this warp issued (at most the latest one per buffer)
                 volatile int dummy = 0;
                 if (kv_use) mbar_wait(&bars[kKVFull], (kv_use - 1) & 1, &dummy);
-                for (int u = q_use - 2; u < q_use; u++)
-                    if (u >= 0) mbar_wait(&bars[kQFull0 + (u & 1)], (u >> 1) & 1, &dummy);
+                for (int hh = 0; hh < 2; hh++)
+                    if (q_use[hh]) mbar_wait(&bars[kQFull0 + hh], (q_use[hh] - 1) & 1, &dummy);
                 for (int hh = 0; hh < 2; hh++)
                     if (dy_use[hh]) mbar_wait(&bars[kDYFull0 + hh], (dy_use[hh] - 1) & 1, &dummy);
             }
         }
     } else if (warp == 9) {
         // ============================================================ MMA issuer
-        int it_use = 0, kv_use = 0, q_use = 0, acc_use = 0;
-        int dy_use[2] = {0, 0}, p_use[2] = {0, 0}, dq_use[2] = {0, 0};
+        // Order per tile t (next visible tile tn):
+        //   [p_full 0] products of half 0 of t;  [Q_0 of tn] S^T_0 of tn;
+        //   [p_full 1] products of half 1 of t;  dP^T_0 of tn;  [Q_1 of tn] S^T_1, dP^T_1 of tn.
+        // Q_h is released after the dK product of half h.
+        // The next tile's scores are then in flight while the elementwise warps
+        // drain dQ and set up, instead of after them.
+        int it_use = 0, kv_use = 0, acc_use = 0;
+        int q_use[2] = {0, 0}, dy_use[2] = {0, 0}, p_use[2] = {0, 0}, dq_use[2] = {0, 0};
         bool ok = true;
         const uint32_t aK = smem_u32(sm + L::k), aV = smem_u32(sm + L::v);
-        const uint32_t aQ0 = smem_u32(sm + L::q0), aQ1 = smem_u32(sm + L::q1);
+        const uint32_t aQ[2] = {smem_u32(sm + L::q0), smem_u32(sm + L::q1)};
         const uint32_t aDY[2] = {smem_u32(sm + L::dy0), smem_u32(sm + L::dy1)};
         const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
+        // S^T_h once Q_h of the tile is loaded
+        auto issue_s = [&](int hh) -> bool {
+            const bool w = mbar_wait(&bars[kQFull0 + hh], q_use[hh] & 1, s_abort);
+            q_use[hh]++;
+            if (!w) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk++) {
+                const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                const uint32_t offh = (kk >> 2) * kHalfPanel + (kk & 3) * 32;
+                mma_ss(tmem + kSCol + 64 * hh, sdesc_sw128(aK + off, 16, 1024),
+                       sdesc_sw128(aQ[hh] + offh, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+            }
+            return true;
+        };
+        // dP^T_h once dY'_h is loaded and the previous dQ^T_h has left the columns
+        auto issue_dp = [&](int hh) -> bool {
+            bool w = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort);
+            if (w) w = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort);
+            if (!w) return false;
+            dy_use[hh]++;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk++) {
+                const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                const uint32_t offh = (kk >> 2) * kHalfPanel + (kk & 3) * 32;
+                mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aV + off, 16, 1024),
+                       sdesc_sw128(aDY[hh] + offh, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars[kSFull0 + hh]);
+            return true;
+        };
+        // dQ^T_h, dV and dK products of half hh once its elementwise step is done
+        auto issue_prods = [&](int hh, bool init) -> bool {
+            if (!mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort)) return false;
+            p_use[hh]++;
+            if (init && !mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort)) return false;
+            tc_fence_after();
+            // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys); first,
+            // so that its drain overlaps the two products below
+#pragma unroll
+            for (int kk = 0; kk < 8; kk++) {
+                mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aK + kk * 2048, kPanel, 1024),
+                       sdesc_sw128(aDZ[hh] + kk * 2048, 16, 1024), kIdQ, kk > 0 ? 1u : 0u);
+            }
+            dq_use[hh]++;
+            tc_commit(&bars[kDQFull0 + hh]);
+            // dV += A^T_h dY'_h   (A^T_h: queries 32g.. at columns 64h + 32g .. +15)
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++) {
+                const uint32_t acol = kSCol + 64 * hh + 32 * (kk >> 1) + 8 * (kk & 1);
+                mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY[hh] + kk * 2048, kHalfPanel, 1024),
+                       kIdV, (!init || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars[kDYEmpty0 + hh]);
+            // dK += dZ^T_h Q_h
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++) {
+                mma_ss(tmem + kKCol, sdesc_sw128(aDZ[hh] + kk * 32, 16, 1024),
+                       sdesc_sw128(aQ[hh] + kk * 2048, kHalfPanel, 1024), kIdK,
+                       (!init || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars[kDZEmpty0 + hh]);
+            tc_commit(&bars[kQEmpty0 + hh]);
+            return true;
+        };
         while (ok) {
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
@@ -364,87 +444,32 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (lane == 0) {
                 const KvItem s = load_kv_item<KIND>(p, it);
                 const int n_qt = (s.L + kTileM - 1) / kTileM;
-                int last = -1;
-                for (int t = 0; t < n_qt; t++)
-                    if (q_class<KIND>(s, t) != 0) last = t;
                 ok = mbar_wait(&bars[kKVFull], kv_use & 1, s_abort);
                 kv_use++;
-                int n_done = 0;
-                for (int t = 0; ok && t <= last; t++) {
-                    if (q_class<KIND>(s, t) == 0) continue;
-                    const int st = q_use & 1;
-                    const uint32_t aQ = st ? aQ1 : aQ0;
-                    ok = mbar_wait(&bars[kQFull0 + st], (q_use >> 1) & 1, s_abort);
-                    if (!ok) break;
-                    q_use++;
-                    tc_fence_after();
-                    // ---- S^T_h and dP^T_h for both halves
-                    for (int hh = 0; ok && hh < 2; hh++) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; kk++) {
-                            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                            mma_ss(tmem + kSCol + 64 * hh, sdesc_sw128(aK + off, 16, 1024),
-                                   sdesc_sw128(aQ + off + hh * kHalfPanel, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
-                        }
-                        ok = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort);
-                        if (ok) ok = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort);
-                        if (!ok) break;
-                        dy_use[hh]++;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; kk++) {
-                            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                            const uint32_t offh = (kk >> 2) * kHalfPanel + (kk & 3) * 32;
-                            mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aV + off, 16, 1024),
-                                   sdesc_sw128(aDY[hh] + offh, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
-                        }
-                        tc_commit(&bars[kSFull0 + hh]);
-                    }
-                    // ---- products that need the elementwise results, half by half
-                    for (int hh = 0; ok && hh < 2; hh++) {
-                        ok = mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort);
-                        if (!ok) break;
-                        p_use[hh]++;
-                        if (n_done == 0 && hh == 0) {
-                            ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
-                            if (!ok) break;
-                        }
-                        tc_fence_after();
-                        const bool first = n_done == 0 && hh == 0;
-                        // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys); first,
-                        // so that its drain overlaps the two products below
-#pragma unroll
-                        for (int kk = 0; kk < 8; kk++) {
-                            mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aK + kk * 2048, kPanel, 1024),
-                                   sdesc_sw128(aDZ[hh] + kk * 2048, 16, 1024), kIdQ, kk > 0 ? 1u : 0u);
-                        }
-                        dq_use[hh]++;
-                        tc_commit(&bars[kDQFull0 + hh]);
-                        // dV += A^T_h dY'_h   (A^T_h: queries 32g.. at columns 64h + 32g .. +15)
-#pragma unroll
-                        for (int kk = 0; kk < 4; kk++) {
-                            const uint32_t acol = kSCol + 64 * hh + 32 * (kk >> 1) + 8 * (kk & 1);
-                            mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY[hh] + kk * 2048, kHalfPanel, 1024),
-                                   kIdV, (!first || kk > 0) ? 1u : 0u);
-                        }
-                        tc_commit(&bars[kDYEmpty0 + hh]);
-                        // dK += dZ^T_h Q_h
-#pragma unroll
-                        for (int kk = 0; kk < 4; kk++) {
-                            mma_ss(tmem + kKCol, sdesc_sw128(aDZ[hh] + kk * 32, 16, 1024),
-                                   sdesc_sw128(aQ + hh * kHalfPanel + kk * 2048, kPanel, 1024), kIdK,
-                                   (!first || kk > 0) ? 1u : 0u);
-                        }
-                        tc_commit(&bars[kDZEmpty0 + hh]);
-                    }
-                    if (!ok) break;
-                    tc_commit(&bars[kQEmpty0 + st]);
-                    if (t == last) tc_commit(&bars[kKVEmpty]);
-                    n_done++;
+                int t = next_visible<KIND>(s, -1, n_qt);
+                bool first = true;
+                if (ok && t < n_qt) {
+                    ok = issue_s(0);
+                    if (ok) ok = issue_dp(0);
+                    if (ok) ok = issue_s(1);
+                    if (ok) ok = issue_dp(1);
                 }
-                if (ok && n_done == 0) {
+                while (ok && t < n_qt) {
+                    const int tn = next_visible<KIND>(s, t, n_qt);
+                    ok = issue_prods(0, first);
+                    if (ok && tn < n_qt) ok = issue_s(0);
+                    if (ok) ok = issue_prods(1, false);
+                    if (ok && tn < n_qt) {
+                        ok = issue_dp(0);
+                        if (ok) ok = issue_s(1);
+                        if (ok) ok = issue_dp(1);
+                    }
+                    first = false;
+                    t = tn;
+                }
+                if (ok) {
                     tc_commit(&bars[kKVEmpty]);
-                    ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
+                    if (first) ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
                 }
                 if (ok) {
                     acc_use++;
@@ -468,7 +493,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
         int64_t* w_qts = s_qts + warp * 32;
-        float* w_stg = reinterpret_cast<float*>(sm + L::stg) + warp * 512;
+        float* w_stg = reinterpret_cast<float*>(sm + L::stg) + warp * 1024;
         int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * 32;
         float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * 64;
         const int nbm1 = p.nb - 1;
@@ -500,8 +525,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int32_t a_j = (int32_t)(ts_j - kmin);
             const int n_qt = (s.L + kTileM - 1) / kTileM;
             int n_done = 0;
-            for (int t = 0; ok && t < n_qt; t++) {
-                if (q_class<KIND>(s, t) == 0) continue;
+            for (int t = next_visible<KIND>(s, -1, n_qt); ok && t < n_qt; t = next_visible<KIND>(s, t, n_qt)) {
                 for (int hh = 0; hh < 2; hh++) {
                     const int i0 = t * kTileM + 64 * hh + 32 * g;   // first query of this warp's block
                     __syncwarp();
