@@ -55,13 +55,13 @@ struct BwdSmem {
     static constexpr uint32_t dy1 = dy0 + kHalf;
     static constexpr uint32_t dz0 = dy1 + kHalf;                 // dZ^T halves: 128 keys x 64 queries
     static constexpr uint32_t dz1 = dz0 + 128u * 64u * 2u;
-    static constexpr uint32_t stg = dz1 + 128u * 64u * 2u;       // float[8 warps][1024]: dQ slabs
-    static constexpr uint32_t rt = stg + 8u * 1024u * 4u;        // float[64]
+    static constexpr uint32_t stg = dz1 + 128u * 64u * 2u;       // float[warps][32 x cols]: dQ slabs
+    static constexpr uint32_t rt = stg + 32u * 1024u;            // float[64]
     static constexpr uint32_t rth = rt + kMaxTBuckets * 4u;      // float[64]: rab_time / 2
-    static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[8 warps][32]
-    static constexpr uint32_t qrel = qts + 8u * 32u * 8u;        // int32[8 warps][32]
-    static constexpr uint32_t diag = qrel + 8u * 32u * 4u;       // float[8 warps][64]
-    static constexpr uint32_t item = diag + 8u * 64u * 4u;       // int4[2]
+    static constexpr uint32_t qts = rth + kMaxTBuckets * 4u;     // int64[warps][cols]
+    static constexpr uint32_t qrel = qts + 64u * 8u * 4u;        // int32[warps][cols]
+    static constexpr uint32_t diag = qrel + 64u * 4u * 4u;       // float[warps][cols + 32]
+    static constexpr uint32_t item = diag + 64u * 4u * 4u + 32u * 4u * 16u;   // int4[2]
     static constexpr uint32_t bars = item + 2u * 16u;            // uint64[32]
     static constexpr uint32_t tmem = bars + 32u * 8u;
     static constexpr uint32_t abort_flag = tmem + 4u;
@@ -76,8 +76,15 @@ enum {
     kNumBars
 };
 
-constexpr int kThreads = 320;
-constexpr int kEwThreads = 256;
+// Warp roles: elementwise warps 0 .. kEwWarps-1 (lane quarter w % 4, query group w / 4 of
+// kEwCols queries in each 64-query half), then the TMA producer and the MMA issuer.
+constexpr int kEwCols = kBwdEwCols;
+constexpr int kEwGroups = 64 / kEwCols;
+constexpr int kEwWarps = 4 * kEwGroups;
+constexpr int kEwThreads = 32 * kEwWarps;
+constexpr int kProducerWarp = kEwWarps;
+constexpr int kMmaWarp = kEwWarps + 1;
+constexpr int kThreads = 32 * (kEwWarps + 2);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 0;
 constexpr uint32_t kPCol = 128;
@@ -128,32 +135,47 @@ __device__ __forceinline__ void flag_timeout(const BwdParams& p, volatile int* a
     atomicOr(&p.ctrl->status, kStatusTimeout);
 }
 
-// One dense 32 x 32 block: keys in lanes, queries along the chunk.  dg points at
+// Per-diagonal sums of a 32-key x C-query block (keys in lanes): at step k lane L takes
+// element k of lane (L + k) mod 32, whose key - query offset is L + ka - i0 (dlo) or,
+// after the wrap, L - 32 + ka - i0 (dhi).
+template <int C>
+__device__ __forceinline__ void diag_sums(const float (&zf)[C], float& dlo, float& dhi) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 0; k < C; k++) {
+        const float vd = __shfl_sync(0xffffffffu, zf[k], (lane + k) & 31);
+        const bool lo = lane + k < 32;
+        dlo += lo ? vd : 0.f;
+        dhi += lo ? 0.f : vd;
+    }
+}
+
+// One dense block of 32 keys (lanes) x C queries (along the chunk).  dg points at
 // this lane's diagonal-row entry for the block's first query (later queries sit at
 // decreasing addresses); the row holds half the position bias, the causal mask and,
 // when the block's time bucket is uniform, half the time bias.  TV: the bucket varies
 // inside the block and is computed per element from qr, the block's 32-bit query
 // times relative to the warp's smallest key time.  Two variants only, so that the
 // elementwise code stays small enough for the instruction cache.
-template <bool TV>
-__device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* dg,
+template <bool TV, int C>
+__device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_t (&dp)[C], const float* dg,
                                           bool pos_diag, float& dlo, float& dhi, const int32_t* qr, int32_t a_j,
                                           const float* rth, int nbm1, float& acc, float* g_rt,
-                                          uint32_t (&pa)[16], uint32_t (&pz)[16]) {
+                                          uint32_t (&pa)[C / 2], uint32_t (&pz)[C / 2]) {
     const int lane = threadIdx.x & 31;
-    int32_t q[32];
+    int32_t q[C];
     if (TV) {
         const int4* q4 = reinterpret_cast<const int4*>(qr);
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
+        for (int e = 0; e < C / 4; e++) {
             const int4 v = q4[e];
             q[4 * e] = v.x; q[4 * e + 1] = v.y; q[4 * e + 2] = v.z; q[4 * e + 3] = v.w;
         }
     }
     // pass 1: independent per-element chains (no cross-lane operations)
-    float zf[32];
+    float zf[C];
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
+    for (int e = 0; e < C; e += 2) {
         float av[2];
 #pragma unroll
         for (int f = 0; f < 2; f++) {
@@ -171,13 +193,13 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
     }
     // pass 2: gradient bookkeeping on finished values
 #pragma unroll
-    for (int k = 0; k < 32; k++) acc += zf[k];
+    for (int k = 0; k < C; k++) acc += zf[k];
     if (TV) {
         // the bucket changes rarely along a row: run-length sums, flushed on change
         int cur_t = time_bucket_u32((uint32_t)abs(q[0] - a_j), nbm1);
         float acc_t = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; k++) {
+        for (int k = 0; k < C; k++) {
             const int tb = time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1);
             if (tb != cur_t) {
                 red_add_f32(&g_rt[cur_t], acc_t);
@@ -188,17 +210,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[32], const uint32
         }
         red_add_f32(&g_rt[cur_t], acc_t);
     }
-    if (pos_diag) {
-        // diagonal m = key lane - query k: lane L collects m = L (dlo) and m = L - 32
-        // (dhi), both held by lane (L + k) mod 32 at step k
-#pragma unroll
-        for (int k = 0; k < 32; k++) {
-            const float vd = __shfl_sync(0xffffffffu, zf[k], (lane + k) & 31);
-            const bool lo = lane + k < 32;
-            dlo += lo ? vd : 0.f;
-            dhi += lo ? 0.f : vd;
-        }
-    }
+    if (pos_diag) diag_sums<C>(zf, dlo, dhi);
 }
 
 template <int KIND, int D>
@@ -208,8 +220,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using L = BwdSmem<D>;
     constexpr int kPanels = D / 64;
-    constexpr int kDqDims = D == 128 ? 32 : 16;     // dQ slab: head dims per warp
-    constexpr int kDqRows = 32;                     // dQ slab: queries (4 KB / 2 KB per warp)
     constexpr uint32_t kKCol = kVCol + D;
     constexpr uint32_t kIdSP = idesc_bf16_f32(128, 64, 0, 0);     // S^T_h, dP^T_h
     constexpr uint32_t kIdV = idesc_bf16_f32(128, D, 0, 1);       // dV: A tmem, B MN-major
@@ -249,14 +259,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         *s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_dy);
         prefetch_tmap(&tm_dq);
     }
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
     }
@@ -265,7 +275,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 8) {
+    if (warp == kProducerWarp) {
         // ============================================================ producer
         int it_use = 0, kv_use = 0, q_use[2] = {0, 0}, dy_use[2] = {0, 0};
         bool ok = true;
@@ -348,7 +358,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (dy_use[hh]) mbar_wait(&bars[kDYFull0 + hh], (dy_use[hh] - 1) & 1, &dummy);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         // Order per tile t (next visible tile tn):
         //   [p_full 0] products of half 0 of t;  [Q_0 of tn] S^T_0 of tn;
@@ -410,10 +420,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             dq_use[hh]++;
             tc_commit(&bars[kDQFull0 + hh]);
-            // dV += A^T_h dY'_h   (A^T_h: queries 32g.. at columns 64h + 32g .. +15)
+            // dV += A^T_h dY'_h   (A^T_h: the kEwCols queries of group c packed into columns
+            // 64h + kEwCols*c .. +kEwCols/2)
 #pragma unroll
             for (int kk = 0; kk < 4; kk++) {
-                const uint32_t acol = kSCol + 64 * hh + 32 * (kk >> 1) + 8 * (kk & 1);
+                const uint32_t acol = kSCol + 64 * hh + kEwCols * ((16 * kk) / kEwCols) + 8 * ((16 * kk) % kEwCols / 16);
                 mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY[hh] + kk * 2048, kHalfPanel, 1024),
                        kIdV, (!init || kk > 0) ? 1u : 0u);
             }
@@ -486,16 +497,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_wait(&bars[kDrain], 0, &dummy);
         }
     } else {
-        // ============================================================ elementwise (warps 0-7)
+        // ============================================================ elementwise warps
+        constexpr int C = kEwCols;
+        constexpr int kDqDims = D == 128 ? 32 : 16;   // dQ slab: head dims per warp
         const int wq = warp & 3;                 // lane quarter: key rows 32*wq .. +31
-        const int g = warp >> 2;                 // column group: queries 32*g .. +31 of each half
+        const int g = warp >> 2;                 // query group: queries C*g .. +C-1 of each half
         const int r = wq * 32 + lane;            // key row within the tile (TMEM lane)
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
-        int64_t* w_qts = s_qts + warp * 32;
-        float* w_stg = reinterpret_cast<float*>(sm + L::stg) + warp * 1024;
-        int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * 32;
-        float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * 64;
+        int64_t* w_qts = s_qts + warp * C;
+        float* w_stg = reinterpret_cast<float*>(sm + L::stg) + warp * (32 * C);
+        int32_t* w_qrel = reinterpret_cast<int32_t*>(sm + L::qrel) + warp * C;
+        float* w_diag = reinterpret_cast<float*>(sm + L::diag) + warp * (C + 32);
         const int nbm1 = p.nb - 1;
         int it_use = 0, acc_use = 0;
         int s_use[2] = {0, 0}, dz_use[2] = {0, 0}, dq_use[2] = {0, 0};
@@ -527,29 +540,29 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int n_done = 0;
             for (int t = next_visible<KIND>(s, -1, n_qt); ok && t < n_qt; t = next_visible<KIND>(s, t, n_qt)) {
                 for (int hh = 0; hh < 2; hh++) {
-                    const int i0 = t * kTileM + 64 * hh + 32 * g;   // first query of this warp's block
+                    const int i0 = t * kTileM + 64 * hh + C * g;    // first query of this warp's block
                     __syncwarp();
-                    const int iq = i0 + lane;
+                    const int iq = i0 + lane % C;                  // lanes past C repeat the block
                     const int64_t tq = iq < s.L ? p.ts[s.off0 + iq] : 0;
-                    w_qts[lane] = tq;
+                    if (lane < C) w_qts[lane] = tq;
                     int64_t qmin = iq < s.L ? tq : INT64_MAX, qmax = iq < s.L ? tq : INT64_MIN;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
                         qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
                         qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
                     }
-                    // ---- classify this warp's block: 32 keys x 32 queries
+                    // ---- classify this warp's block: 32 keys x C queries
                     int wcls = 0;
                     if (warp_keys > 0 && i0 < s.L)
-                        wcls = tile_class(KIND, i0, min(i0 + 31, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
+                        wcls = tile_class(KIND, i0, min(i0 + C - 1, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
                     int pm = -1, tm = -1;                // -1 = element-by-element rules
                     int pidx_u = 0;
                     TimeClass tc;
                     tc.tb_lo = tc.tb_hi = 0;
                     tc.thr = 0;
-                    const bool dense = wcls != 0 && warp_keys == 32 && i0 + 32 <= s.L &&
+                    const bool dense = wcls != 0 && warp_keys == 32 && i0 + C <= s.L &&
                                        (KIND == HSTU_KIND_CAUSAL || wcls == 2);
-                    const int dmin = ka - (i0 + 31);     // smallest key - query of the block
+                    const int dmin = ka - (i0 + C - 1);  // smallest key - query of the block
                     if (dense) {
                         tc = classify_time(kmin, kmax, qmin, qmax, p.nb);
                         if (tc.mode >= 0) {
@@ -558,16 +571,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             if (wcls == 2 && dmax <= -(p.P - 1)) { pm = kPosUniform; pidx_u = 0; }
                             else if (wcls == 2 && dmin >= p.P - 1) { pm = kPosUniform; pidx_u = 2 * p.P - 2; }
                             else pm = kPosDiag;
-                            // diagonal row: key - query = dmin + k, k in [0, 63); constant when
+                            // diagonal row: key - query = dmin + k, k in [0, C + 31); constant when
                             // the position index is clamped across the whole block
                             const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
-                            for (int k = lane; k < 63; k += 32) {
+                            for (int k = lane; k < C + 31; k += 32) {
                                 const int dl = dmin + k;
                                 const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
                                 w_diag[k] = masked ? kMaskedHalfBias
                                                    : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
                             }
-                            if (tm != kTimeUniform) w_qrel[lane] = (int32_t)(tq - kmin);
+                            if (tm != kTimeUniform && lane < C) w_qrel[lane] = (int32_t)(tq - kmin);
                         }
                     }
                     __syncwarp();
@@ -578,28 +591,28 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     dz_use[hh]++;
                     tc_fence_after();
                     float acc = 0.f, dlo = 0.f, dhi = 0.f;
-                    uint32_t pa[16], pz[16];
+                    uint32_t pa[C / 2], pz[C / 2];
                     if (wcls == 0) {
 #pragma unroll
-                        for (int e = 0; e < 16; e++) pa[e] = pz[e] = 0u;
+                        for (int e = 0; e < C / 2; e++) pa[e] = pz[e] = 0u;
                     } else {
-                        uint32_t sv[32], dp[32];
-                        tmem_ld32(tmem + lane_base + kSCol + 64 * hh + 32 * g, sv);
-                        tmem_ld32(tmem + lane_base + kPCol + 64 * hh + 32 * g, dp);
+                        uint32_t sv[C], dp[C];
+                        tmem_ld(tmem + lane_base + kSCol + 64 * hh + C * g, sv);
+                        tmem_ld(tmem + lane_base + kPCol + 64 * hh + C * g, dp);
                         tmem_ld_wait(sv);
                         tmem_ld_wait(dp);
-                        const float* dg = w_diag + lane + 31;
+                        const float* dg = w_diag + lane + C - 1;
                         if (tm == kTimeUniform)
-                            bwd_block<false>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
+                            bwd_block<false, C>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
                         else if (tm >= 0)
-                            bwd_block<true>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
+                            bwd_block<true, C>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
                         else {
                             // element by element (MTGR candidates, ragged edges, int64-wide times)
                             int cur_p = -1, cur_t = -1;
                             float acc_p = 0.f, acc_t = 0.f;
-                            float zf[32];
+                            float zf[C];
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
+                            for (int e = 0; e < C; e += 2) {
                                 float av[2];
 #pragma unroll
                                 for (int f = 0; f < 2; f++) {
@@ -635,24 +648,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                             if (cur_p >= 0 && acc_p != 0.f) red_add_f32(&g_rp[cur_p], acc_p);
                             if (cur_t >= 0 && acc_t != 0.f) red_add_f32(&g_rt[cur_t], acc_t);
-                            if (KIND == HSTU_KIND_CAUSAL) {
-#pragma unroll
-                                for (int k = 0; k < 32; k++) {
-                                    const float vd = __shfl_sync(kFull, zf[k], (lane + k) & 31);
-                                    const bool lo = lane + k < 32;
-                                    dlo += lo ? vd : 0.f;
-                                    dhi += lo ? 0.f : vd;
-                                }
-                            }
+                            if (KIND == HSTU_KIND_CAUSAL) diag_sums<C>(zf, dlo, dhi);
                         }
                     }
                     // A^T_h back into TMEM inside the S^T_h columns this warp has read
-                    tmem_st16(tmem + lane_base + kSCol + 64 * hh + 32 * g, pa);
-                    // dZ^T_h into shared memory: row r, queries 32g.. (128-byte swizzle)
+                    tmem_st(tmem + lane_base + kSCol + 64 * hh + C * g, pa);
+                    // dZ^T_h into shared memory: row r, queries C*g .. (128-byte swizzle)
                     const uint32_t row_addr = aDZ[hh] + r * 128;
 #pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const uint32_t ch = (uint32_t)((4 * g + e) ^ (r & 7));
+                    for (int e = 0; e < C / 8; e++) {
+                        const uint32_t ch = (uint32_t)(((C / 8) * g + e) ^ (r & 7));
                         st_shared_v4(row_addr + ch * 16, pz[4 * e], pz[4 * e + 1], pz[4 * e + 2], pz[4 * e + 3]);
                     }
                     // ---- rab gradients of the block
@@ -666,10 +671,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     if (pm == kPosDiag || (pm < 0 && wcls != 0 && KIND == HSTU_KIND_CAUSAL)) {
                         const int np1 = p.P - 1;
-                        // dlo: key - query = dmin + lane + 31;  dhi: dmin + lane - 1
-                        if (dlo != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + 31, -np1), np1) + np1], dlo);
-                        if (lane > 0 && dhi != 0.f)
-                            red_add_f32(&g_rp[min(max(dmin + lane - 1, -np1), np1) + np1], dhi);
+                        // dlo: key - query = dmin + lane + C - 1;  dhi: dmin + lane + C - 33
+                        if (dlo != 0.f) red_add_f32(&g_rp[min(max(dmin + lane + C - 1, -np1), np1) + np1], dlo);
+                        if (lane > 32 - C && dhi != 0.f)
+                            red_add_f32(&g_rp[min(max(dmin + lane + C - 33, -np1), np1) + np1], dhi);
                     }
                     tmem_st_wait();
                     fence_proxy_async_smem();
@@ -677,35 +682,33 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     mbar_arrive(&bars[kPFull0 + hh]);
                 }
                 if (!ok) break;
-                // ---- drain dQ^T of both halves (lanes = head dims, columns = queries)
+                // ---- drain dQ^T of both halves (lanes = head dims, columns = queries): one
+                // slab of C queries x kDqDims head dims (row-major) per warp, one TMA reduce-add.
+                // M = 128 puts head dim 32*wq + lane in this lane; M = 64 puts head dims
+                // 16*wq .. +15 in the first 16 lanes of the lane quarter.  Queries past the
+                // sequence end carry exact zeros (their dZ is zero).
                 for (int hh = 0; hh < 2; hh++) {
                     ok = mbar_wait(&bars[kDQFull0 + hh], dq_use[hh] & 1, s_abort);
                     if (!__all_sync(kFull, ok)) { ok = false; break; }
                     dq_use[hh]++;
                     tc_fence_after();
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + kPCol + 64 * hh + 32 * g, v);
+                    uint32_t v[C];
+                    tmem_ld(tmem + lane_base + kPCol + 64 * hh + C * g, v);
                     tmem_ld_wait(v);
                     tc_fence_before();
                     mbar_arrive(&bars[kDQDrained0 + hh]);      // the columns are free again
-                    // Slabs of kDqRows queries x kDqDims head dims, row-major, one TMA
-                    // reduce-add each.  M = 128 puts head dim 32*wq + lane in this lane; M = 64
-                    // puts head dims 16*wq .. +15 in the first 16 lanes of the lane quarter.
-                    // Queries past the sequence end carry exact zeros (their dZ is zero).
-                    const int qi = t * kTileM + 64 * hh + 32 * g;  // first query of the columns
-#pragma unroll
-                    for (int ps = 0; ps < 32 / kDqRows; ps++) {
-                        if (qi + ps * kDqRows >= s.L) break;
-                        if (lane == 0) bulk_wait_read_all();   // the previous slab has been read
+                    const int qi = t * kTileM + 64 * hh + C * g;   // first query of the columns
+                    if (qi < s.L) {
+                        if (lane == 0) bulk_wait_read_all();       // the previous slab has been read
                         __syncwarp();
                         if (D == 128 || lane < 16) {
 #pragma unroll
-                            for (int e = 0; e < kDqRows; e++) w_stg[e * kDqDims + lane] = __uint_as_float(v[ps * kDqRows + e]);
+                            for (int e = 0; e < C; e++) w_stg[e * kDqDims + lane] = __uint_as_float(v[e]);
                         }
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_reduce_add_2d(&tm_dq, w_stg, s.h * D + wq * kDqDims, s.off0 + qi + ps * kDqRows);
+                            tma_reduce_add_2d(&tm_dq, w_stg, s.h * D + wq * kDqDims, s.off0 + qi);
                             bulk_commit_group();
                         }
                     }
@@ -713,36 +716,36 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 n_done++;
             }
             if (!ok) break;
-            // ---------------- epilogue: dV, dK rows of this key tile
+            // ---------------- epilogue: dV, dK rows of this key tile (D / kEwGroups columns per warp)
             ok = mbar_wait(&bars[kAccFull], acc_use & 1, s_abort);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             acc_use++;
             tc_fence_after();
+            constexpr int kEpCols = D / kEwGroups;
 #pragma unroll 1
-            for (int c = 0; c < D / 64; c++) {
-                const int col = g * (D / 2) + 32 * c;
-                uint32_t vv[32], kv[32];
-                tmem_ld32(tmem + lane_base + kVCol + col, vv);
-                tmem_ld32(tmem + lane_base + kKCol + col, kv);
+            for (int c = 0; c < kEpCols / 16; c++) {
+                const int col = g * kEpCols + 16 * c;
+                uint32_t vv[16], kv[16];
+                tmem_ld16(tmem + lane_base + kVCol + col, vv);
+                tmem_ld16(tmem + lane_base + kKCol + col, kv);
                 tmem_ld_wait(vv);
                 tmem_ld_wait(kv);
                 if (key_ok) {
-                    uint4 wv[4], wk[4];
+                    uint4 wv[2], wk[2];
                     uint32_t* pv = reinterpret_cast<uint32_t*>(wv);
                     uint32_t* pk = reinterpret_cast<uint32_t*>(wk);
 #pragma unroll
-                    for (int e = 0; e < 16; e++) {
+                    for (int e = 0; e < 8; e++) {
                         pv[e] = n_done ? pack_bf16x2(2.f * __uint_as_float(vv[2 * e]), 2.f * __uint_as_float(vv[2 * e + 1])) : 0u;
                         pk[e] = n_done ? pack_bf16x2(__uint_as_float(kv[2 * e]), __uint_as_float(kv[2 * e + 1])) : 0u;
                     }
                     const size_t o = (size_t)(s.off0 + j) * p.ld + (size_t)s.h * D + col;
                     uint4* dv = reinterpret_cast<uint4*>(p.dv + o);
                     uint4* dk = reinterpret_cast<uint4*>(p.dk + o);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        dv[e] = wv[e];
-                        dk[e] = wk[e];
-                    }
+                    dv[0] = wv[0];
+                    dv[1] = wv[1];
+                    dk[0] = wk[0];
+                    dk[1] = wk[1];
                 }
             }
             tc_fence_before();
@@ -755,7 +758,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }

@@ -436,7 +436,7 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     float* dq_acc = at<float>(workspace, L.dq_acc);
     const int dq_box_cols = d.d_qk == 128 ? 32 : 16;
     if (!make_tmap(&tq, q, d.T, D, 64) || !make_tmap(&tk, k, d.T, D) || !make_tmap(&tv, v, d.T, D) ||
-        !make_tmap(&tdy, lp.dy, d.T, D, 64) || !make_tmap_f32(&tdq, dq_acc, d.T, D, dq_box_cols, 32))
+        !make_tmap(&tdy, lp.dy, d.T, D, 64) || !make_tmap_f32(&tdq, dq_acc, d.T, D, dq_box_cols, kBwdEwCols))
         return HSTU_ERR_CUDA;
     st = cuda_status(cudaMemsetAsync(dq_acc, 0, (size_t)d.T * D * sizeof(float), s));
     if (st != HSTU_OK) return st;

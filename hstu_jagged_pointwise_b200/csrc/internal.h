@@ -150,8 +150,13 @@ cudaError_t launch_attn_fwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
 int attn_fwd_tc_ctas_per_sm(int kind, int d);
 cudaError_t launch_attn_fwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(int dtype_f32, int d, const SimtParams& p, cudaStream_t s);
+// Queries per elementwise warp and 64-query half in the tensor-core backward (16 or 32);
+// it also sets the row count of the dQ reduce-add boxes.
+constexpr int kBwdEwCols = 16;
+
 // tq and tdy map Q and dY / (2 alpha) (bf16, 64-row boxes); tdq maps the fp32 dQ
-// accumulator with boxes of (32 dims x 32 rows) for d = 128 and (16 dims x 32 rows) for d = 64.
+// accumulator with boxes of (32 dims x kBwdEwCols rows) for d = 128 and (16 dims x kBwdEwCols
+// rows) for d = 64.
 cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdy, const CUtensorMap& tdq,
                                const BwdParams& p, int grid, cudaStream_t s);
