@@ -34,9 +34,9 @@ struct FwdSmem {
     static constexpr uint32_t v = k + kTileBytes;
     static constexpr uint32_t rt = v + kTileBytes;                 // float[64]
     static constexpr uint32_t rth = rt + kMaxTBuckets * 4u;        // float[64]: rab_time / 2
-    static constexpr uint32_t cts = rth + kMaxTBuckets * 4u;       // int64[4 warps][128]
-    static constexpr uint32_t diag = cts + 4u * 128u * 8u;         // float[4 warps][160]
-    static constexpr uint32_t item = diag + 4u * 160u * 4u;        // int4[2]
+    static constexpr uint32_t cts = rth + kMaxTBuckets * 4u;       // int64[8 warps][64]
+    static constexpr uint32_t diag = cts + 8u * 64u * 8u;          // float[8 warps][96]
+    static constexpr uint32_t item = diag + 8u * 96u * 4u;         // int4[2]
     static constexpr uint32_t bars = item + 2u * 16u;              // uint64[16]
     static constexpr uint32_t tmem = bars + 16u * 8u;              // uint32
     static constexpr uint32_t abort_flag = tmem + 4u;              // int
@@ -50,7 +50,13 @@ enum {
     kItFull0, kItFull1, kItEmpty0, kItEmpty1, kDrain, kNumBars
 };
 
-constexpr int kThreads = 192;
+// Warp roles: 8 elementwise warps (lane quarter w % 4 of the tile rows, key half w / 4),
+// then the TMA producer and the MMA issuer.
+constexpr int kEwWarps = 8;
+constexpr int kEwThreads = 32 * kEwWarps;
+constexpr int kProducerWarp = kEwWarps;
+constexpr int kMmaWarp = kEwWarps + 1;
+constexpr int kThreads = 32 * (kEwWarps + 2);
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kSCol = 0;
 constexpr uint32_t kOCol = 128;
@@ -180,23 +186,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(&bars[kVFull], 1);
         mbar_init(&bars[kVEmpty], 1);
         mbar_init(&bars[kSFull], 1);
-        mbar_init(&bars[kPFull], 128);
+        mbar_init(&bars[kPFull], kEwThreads);
         mbar_init(&bars[kOFull], 1);
-        mbar_init(&bars[kOEmpty], 128);
+        mbar_init(&bars[kOEmpty], kEwThreads);
         mbar_init(&bars[kItFull0], 1);
         mbar_init(&bars[kItFull1], 1);
-        mbar_init(&bars[kItEmpty0], 129);
-        mbar_init(&bars[kItEmpty1], 129);
+        mbar_init(&bars[kItEmpty0], kEwThreads + 1);
+        mbar_init(&bars[kItEmpty1], kEwThreads + 1);
         mbar_init(&bars[kDrain], 1);
         *s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
     }
@@ -205,7 +211,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ============================================================ producer
         int it_use = 0, q_use = 0, k_use = 0, v_use = 0;
         bool ok = true;
@@ -279,7 +285,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (v_use) mbar_wait(&bars[kVFull], (v_use - 1) & 1, &dummy);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         int it_use = 0, q_use = 0, k_use = 0, v_use = 0, p_use = 0, o_use = 0;
         bool ok = true;
@@ -334,7 +340,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kTileN / 16; kk++) {
-                        mma_ts(tmem + kOCol, tmem + kSCol + kk * 8,
+                        // P of keys 32c .. 32c+31 sits in the first 16 columns of S chunk c
+                        mma_ts(tmem + kOCol, tmem + kSCol + 32 * (kk >> 1) + 8 * (kk & 1),
                                sdesc_sw128(aV + kk * 2048, kPanelBytes, 1024), kIdescO,
                                (n_done > 0 || kk > 0) ? 1u : 0u);
                     }
@@ -361,13 +368,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_wait(&bars[kDrain], 0, &dummy);
         }
     } else {
-        // ============================================================ elementwise (warps 0-3)
+        // ============================================================ elementwise (warps 0-7)
         int it_use = 0, s_use = 0, o_use = 0;
-        const int r = tid;                                  // TMEM lane = tile row
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        int64_t* w_cts = s_cts + warp * 128;                // this warp's column times (int64)
+        const int wq = warp & 3;                            // lane quarter: tile rows 32*wq .. +31
+        const int g = warp >> 2;                            // key half: tile keys 64*g .. +63
+        const int r = wq * 32 + lane;                       // TMEM lane = tile row
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        int64_t* w_cts = s_cts + warp * 64;                 // this warp's column times (int64)
         int32_t* w_crel = reinterpret_cast<int32_t*>(w_cts); // or 32-bit relative times
-        float* w_diag = s_diag + warp * 160;
+        float* w_diag = s_diag + warp * 96;
         const int nbm1 = p.nb - 1;
         const float rp_self = s_rp[p.P - 1];
         const float rt_zero = s_rt[0];
@@ -385,7 +394,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int ic = min(i, s.row_end - 1);           // clamped row for lookups
             const int64_t ts_i = p.q_ts[s.q0 + ic];
             const int pos_i = row_pos<KIND>(s, ic);
-            const int r0 = s.row0 + 32 * warp;              // first row of this warp
+            const int r0 = s.row0 + 32 * wq;                // first row of this warp
             // this warp's row range (positions and timestamps)
             int64_t rmin = row_ok ? ts_i : INT64_MAX, rmax = row_ok ? ts_i : INT64_MIN;
             int pr_lo = row_ok ? pos_i : INT32_MAX, pr_hi = row_ok ? pos_i : INT32_MIN;
@@ -402,13 +411,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int t = 0; t < n_kt; t++) {
                 const int cls = kv_class<KIND>(s, t);
                 if (cls == 0) continue;
-                const int n0 = t * kTileN;
-                // column timestamps of this tile
+                const int n0 = t * kTileN + 64 * g;         // first key of this warp's half
+                // column timestamps of this warp's keys
                 __syncwarp();
-                int64_t tj[4];
+                int64_t tj[2];
                 int64_t cmin = INT64_MAX, cmax = INT64_MIN;
 #pragma unroll
-                for (int e = 0; e < 4; e++) {
+                for (int e = 0; e < 2; e++) {
                     const int j = n0 + lane + 32 * e;
                     tj[e] = j < s.Lk ? p.kv_ts[s.kv0 + j] : 0;
                     if (j < s.Lk) {
@@ -421,23 +430,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     cmin = min(cmin, (int64_t)__shfl_xor_sync(kFull, (long long)cmin, o));
                     cmax = max(cmax, (int64_t)__shfl_xor_sync(kFull, (long long)cmax, o));
                 }
-                // ---- classify this warp's block: 32 rows x 128 columns
+                // ---- classify this warp's block: 32 rows x 64 columns
                 int pm = -1, tm = -1;
                 float c0 = 0.f;
                 TimeClass tc;
                 tc.tb_lo = tc.tb_hi = 0;
                 tc.thr = 0;
                 int wcls = 0;
-                if (warp_rows)
+                if (warp_rows && n0 < s.Lk)
                     wcls = KIND == HSTU_KIND_MFALCON
                                ? 2
                                : tile_class(KIND, r0, min(r0 + 31, s.row_end - 1), n0,
-                                            min(n0 + kTileN - 1, s.Lk - 1), s.S, s.R);
-                const bool dense = wcls != 0 && n0 + kTileN <= s.Lk &&
+                                            min(n0 + 63, s.Lk - 1), s.S, s.R);
+                const bool dense = wcls != 0 && n0 + 64 <= s.Lk &&
                                    (KIND == HSTU_KIND_CAUSAL || wcls == 2);
                 if (dense) {
                     tc = classify_time(rmin, rmax, cmin, cmax, p.nb);
-                    const int dmax = col_pos<KIND>(s, n0 + kTileN - 1) - pr_lo;
+                    const int dmax = col_pos<KIND>(s, n0 + 63) - pr_lo;
                     const int dmin = col_pos<KIND>(s, n0) - pr_hi;
                     int pidx_u = -1;
                     if (wcls == 2 && dmax <= -(p.P - 1)) pidx_u = 0;
@@ -450,10 +459,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         if (pm == kPosUniform && tm == kTimeUniform) {
                             c0 = 0.5f * s_rp[pidx_u] + tadd;
                         } else {
-                            // diagonal row: delta = j - i = (n0 - r0 - 31) + k, k in [0, 159);
+                            // diagonal row: delta = j - i = (n0 - r0 - 31) + k, k in [0, 95);
                             // constant when the position index is clamped across the block
                             const int d0 = n0 - r0 - 31;
-                            for (int k = lane; k < 159; k += 32) {
+                            for (int k = lane; k < 95; k += 32) {
                                 const int dl = d0 + k;
                                 const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
                                 const int pi = pm == kPosUniform ? pidx_u : min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1;
@@ -467,11 +476,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (pm >= 0) {
                     if (tm != kTimeUniform) {
 #pragma unroll
-                        for (int e = 0; e < 4; e++) w_crel[lane + 32 * e] = (int32_t)(tj[e] - cmin);
+                        for (int e = 0; e < 2; e++) w_crel[lane + 32 * e] = (int32_t)(tj[e] - cmin);
                     }
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 4; e++) w_cts[lane + 32 * e] = tj[e];
+                    for (int e = 0; e < 2; e++) w_cts[lane + 32 * e] = tj[e];
                 }
                 __syncwarp();
                 const int32_t a_i = (int32_t)(ts_i - cmin);
@@ -480,13 +489,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 s_use++;
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < 4; c++) {
+                for (int cc = 0; cc < 2; cc++) {
+                    const int c = 2 * g + cc;                // 32-column chunk of the tile
                     uint32_t v[32];
                     tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
                     tmem_ld_wait(v);
                     uint32_t pk[16];
-                    const float* dg = w_diag + 31 - lane + 32 * c;
-                    const int32_t* cr = w_crel + 32 * c;
+                    const float* dg = w_diag + 31 - lane + 32 * cc;
+                    const int32_t* cr = w_crel + 32 * cc;
                     if (pm == kPosUniform && tm == kTimeUniform) fwd_block<kBiasConst>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else if (pm >= 0 && tm == kTimeUniform) fwd_block<kBiasRow>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else if (pm >= 0 && tm >= 0) fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
@@ -495,7 +505,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         float pv[32];
 #pragma unroll
                         for (int e = 0; e < 32; e++) {
-                            const int jj = 32 * c + e;
+                            const int jj = 32 * cc + e;
                             const int j = n0 + jj;
                             const int64_t ts_j = w_cts[jj];
                             bool vis = row_ok && j < s.Lk;
@@ -509,7 +519,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                         for (int e = 0; e < 16; e++) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
                     }
-                    tmem_st16(tmem + lane_base + kSCol + 16 * c, pk);
+                    // P (bf16 pairs) into the chunk's own, already read, S columns: two warps
+                    // share these TMEM lanes and each may only overwrite what it has read
+                    tmem_st16(tmem + lane_base + kSCol + 32 * c, pk);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -545,7 +557,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             o_use++;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < D / 32; c++) {
+            for (int c = g * (D / 64); c < (g + 1) * (D / 64); c++) {   // this warp's half of the columns
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_base + kOCol + 32 * c, v);
                 tmem_ld_wait(v);
@@ -587,7 +599,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
