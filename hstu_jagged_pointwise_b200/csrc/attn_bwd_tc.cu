@@ -156,9 +156,10 @@ __device__ __forceinline__ void diag_sums(const float (&zf)[C], float& dlo, floa
 // when the block's time bucket is uniform, half the time bias.  TV: the bucket varies
 // inside the block and is computed per element from qr, the block's 32-bit query
 // times relative to the warp's smallest key time.  Two variants only, so that the
-// elementwise code stays small enough for the instruction cache.
-template <bool TV, int C>
-__device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_t (&dp)[C], const float* dg,
+// elementwise code stays small enough for the instruction cache.  CONST: one bias c0
+// for the whole block (position and time bias uniform), no diagonal row.
+template <bool TV, int C, bool CONST = false>
+__device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_t (&dp)[C], const float* dg, float c0,
                                           bool pos_diag, float& dlo, float& dhi, const int32_t* qr, int32_t a_j,
                                           const float* rth, int nbm1, float& acc, float* g_rt,
                                           uint32_t (&pa)[C / 2], uint32_t (&pz)[C / 2]) {
@@ -180,7 +181,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_
 #pragma unroll
         for (int f = 0; f < 2; f++) {
             const int k = e + f;
-            float hb = dg[-k];
+            float hb = CONST ? c0 : dg[-k];
             if (TV) hb += rth[time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1)];
             const float h = fmaf(__uint_as_float(sv[k]), 0.5f, hb);
             const float th = tanh_approx(h);
@@ -557,6 +558,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         wcls = tile_class(KIND, i0, min(i0 + C - 1, s.L - 1), ka, min(ka + 31, s.n_end - 1), s.S, s.R);
                     int pm = -1, tm = -1;                // -1 = element-by-element rules
                     int pidx_u = 0;
+                    float c0 = 0.f;
                     TimeClass tc;
                     tc.tb_lo = tc.tb_hi = 0;
                     tc.thr = 0;
@@ -571,10 +573,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             if (wcls == 2 && dmax <= -(p.P - 1)) { pm = kPosUniform; pidx_u = 0; }
                             else if (wcls == 2 && dmin >= p.P - 1) { pm = kPosUniform; pidx_u = 2 * p.P - 2; }
                             else pm = kPosDiag;
-                            // diagonal row: key - query = dmin + k, k in [0, C + 31); constant when
-                            // the position index is clamped across the whole block
+                            // diagonal row: key - query = dmin + k, k in [0, C + 31); a single
+                            // constant when both biases are uniform over the block
                             const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
-                            for (int k = lane; k < C + 31; k += 32) {
+                            if (pm == kPosUniform && tm == kTimeUniform) c0 = 0.5f * s_rp[pidx_u] + tadd;
+                            else for (int k = lane; k < C + 31; k += 32) {
                                 const int dl = dmin + k;
                                 const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
                                 w_diag[k] = masked ? kMaskedHalfBias
@@ -602,10 +605,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_ld_wait(sv);
                         tmem_ld_wait(dp);
                         const float* dg = w_diag + lane + C - 1;
-                        if (tm == kTimeUniform)
-                            bwd_block<false, C>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
+                        if (pm == kPosUniform && tm == kTimeUniform)
+                            bwd_block<false, C, true>(sv, dp, dg, c0, false, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
+                        else if (tm == kTimeUniform)
+                            bwd_block<false, C>(sv, dp, dg, c0, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
                         else if (tm >= 0)
-                            bwd_block<true, C>(sv, dp, dg, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
+                            bwd_block<true, C>(sv, dp, dg, c0, pm == kPosDiag, dlo, dhi, w_qrel, a_j, s_rth, nbm1, acc, g_rt, pa, pz);
                         else {
                             // element by element (MTGR candidates, ragged edges, int64-wide times)
                             int cur_p = -1, cur_t = -1;
