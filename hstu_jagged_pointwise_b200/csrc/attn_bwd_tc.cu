@@ -163,7 +163,6 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_
                                           bool pos_diag, float& dlo, float& dhi, const int32_t* qr, int32_t a_j,
                                           const float* rth, int nbm1, float& acc, float* g_rt,
                                           uint32_t (&pa)[C / 2], uint32_t (&pz)[C / 2]) {
-    const int lane = threadIdx.x & 31;
     int32_t q[C];
     if (TV) {
         const int4* q4 = reinterpret_cast<const int4*>(qr);

@@ -112,6 +112,8 @@ int check_dims(const hstu_dims* d) {
     if (!(d->alpha > 0.f) || !isfinite(d->alpha)) return HSTU_ERR_INVALID_ARG;
     if (!(d->ln_eps >= 0.f) || !isfinite(d->ln_eps)) return HSTU_ERR_INVALID_ARG;
     if ((long long)d->H * d->d_v > 8192) return HSTU_ERR_UNSUPPORTED;
+    // LayerNorm rows are held in registers: at most 8 x 4 x 32 vectors of 8 bf16 or 4 fp32
+    if (d->dtype == HSTU_F32 && (long long)d->H * d->d_v > 4096) return HSTU_ERR_UNSUPPORTED;
     return HSTU_OK;
 }
 

@@ -6,14 +6,14 @@
 //
 // HBM-bound: forward reads Y and U and writes O_pre (6D + 8 bytes per bf16
 // token incl. mean/rstd); backward reads dO_pre, U, Y, mean, rstd and writes
-// dY, dU (10D + 8 bytes per token).  One warp owns one token row; every lane
-// moves 16-byte vectors, rows are held in registers between the passes.
+// dY, dU (10D + 8 bytes per token).  Up to four warps share one token row; every
+// lane moves 16-byte vectors, rows are held in registers between the passes.
 #include "internal.h"
 
 namespace hstu {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr long long kLnMaxBlocks = 148 * 16;   // resident blocks of up to 4 warps
 
 template <typename T>
 struct Vec;
@@ -56,115 +56,145 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-__device__ __forceinline__ void load_f32x(const float* base, int c, int n, float* out) {
+// Rows are spread over WPR warps (one block per row at a time, grid-stride over rows):
+// thread t of the block owns the 16-byte vectors vi = k * 32 * WPR + t (k < NCW), so a
+// warp's lanes touch consecutive vectors.  gamma and beta stay in registers across rows;
+// row sums go through shared memory (one slot per reduction of a row).
+template <int WPR>
+__device__ __forceinline__ float block_sum(float x, float (*red)[4], int slot) {
+    x = warp_sum(x);
+    if (WPR == 1) return x;
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[slot][warp] = x;
+    __syncthreads();
+    float t = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; e++)
-        if (e < n) out[e] = base[c + e];
+    for (int w = 0; w < WPR; w++) t += red[slot][w];
+    return t;
 }
 
-// NC = vectors per lane (upper bound); D must be a multiple of Vec<T>::N.
-template <typename T, int NC>
-__global__ void __launch_bounds__(kWarps * 32) ln_fwd_kernel(LnParams p) {
+__device__ __forceinline__ void load_f32v(const float* base, int c, int n, float* out) {
+    if (n == 8) {
+        const float4 a = *reinterpret_cast<const float4*>(base + c);
+        const float4 b = *reinterpret_cast<const float4*>(base + c + 4);
+        out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+        out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(base + c);
+        out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    }
+}
+
+template <typename T, int WPR, int NCW>
+__global__ void __launch_bounds__(32 * WPR) ln_fwd_kernel(LnParams p) {
     constexpr int V = Vec<T>::N;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row = (long long)blockIdx.x * kWarps + warp;
-    if (row >= p.T) return;
+    __shared__ float red[2][4];
     const int nvec = p.D / V;
-    const size_t base = (size_t)row * p.D;
-    float x[NC][V];
-    float s = 0.f;
+    float gm[NCW][V], bt[NCW][V];
 #pragma unroll
-    for (int k = 0; k < NC; k++) {
-        const int vi = lane + 32 * k;
+    for (int k = 0; k < NCW; k++) {
+        const int vi = k * 32 * WPR + threadIdx.x;
         if (vi < nvec) {
-            Vec<T>::load(p.y, base + (size_t)vi * V, x[k]);
-#pragma unroll
-            for (int e = 0; e < V; e++) s += x[k][e];
+            load_f32v(p.gamma, vi * V, V, gm[k]);
+            load_f32v(p.beta, vi * V, V, bt[k]);
         }
     }
-    const float mean = warp_sum(s) / p.D;
-    float q = 0.f;
+    for (long long row = blockIdx.x; row < p.T; row += gridDim.x) {
+        const size_t base = (size_t)row * p.D;
+        float x[NCW][V], u[NCW][V];
+        float s = 0.f;
 #pragma unroll
-    for (int k = 0; k < NC; k++) {
-        const int vi = lane + 32 * k;
-        if (vi < nvec) {
+        for (int k = 0; k < NCW; k++) {
+            const int vi = k * 32 * WPR + threadIdx.x;
+            if (vi < nvec) {
+                Vec<T>::load(p.y, base + (size_t)vi * V, x[k]);
+                Vec<T>::load(p.u, base + (size_t)vi * V, u[k]);
 #pragma unroll
-            for (int e = 0; e < V; e++) {
-                const float d = x[k][e] - mean;
-                q += d * d;
+                for (int e = 0; e < V; e++) s += x[k][e];
             }
         }
-    }
-    const float rstd = rsqrtf(warp_sum(q) / p.D + p.eps);
+        const float mean = block_sum<WPR>(s, red, 0) / p.D;
+        float q = 0.f;
 #pragma unroll
-    for (int k = 0; k < NC; k++) {
-        const int vi = lane + 32 * k;
-        if (vi < nvec) {
-            float u[V], g[8], bb[8], o[V];
-            Vec<T>::load(p.u, base + (size_t)vi * V, u);
-            load_f32x(p.gamma, vi * V, V, g);
-            load_f32x(p.beta, vi * V, V, bb);
+        for (int k = 0; k < NCW; k++) {
+            const int vi = k * 32 * WPR + threadIdx.x;
+            if (vi < nvec) {
 #pragma unroll
-            for (int e = 0; e < V; e++) o[e] = ((x[k][e] - mean) * rstd * g[e] + bb[e]) * u[e];
-            Vec<T>::store(p.o, base + (size_t)vi * V, o);
+                for (int e = 0; e < V; e++) {
+                    const float d = x[k][e] - mean;
+                    q += d * d;
+                }
+            }
         }
-    }
-    if (lane == 0) {
-        if (p.mean) p.mean[row] = mean;
-        if (p.rstd) p.rstd[row] = rstd;
+        const float rstd = rsqrtf(block_sum<WPR>(q, red, 1) / p.D + p.eps);
+#pragma unroll
+        for (int k = 0; k < NCW; k++) {
+            const int vi = k * 32 * WPR + threadIdx.x;
+            if (vi < nvec) {
+                float o[V];
+#pragma unroll
+                for (int e = 0; e < V; e++) o[e] = ((x[k][e] - mean) * rstd * gm[k][e] + bt[k][e]) * u[k][e];
+                Vec<T>::store(p.o, base + (size_t)vi * V, o);
+            }
+        }
+        if (threadIdx.x == 0) {
+            if (p.mean) p.mean[row] = mean;
+            if (p.rstd) p.rstd[row] = rstd;
+        }
     }
 }
 
-// Grid-stride over rows; each block leaves its partial dgamma / dbeta in p.part[block].
-template <typename T, int NC>
-__global__ void __launch_bounds__(kWarps * 32) ln_bwd_kernel(LnParams p) {
+// Each block leaves its partial dgamma / dbeta in p.part[block]: every column is owned by
+// one thread of the block, so the partials are deterministic for a given grid.
+template <typename T, int WPR, int NCW>
+__global__ void __launch_bounds__(32 * WPR) ln_bwd_kernel(LnParams p) {
     constexpr int V = Vec<T>::N;
-    extern __shared__ float s_acc[];                 // [2][D]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ float red[2][4];
     const int nvec = p.D / V;
-    for (int c = threadIdx.x; c < 2 * p.D; c += blockDim.x) s_acc[c] = 0.f;
-    float ag[NC][V], ab[NC][V];
+    float gm[NCW][V], bt[NCW][V], ag[NCW][V], ab[NCW][V];
 #pragma unroll
-    for (int k = 0; k < NC; k++)
+    for (int k = 0; k < NCW; k++) {
+        const int vi = k * 32 * WPR + threadIdx.x;
 #pragma unroll
         for (int e = 0; e < V; e++) ag[k][e] = ab[k][e] = 0.f;
-    __syncthreads();
-    for (long long row = (long long)blockIdx.x * kWarps + warp; row < p.T;
-         row += (long long)gridDim.x * kWarps) {
+        if (vi < nvec) {
+            load_f32v(p.gamma, vi * V, V, gm[k]);
+            load_f32v(p.beta, vi * V, V, bt[k]);
+        }
+    }
+    for (long long row = blockIdx.x; row < p.T; row += gridDim.x) {
         const size_t base = (size_t)row * p.D;
         const float mean = p.mean[row], rstd = p.rstd[row];
-        float xh[NC][V], gx[NC][V];
+        float xh[NCW][V], gx[NCW][V];
         float m1 = 0.f, m2 = 0.f;
 #pragma unroll
-        for (int k = 0; k < NC; k++) {
-            const int vi = lane + 32 * k;
+        for (int k = 0; k < NCW; k++) {
+            const int vi = k * 32 * WPR + threadIdx.x;
             if (vi < nvec) {
-                float y[V], u[V], g[V], gm[8], bt[8], du[V];
+                float y[V], u[V], g[V], du[V];
                 Vec<T>::load(p.y, base + (size_t)vi * V, y);
                 Vec<T>::load(p.u, base + (size_t)vi * V, u);
                 Vec<T>::load(p.g, base + (size_t)vi * V, g);
-                load_f32x(p.gamma, vi * V, V, gm);
-                load_f32x(p.beta, vi * V, V, bt);
 #pragma unroll
                 for (int e = 0; e < V; e++) {
                     xh[k][e] = (y[e] - mean) * rstd;
-                    du[e] = g[e] * (xh[k][e] * gm[e] + bt[e]);
+                    du[e] = g[e] * (xh[k][e] * gm[k][e] + bt[k][e]);
                     const float gl = g[e] * u[e];
                     ag[k][e] += gl * xh[k][e];
                     ab[k][e] += gl;
-                    gx[k][e] = gl * gm[e];
+                    gx[k][e] = gl * gm[k][e];
                     m1 += gx[k][e];
                     m2 += gx[k][e] * xh[k][e];
                 }
                 Vec<T>::store(p.du, base + (size_t)vi * V, du);
             }
         }
-        m1 = warp_sum(m1) / p.D;
-        m2 = warp_sum(m2) / p.D;
+        m1 = block_sum<WPR>(m1, red, 0) / p.D;
+        m2 = block_sum<WPR>(m2, red, 1) / p.D;
         const float rs = rstd * p.dy_scale;
 #pragma unroll
-        for (int k = 0; k < NC; k++) {
-            const int vi = lane + 32 * k;
+        for (int k = 0; k < NCW; k++) {
+            const int vi = k * 32 * WPR + threadIdx.x;
             if (vi < nvec) {
                 float dy[V];
 #pragma unroll
@@ -173,76 +203,97 @@ __global__ void __launch_bounds__(kWarps * 32) ln_bwd_kernel(LnParams p) {
             }
         }
     }
+    float* part = p.part + (size_t)blockIdx.x * 2 * p.D;
 #pragma unroll
-    for (int k = 0; k < NC; k++) {
-        const int vi = lane + 32 * k;
+    for (int k = 0; k < NCW; k++) {
+        const int vi = k * 32 * WPR + threadIdx.x;
         if (vi < nvec) {
 #pragma unroll
             for (int e = 0; e < V; e++) {
-                atomicAdd(&s_acc[vi * V + e], ag[k][e]);
-                atomicAdd(&s_acc[p.D + vi * V + e], ab[k][e]);
+                part[vi * V + e] = ag[k][e];
+                part[p.D + vi * V + e] = ab[k][e];
             }
         }
     }
-    __syncthreads();
-    float* part = p.part + (size_t)blockIdx.x * 2 * p.D;
-    for (int c = threadIdx.x; c < 2 * p.D; c += blockDim.x) part[c] = s_acc[c];
 }
 
-// Sums the per-block partials (fixed order: deterministic).
-__global__ void ln_bwd_reduce_kernel(LnParams p) {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= 2 * p.D) return;
+// Sums the per-block partials in a fixed order (deterministic): a block owns 32 of the
+// 2D columns; warp w sums the partials w, w+8, w+16, ... of each column (coalesced
+// 128-byte rows), and warp 0 adds the eight warp sums in order.
+__global__ void __launch_bounds__(256) ln_bwd_reduce_kernel(LnParams p) {
+    __shared__ float acc[8][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * 32 + lane;
     float s = 0.f;
-    for (int k = 0; k < p.n_part; k++) s += p.part[(size_t)k * 2 * p.D + c];
-    if (c < p.D) p.d_gamma[c] = s;
-    else p.d_beta[c - p.D] = s;
+    if (c < 2 * p.D)
+        for (int k = warp; k < p.n_part; k += 8) s += p.part[(size_t)k * 2 * p.D + c];
+    acc[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0 && c < 2 * p.D) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; w++) t += acc[w][lane];
+        if (c < p.D) p.d_gamma[c] = t;
+        else p.d_beta[c - p.D] = t;
+    }
 }
+
+// Warps per row and 16-byte vectors per thread for a row of D elements.
+template <typename T>
+bool pick_shape(int D, int* wpr, int* ncw) {
+    constexpr int V = Vec<T>::N;
+    const int nvec = D / V;
+    *wpr = nvec > 64 ? 4 : (nvec > 32 ? 2 : 1);   // below four warps one vector per thread
+    const int per = 32 * *wpr;
+    const int n = (nvec + per - 1) / per;
+    *ncw = n <= 1 ? 1 : (n <= 2 ? 2 : (n <= 4 ? 4 : (n <= 8 ? 8 : 0)));
+    return *ncw != 0;
+}
+
+#define HSTU_LN_DISPATCH(KERNEL, GRID, WPR_, NCW_)                                          \
+    do {                                                                                     \
+        if (WPR_ == 1) KERNEL<T, 1, 1><<<GRID, 32, 0, s>>>(p);                              \
+        else if (WPR_ == 2) KERNEL<T, 2, 1><<<GRID, 64, 0, s>>>(p);                          \
+        else if (NCW_ == 1) KERNEL<T, 4, 1><<<GRID, 128, 0, s>>>(p);                         \
+        else if (NCW_ == 2) KERNEL<T, 4, 2><<<GRID, 128, 0, s>>>(p);                         \
+        else if (NCW_ == 4) KERNEL<T, 4, 4><<<GRID, 128, 0, s>>>(p);                         \
+        else KERNEL<T, 4, 8><<<GRID, 128, 0, s>>>(p);                                        \
+    } while (0)
 
 template <typename T>
 cudaError_t fwd_t(const LnParams& p, cudaStream_t s) {
-    constexpr int V = Vec<T>::N;
-    const int nc = (p.D / V + 31) / 32;
-    const unsigned grid = (unsigned)((p.T + kWarps - 1) / kWarps);
-    if (nc > 8) return cudaErrorInvalidValue;
+    int wpr = 0, ncw = 0;
+    if (!pick_shape<T>(p.D, &wpr, &ncw)) return cudaErrorInvalidValue;
+    const unsigned grid = (unsigned)(p.T < kLnMaxBlocks ? p.T : kLnMaxBlocks);
     prof_begin(kProfLnFwd, s);
-    if (nc <= 1) ln_fwd_kernel<T, 1><<<grid, kWarps * 32, 0, s>>>(p);
-    else if (nc <= 2) ln_fwd_kernel<T, 2><<<grid, kWarps * 32, 0, s>>>(p);
-    else if (nc <= 4) ln_fwd_kernel<T, 4><<<grid, kWarps * 32, 0, s>>>(p);
-    else ln_fwd_kernel<T, 8><<<grid, kWarps * 32, 0, s>>>(p);
+    HSTU_LN_DISPATCH(ln_fwd_kernel, grid, wpr, ncw);
     prof_end(kProfLnFwd, s);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t bwd_t(const LnParams& p, cudaStream_t s) {
-    constexpr int V = Vec<T>::N;
-    const int nc = (p.D / V + 31) / 32;
-    const size_t smem = 2 * (size_t)p.D * 4;
+    int wpr = 0, ncw = 0;
+    if (!pick_shape<T>(p.D, &wpr, &ncw)) return cudaErrorInvalidValue;
     const unsigned grid = (unsigned)p.n_part;
-    if (nc > 8) return cudaErrorInvalidValue;
     prof_begin(kProfLnBwd, s);
-    if (nc <= 1) ln_bwd_kernel<T, 1><<<grid, kWarps * 32, smem, s>>>(p);
-    else if (nc <= 2) ln_bwd_kernel<T, 2><<<grid, kWarps * 32, smem, s>>>(p);
-    else if (nc <= 4) ln_bwd_kernel<T, 4><<<grid, kWarps * 32, smem, s>>>(p);
-    else ln_bwd_kernel<T, 8><<<grid, kWarps * 32, smem, s>>>(p);
+    HSTU_LN_DISPATCH(ln_bwd_kernel, grid, wpr, ncw);
     prof_end(kProfLnBwd, s);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     prof_begin(kProfLnBwdReduce, s);
-    ln_bwd_reduce_kernel<<<(2 * p.D + 255) / 256, 256, 0, s>>>(p);
+    ln_bwd_reduce_kernel<<<(2 * p.D + 31) / 32, 256, 0, s>>>(p);
     prof_end(kProfLnBwdReduce, s);
     return cudaGetLastError();
 }
 
+#undef HSTU_LN_DISPATCH
+
 }  // namespace
 
 int ln_bwd_partials(long long T) {
-    long long rows_per_block = kWarps * 8;   // at least 8 rows per warp
-    long long n = (T + rows_per_block - 1) / rows_per_block;
-    if (n < 1) n = 1;
-    if (n > 1184) n = 1184;                  // 8 blocks per SM on 148 SMs
-    return (int)n;
+    long long n = T < kLnMaxBlocks ? T : kLnMaxBlocks;   // one block per row, grid-stride beyond
+    return n < 1 ? 1 : (int)n;
 }
 
 cudaError_t launch_ln_fwd(int dtype_f32, const LnParams& p, cudaStream_t s) {

@@ -41,7 +41,8 @@
  *    clear it with hstu_check_device_error().
  *  - Alignment: every tensor pointer 16-byte aligned; H*d*elem_size a multiple of 16.
  *  - Supported: dtype HSTU_BF16 with d_qk = d_v in {64, 128}; dtype HSTU_F32 with
- *    d_qk = d_v in {32, 64, 128}; P in [1, 1024]; nb in [1, 64]; H >= 1; H*d_v <= 8192;
+ *    d_qk = d_v in {32, 64, 128}; P in [1, 1024]; nb in [1, 64]; H >= 1; H*d_v <= 8192
+ *    (<= 4096 for HSTU_F32);
  *    max_seq_len <= 524287.
  */
 #ifndef HSTU_B200_H

@@ -70,6 +70,9 @@ def test_fwd_rejects_bad_arguments_before_launch():
     # unsupported width
     d2 = dims(d_qk=48, d_v=48)
     assert capi.LIB.hstu_attn_fwd(C.byref(d2), C.byref(m), *nulls, 0, None) == capi.HSTU_ERR_UNSUPPORTED
+    # fp32 rows wider than 4096 (LayerNorm rows are held in registers)
+    d3 = dims(dtype=capi.HSTU_F32, H=33, d_qk=128, d_v=128)
+    assert capi.LIB.hstu_attn_fwd(C.byref(d3), C.byref(m), *nulls, 0, None) == capi.HSTU_ERR_UNSUPPORTED
     # MTGR without segment arrays
     m2 = capi.HstuMaskSpec(kind=1, n_static=None, n_realtime=None)
     assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m2), *nulls, 0, None) == capi.HSTU_ERR_INVALID_ARG
