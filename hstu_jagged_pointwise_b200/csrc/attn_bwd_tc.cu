@@ -379,12 +379,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             q_use[hh]++;
             if (!w) return false;
             tc_fence_after();
+            const uint64_t dK = sdesc_sw128(aK, 16, 1024), dQ = sdesc_sw128(aQ[hh], 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; kk++) {
                 const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
                 const uint32_t offh = (kk >> 2) * kHalfPanel + (kk & 3) * 32;
-                mma_ss(tmem + kSCol + 64 * hh, sdesc_sw128(aK + off, 16, 1024),
-                       sdesc_sw128(aQ[hh] + offh, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+                mma_ss(tmem + kSCol + 64 * hh, dK + (off >> 4), dQ + (offh >> 4), kIdSP, kk > 0 ? 1u : 0u);
             }
             return true;
         };
@@ -395,12 +395,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (!w) return false;
             dy_use[hh]++;
             tc_fence_after();
+            const uint64_t dV = sdesc_sw128(aV, 16, 1024), dY = sdesc_sw128(aDY[hh], 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; kk++) {
                 const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
                 const uint32_t offh = (kk >> 2) * kHalfPanel + (kk & 3) * 32;
-                mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aV + off, 16, 1024),
-                       sdesc_sw128(aDY[hh] + offh, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+                mma_ss(tmem + kPCol + 64 * hh, dV + (off >> 4), dY + (offh >> 4), kIdSP, kk > 0 ? 1u : 0u);
             }
             tc_commit(&bars[kSFull0 + hh]);
             return true;
@@ -413,27 +413,27 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tc_fence_after();
             // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys); first,
             // so that its drain overlaps the two products below
+            const uint64_t dKm = sdesc_sw128(aK, kPanel, 1024), dZm = sdesc_sw128(aDZ[hh], 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 8; kk++) {
-                mma_ss(tmem + kPCol + 64 * hh, sdesc_sw128(aK + kk * 2048, kPanel, 1024),
-                       sdesc_sw128(aDZ[hh] + kk * 2048, 16, 1024), kIdQ, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 8; kk++)
+                mma_ss(tmem + kPCol + 64 * hh, dKm + (kk * 2048 >> 4), dZm + (kk * 2048 >> 4), kIdQ, kk > 0 ? 1u : 0u);
             dq_use[hh]++;
             tc_commit(&bars[kDQFull0 + hh]);
+            const uint64_t dYm = sdesc_sw128(aDY[hh], kHalfPanel, 1024);
             // dV += A^T_h dY'_h   (A^T_h: the kEwCols queries of group c packed into columns
             // 64h + kEwCols*c .. +kEwCols/2)
 #pragma unroll
             for (int kk = 0; kk < 4; kk++) {
                 const uint32_t acol = kSCol + 64 * hh + kEwCols * ((16 * kk) / kEwCols) + 8 * ((16 * kk) % kEwCols / 16);
-                mma_ts(tmem + kVCol, tmem + acol, sdesc_sw128(aDY[hh] + kk * 2048, kHalfPanel, 1024),
+                mma_ts(tmem + kVCol, tmem + acol, dYm + (kk * 2048 >> 4),
                        kIdV, (!init || kk > 0) ? 1u : 0u);
             }
             tc_commit(&bars[kDYEmpty0 + hh]);
+            const uint64_t dZk = sdesc_sw128(aDZ[hh], 16, 1024), dQm = sdesc_sw128(aQ[hh], kHalfPanel, 1024);
             // dK += dZ^T_h Q_h
 #pragma unroll
             for (int kk = 0; kk < 4; kk++) {
-                mma_ss(tmem + kKCol, sdesc_sw128(aDZ[hh] + kk * 32, 16, 1024),
-                       sdesc_sw128(aQ[hh] + kk * 2048, kHalfPanel, 1024), kIdK,
+                mma_ss(tmem + kKCol, dZk + (kk * 32 >> 4), dQm + (kk * 2048 >> 4), kIdK,
                        (!init || kk > 0) ? 1u : 0u);
             }
             tc_commit(&bars[kDZEmpty0 + hh]);

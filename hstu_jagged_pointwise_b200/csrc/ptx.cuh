@@ -166,7 +166,9 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version 1.
-// Start address, leading and stride byte offsets are encoded >> 4.
+// Start address, leading and stride byte offsets are encoded >> 4.  The start address
+// is the low field, so desc(a) + (off >> 4) == desc(a + off) for 16-byte multiples as
+// long as a + off stays below 256 KB (every shared-memory address does).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
                                                 uint32_t sbo_bytes) {
     uint64_t d = 0;
