@@ -290,6 +290,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int it_use = 0, q_use = 0, k_use = 0, v_use = 0, p_use = 0, o_use = 0;
         bool ok = true;
         const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+        // operand descriptors: per-buffer bases plus constant offsets
+        const uint64_t dQ = sdesc_sw128(aQ, 16, 1024), dK = sdesc_sw128(aK, 16, 1024);
+        const uint64_t dV = sdesc_sw128(aV, kPanelBytes, 1024);
         while (ok) {
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
@@ -321,8 +324,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                     for (int kk = 0; kk < D / 16; kk++) {
                         const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-                        mma_ss(tmem + kSCol, sdesc_sw128(aQ + off, 16, 1024),
-                               sdesc_sw128(aK + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + kSCol, dQ + (off >> 4), dK + (off >> 4), kIdescS, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&bars[kSFull]);
                     tc_commit(&bars[kKEmpty]);
@@ -342,7 +344,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int kk = 0; kk < kTileN / 16; kk++) {
                         // P of keys 32c .. 32c+31 sits in the first 16 columns of S chunk c
                         mma_ts(tmem + kOCol, tmem + kSCol + 32 * (kk >> 1) + 8 * (kk & 1),
-                               sdesc_sw128(aV + kk * 2048, kPanelBytes, 1024), kIdescO,
+                               dV + (kk * 2048 >> 4), kIdescO,
                                (n_done > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&bars[kVEmpty]);
@@ -407,19 +409,32 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             const bool warp_rows = pr_lo <= pr_hi;          // any valid row in this warp
             const int n_kt = (s.Lk + kTileN - 1) / kTileN;
+            // column timestamps of this warp's keys, loaded one key tile ahead
+            auto next_tile = [&](int tt) {
+                for (tt++; tt < n_kt; tt++)
+                    if (kv_class<KIND>(s, tt) != 0) break;
+                return tt;
+            };
+            int64_t tj_next[2];
+            auto load_tj = [&](int tt) {
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    const int j = tt * kTileN + 64 * g + lane + 32 * e;
+                    tj_next[e] = (tt < n_kt && j < s.Lk) ? __ldg(p.kv_ts + s.kv0 + j) : 0;
+                }
+            };
             int n_done = 0;
-            for (int t = 0; t < n_kt; t++) {
-                const int cls = kv_class<KIND>(s, t);
-                if (cls == 0) continue;
+            int t = next_tile(-1);
+            load_tj(t);
+            for (; t < n_kt; t = next_tile(t)) {
                 const int n0 = t * kTileN + 64 * g;         // first key of this warp's half
-                // column timestamps of this warp's keys
                 __syncwarp();
-                int64_t tj[2];
+                int64_t tj[2] = {tj_next[0], tj_next[1]};
+                load_tj(next_tile(t));
                 int64_t cmin = INT64_MAX, cmax = INT64_MIN;
 #pragma unroll
                 for (int e = 0; e < 2; e++) {
                     const int j = n0 + lane + 32 * e;
-                    tj[e] = j < s.Lk ? p.kv_ts[s.kv0 + j] : 0;
                     if (j < s.Lk) {
                         cmin = min(cmin, tj[e]);
                         cmax = max(cmax, tj[e]);
