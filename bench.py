@@ -98,6 +98,56 @@ def alu_fp32_peak_tflops(sm_mhz: float) -> float:
 # clocks during the timed region
 # ----------------------------------------------------------------------------
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons every 10 ms through NVML (read-only queries)."""
+    PERIOD_S = 0.01
+
+    def __init__(self, device_index: int):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(device_index)
+        bus = "%08X:%02X:%02X.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id, props.pci_device_id)
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.bits = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                     "hw_thermal_slowdown": 0x40}
+        self.samples, self.reasons = [], set()
+        self.stop_flag = threading.Event()
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(float(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)))
+                r = int(self.get_reasons(self.h))
+                for name, bit in self.bits.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except self.nv.NVMLError:
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def start(self):
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self) -> dict:
+        self.stop_flag.set()
+        self.thread.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml"}
+
+
+def make_clock_sampler(device_index: int):
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
+
+
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -280,7 +330,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"device status {capi.status_string(st)} after warm-up")
 
     # ---- device-timed region
-    sampler = ClockSampler(local)
+    sampler = make_clock_sampler(local)
     capi.profile_enable(True)
     barrier(world)
     torch.cuda.synchronize()
@@ -499,7 +549,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
