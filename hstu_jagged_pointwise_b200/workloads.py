@@ -43,7 +43,7 @@ MASK_MTGR = 1
 class Workload:
     """One batch of synthetic inputs (torch CPU tensors / numpy arrays)."""
     name: str
-    kind: str                      # "causal" | "mtgr" | "mfalcon"
+    kind: str                      # "causal" | "mtgr" | "mfalcon" | "mfalcon_seq"
     dtype: torch.dtype             # element type of q/k/v/u (bf16 or fp32)
     H: int
     d: int
@@ -63,7 +63,7 @@ class Workload:
     v: Optional[torch.Tensor] = None
     u: Optional[torch.Tensor] = None
     n_static: Optional[np.ndarray] = None     # int32 [B] (mtgr)
-    n_realtime: Optional[np.ndarray] = None   # int32 [B] (mtgr)
+    n_realtime: Optional[np.ndarray] = None   # int32 [B] (mtgr; history length for mfalcon_seq)
     grad: Optional[torch.Tensor] = None       # upstream gradient of o_pre [T, H*d]
     # M-FALCON layout
     hist_offsets: Optional[np.ndarray] = None
@@ -289,6 +289,35 @@ def make_mfalcon(n_hist, n_cand, H: int, d: int, dtype=torch.bfloat16, seed: int
                     hist_k=hk, hist_v=hv, cand_offsets=co,
                     cand_ts=np.concatenate(cand_ts) if Tc else np.zeros(0, np.int64),
                     cand_q=cq, cand_k=ck, cand_v=cv, cand_u=cu, b_m=b_m)
+
+
+def mfalcon_seq_from(w: Workload, seed: int = 0, name: str = "mfalcon_seq") -> Workload:
+    """The same users as an M-FALCON workload, laid out as one jagged row per user:
+    [history ; candidates].  History K/V and all candidate tensors are w's; the
+    history Q and U (which the cached layout does not need) are drawn here."""
+    gen = torch.Generator().manual_seed(seed)
+    ho, co = np.asarray(w.hist_offsets, np.int64), np.asarray(w.cand_offsets, np.int64)
+    n_hist, n_cand = np.diff(ho), np.diff(co)
+    D = w.H * w.d
+    hq = randn(gen, (int(ho[-1]), D), w.dtype)
+    hu = randn(gen, (int(ho[-1]), D), w.dtype)
+    rows_h = [np.arange(ho[b], ho[b + 1]) for b in range(len(n_hist))]
+    rows_c = [np.arange(co[b], co[b + 1]) for b in range(len(n_cand))]
+
+    def cat(hist, cand):
+        parts = []
+        for rh, rc in zip(rows_h, rows_c):
+            parts.append(hist[torch.as_tensor(rh, dtype=torch.long)])
+            parts.append(cand[torch.as_tensor(rc, dtype=torch.long)])
+        return torch.cat(parts) if parts else hist[:0]
+
+    ts = np.concatenate([np.concatenate([w.hist_ts[ho[b]:ho[b + 1]], w.cand_ts[co[b]:co[b + 1]]])
+                         for b in range(len(n_hist))]) if len(n_hist) else np.zeros(0, np.int64)
+    return Workload(name=name, kind="mfalcon_seq", dtype=w.dtype, H=w.H, d=w.d, alpha=w.alpha,
+                    rab_pos=w.rab_pos, rab_time=w.rab_time, gamma=w.gamma, beta=w.beta,
+                    offsets=_offsets(n_hist + n_cand).astype(np.int32), ts=ts.astype(np.int64),
+                    q=cat(hq, w.cand_q), k=cat(w.hist_k, w.cand_k), v=cat(w.hist_v, w.cand_v),
+                    u=cat(hu, w.cand_u), n_realtime=n_hist.astype(np.int32))
 
 
 # ----------------------------------------------------------------------------

@@ -27,6 +27,7 @@ _lib = None
 
 MASK_CAUSAL = 0
 MASK_MTGR = 1
+MASK_MFSEQ = 2   # full-sequence M-FALCON: [history ; candidates], n_realtime = history length
 
 
 def build(force: bool = False) -> str:
@@ -102,12 +103,14 @@ def _ptr(a):
 
 
 def _kind(w) -> int:
-    return MASK_MTGR if w.kind == "mtgr" else MASK_CAUSAL
+    return {"mtgr": MASK_MTGR, "mfalcon_seq": MASK_MFSEQ}.get(w.kind, MASK_CAUSAL)
 
 
 def _segs(w):
     if w.kind == "mtgr":
         return _c(w.n_static, np.int32), _c(w.n_realtime, np.int32)
+    if w.kind == "mfalcon_seq":
+        return np.zeros(len(w.n_realtime), np.int32), _c(w.n_realtime, np.int32)
     return None, None
 
 

@@ -20,6 +20,10 @@
  *       candidate sees history only with a strictly earlier timestamp.
  *     M-FALCON (HSTU blog, sections 4.2-4.3): candidates see the whole cached
  *       history and themselves, never each other.
+ *     Full-sequence M-FALCON (HSTU blog, section 4.2, the single pass over
+ *       [history ; candidates] before caching): history tokens causal among
+ *       themselves, each candidate sees every history token and itself; no
+ *       timestamp filter.
  *
  * Readings where the pages are silent (each also listed with the design notes):
  *   - alpha divides A after SiLU (Y = sum_j mask*SiLU(z)*v / alpha); no 1/sqrt(d).
@@ -44,6 +48,7 @@
 
 #define ORACLE_CAUSAL 0
 #define ORACLE_MTGR 1
+#define ORACLE_MFSEQ 2      /* full-sequence M-FALCON: n_rt[b] = history length, no static part */
 
 /* ------------------------------------------------------------------ */
 /* index rules                                                         */
@@ -58,7 +63,7 @@ static int token_class(int64_t i, int64_t S, int64_t R) {
 
 /* position used by the relative position bias */
 static int64_t token_pos(int kind, int64_t i, int64_t S, int64_t R) {
-    if (kind == ORACLE_MTGR && i >= S + R) return S + R;
+    if ((kind == ORACLE_MTGR || kind == ORACLE_MFSEQ) && i >= S + R) return S + R;
     return i;
 }
 
@@ -92,6 +97,7 @@ static int visible(int kind, int64_t i, int64_t j, int64_t S, int64_t R, const i
     if (ci == 0) return cj == 0;
     if (ci == 1) return cj == 0 || (cj == 1 && j <= i);
     if (j == i) return 1;
+    if (kind == ORACLE_MFSEQ) return cj != 2;
     return cj != 2 && ts[j] < ts[i];
 }
 
@@ -118,6 +124,9 @@ static void seg_sizes(int kind, const int32_t* n_static, const int32_t* n_rt, in
                       int64_t* S, int64_t* R) {
     if (kind == ORACLE_MTGR) {
         *S = n_static[b];
+        *R = n_rt[b];
+    } else if (kind == ORACLE_MFSEQ) {
+        *S = 0;
         *R = n_rt[b];
     } else {
         *S = L;

@@ -297,6 +297,32 @@ def test_mtgr_candidates_reduce_to_mfalcon():
     np.testing.assert_allclose(oracle.mfalcon(wm), y[n:], rtol=1e-13, atol=1e-14)
 
 
+def test_full_sequence_mfalcon_matches_cache_and_causal_history():
+    """[history ; candidates] in one pass: candidate rows equal the cached M-FALCON
+    scores (no timestamp filter: some candidates share the last history timestamp),
+    history rows equal a causal layer over the history alone."""
+    wm = W.make_mfalcon([0, 17, 130], [3, 5, 2], H=2, d=8, dtype=torch.float32, seed=24, alpha=131.0)
+    ho = np.asarray(wm.hist_offsets)
+    for b in range(len(ho) - 1):          # a candidate at the same second as the last history token
+        if ho[b + 1] > ho[b]:
+            wm.cand_ts[wm.cand_offsets[b]] = wm.hist_ts[ho[b + 1] - 1]
+    ws = W.mfalcon_seq_from(wm, seed=3)
+    y = oracle.attn_fwd(ws)
+    off = np.asarray(ws.offsets)
+    cand_rows = np.concatenate([np.arange(off[b] + ws.n_realtime[b], off[b + 1]) for b in range(len(off) - 1)])
+    np.testing.assert_allclose(y[cand_rows], oracle.mfalcon(wm), rtol=1e-12, atol=1e-14)
+    for b in range(len(off) - 1):
+        n = int(ws.n_realtime[b])
+        if n == 0:
+            continue
+        rows = slice(off[b], off[b] + n)
+        wc = W.make_causal([n], H=2, d=8, dtype=torch.float32, seed=1, alpha=ws.alpha,
+                           ts_list=[ws.ts[rows]])
+        wc.q, wc.k, wc.v = ws.q[rows], ws.k[rows], ws.v[rows]
+        wc.rab_pos, wc.rab_time = ws.rab_pos, ws.rab_time
+        np.testing.assert_allclose(y[rows], oracle.attn_fwd(wc), rtol=1e-12, atol=1e-14)
+
+
 # ----------------------------------------------------------------------------
 # LayerNorm (.) U
 # ----------------------------------------------------------------------------
