@@ -507,12 +507,56 @@ def run_mfalcon(args, world, rank, local):
     if m.check_device_error() != 0:
         raise RuntimeError("device status set in M-FALCON")
     n_c = w.T
-    pairs = int(w.H * np.sum(np.diff(w.cand_offsets) * (np.diff(w.hist_offsets) + 1)))
+    nh, nc = np.diff(w.hist_offsets).astype(np.int64), np.diff(w.cand_offsets).astype(np.int64)
+    pairs = int(w.H * np.sum(nc * (nh + 1)))
     pk, _ = peaks()
     tfl = 4 * w.d * pairs / (ms * 1e-3) / 1e12
+    del d, out, m
+    seq = run_mfalcon_seq(args, world, w, dev)
     return {"workload": w.name, "cands_per_s": round(world * n_c / (ms * 1e-3), 1), "ms_per_pass": round(ms, 4),
             "tflops": round(world * tfl, 3), "pct_bf16_peak": round(tfl / pk["bf16_tflops_sustained"], 4),
-            "b_m": w.b_m}
+            "b_m": w.b_m, "full_sequence": seq}
+
+
+def run_mfalcon_seq(args, world, w, dev):
+    """The same users as one jagged row each, [history ; candidates], through the
+    attention forward with the full-sequence M-FALCON mask: history rows causal,
+    candidates against all history and themselves."""
+    from hstu_jagged_pointwise_b200 import ops
+    ws = W.mfalcon_seq_from(w, seed=args.seed + 1)
+    t = {n: getattr(ws, n).to(dev) for n in ("q", "k", "v", "u", "rab_pos", "rab_time", "gamma", "beta")}
+    off = torch.as_tensor(ws.offsets).to(dev)
+    ts = torch.as_tensor(ws.ts).to(dev)
+    nr = torch.as_tensor(ws.n_realtime).to(dev)
+    layer = ops.Layer(off, ts, ws.H, ws.d, ws.dtype, ws.alpha, ws.max_len, mask_kind="mfalcon_seq", n_realtime=nr)
+    out = dict(y=torch.empty_like(t["q"]), o_pre=torch.empty_like(t["q"]),
+               mean=torch.empty(ws.T, dtype=torch.float32, device=dev),
+               rstd=torch.empty(ws.T, dtype=torch.float32, device=dev))
+
+    def go():
+        layer.forward(t["q"], t["k"], t["v"], t["u"], t["rab_pos"], t["rab_time"], t["gamma"], t["beta"], out=out)
+
+    for _ in range(args.warmup):
+        go()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        go()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    if layer.check_device_error() != 0:
+        raise RuntimeError("device status set in the full-sequence M-FALCON forward")
+    nh, nc = np.diff(w.hist_offsets).astype(np.int64), np.diff(w.cand_offsets).astype(np.int64)
+    pairs = int(w.H * np.sum(nh * (nh + 1) // 2 + nc * (nh + 1)))
+    pk, _ = peaks()
+    tfl = 4 * w.d * pairs / (ms * 1e-3) / 1e12
+    return {"workload": f"{w.name}_one_row", "tokens": int(ws.T), "cands_per_s": round(world * w.T / (ms * 1e-3), 1),
+            "ms_per_pass": round(ms, 4), "tflops": round(world * tfl, 3),
+            "pct_bf16_peak": round(tfl / pk["bf16_tflops_sustained"], 4)}
 
 
 # ----------------------------------------------------------------------------

@@ -23,6 +23,7 @@ HSTU_BF16 = 0
 HSTU_F32 = 1
 HSTU_MASK_CAUSAL = 0
 HSTU_MASK_MTGR = 1
+HSTU_MASK_MFALCON_SEQ = 2
 
 # every symbol the header declares
 EXPORTS = (

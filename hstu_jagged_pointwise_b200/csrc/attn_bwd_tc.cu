@@ -104,13 +104,7 @@ __device__ __forceinline__ KvItem load_kv_item(const BwdParams& p, int4 it) {
     s.b = it.x; s.n0 = it.y; s.h = it.z; s.n_end = it.w;
     s.off0 = p.off[s.b];
     s.L = p.off[s.b + 1] - s.off0;
-    if (KIND == HSTU_KIND_MTGR) {
-        s.S = p.n_static[s.b];
-        s.R = p.n_rt[s.b];
-    } else {
-        s.S = s.L;
-        s.R = 0;
-    }
+    segment_sizes(KIND, p.n_static, p.n_rt, s.b, s.L, &s.S, &s.R);
     return s;
 }
 

@@ -75,13 +75,7 @@ __device__ __forceinline__ Item load_item(const FwdParams& p, int4 it) {
     s.Lq = p.q_off[s.b + 1] - s.q0;
     s.kv0 = p.kv_off[s.b];
     s.Lk = p.kv_off[s.b + 1] - s.kv0;
-    if (KIND == HSTU_KIND_MTGR) {
-        s.S = p.n_static[s.b];
-        s.R = p.n_rt[s.b];
-    } else {
-        s.S = s.Lq;
-        s.R = 0;
-    }
+    segment_sizes(KIND, p.n_static, p.n_rt, s.b, s.Lq, &s.S, &s.R);
     return s;
 }
 
@@ -457,8 +451,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                ? 2
                                : tile_class(KIND, r0, min(r0 + 31, s.row_end - 1), n0,
                                             min(n0 + 63, s.Lk - 1), s.S, s.R);
-                const bool dense = wcls != 0 && n0 + 64 <= s.Lk &&
-                                   (KIND == HSTU_KIND_CAUSAL || wcls == 2);
+                const int r_hi = min(r0 + 31, s.row_end - 1);
+                // every row of the block is a candidate sharing one position
+                const bool rows_shared = KIND == HSTU_KIND_MFALCON || (KIND != HSTU_KIND_CAUSAL && r0 >= s.S + s.R);
+                // real-time / history rows against real-time / history keys: the mask is j <= i
+                const bool causal_rows = KIND == HSTU_KIND_CAUSAL ||
+                                         (KIND != HSTU_KIND_MFALCON && r0 >= s.S && r_hi < s.S + s.R &&
+                                          n0 >= s.S && n0 + 63 < s.S + s.R);
+                const bool dense = wcls != 0 && n0 + 64 <= s.Lk && (wcls == 2 || causal_rows);
                 if (dense) {
                     tc = classify_time(rmin, rmax, cmin, cmax, p.nb);
                     const int dmax = col_pos<KIND>(s, n0 + 63) - pr_lo;
@@ -466,20 +466,26 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     int pidx_u = -1;
                     if (wcls == 2 && dmax <= -(p.P - 1)) pidx_u = 0;
                     else if (wcls == 2 && dmin >= p.P - 1) pidx_u = 2 * p.P - 2;
+                    // a dense block's rows are all candidates or all indexed by position
+                    // (pos_j - pos_i == j - i): one tile class never mixes the two
                     if (pidx_u >= 0) pm = kPosUniform;
-                    else if (KIND != HSTU_KIND_MFALCON) pm = kPosDiag;
+                    else pm = rows_shared ? kPosCol : kPosDiag;
                     if (pm >= 0 && tc.mode >= 0) {
                         tm = tc.mode;
                         const float tadd = tm == kTimeUniform ? s_rth[tc.tb_lo] : 0.f;
                         if (pm == kPosUniform && tm == kTimeUniform) {
                             c0 = 0.5f * s_rp[pidx_u] + tadd;
+                        } else if (KIND != HSTU_KIND_CAUSAL && pm == kPosCol) {
+                            // one row position pr_lo: the bias of key n0 + k sits at w_diag[31 + k]
+                            for (int k = lane; k < 64; k += 32)
+                                w_diag[31 + k] = 0.5f * s_rp[pos_index(pr_lo, col_pos<KIND>(s, n0 + k), p.P)] + tadd;
                         } else {
                             // diagonal row: delta = j - i = (n0 - r0 - 31) + k, k in [0, 95);
                             // constant when the position index is clamped across the block
                             const int d0 = n0 - r0 - 31;
                             for (int k = lane; k < 95; k += 32) {
                                 const int dl = d0 + k;
-                                const bool masked = KIND == HSTU_KIND_CAUSAL && dl > 0;
+                                const bool masked = causal_rows && dl > 0;
                                 const int pi = pm == kPosUniform ? pidx_u : min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1;
                                 w_diag[k] = masked ? kMaskedHalfBias : 0.5f * s_rp[pi] + tadd;
                             }
@@ -510,7 +516,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
                     tmem_ld_wait(v);
                     uint32_t pk[16];
-                    const float* dg = w_diag + 31 - lane + 32 * cc;
+                    const float* dg = w_diag + 31 - (KIND != HSTU_KIND_CAUSAL && pm == kPosCol ? 0 : lane) + 32 * cc;
                     const int32_t* cr = w_crel + 32 * cc;
                     if (pm == kPosUniform && tm == kTimeUniform) fwd_block<kBiasConst>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else if (pm >= 0 && tm == kTimeUniform) fwd_block<kBiasRow>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
@@ -667,6 +673,8 @@ cudaError_t launch_attn_fwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
     HSTU_FWD_CASE(HSTU_KIND_MTGR, 64)
     HSTU_FWD_CASE(HSTU_KIND_MFALCON, 128)
     HSTU_FWD_CASE(HSTU_KIND_MFALCON, 64)
+    HSTU_FWD_CASE(HSTU_KIND_MFSEQ, 128)
+    HSTU_FWD_CASE(HSTU_KIND_MFSEQ, 64)
 #undef HSTU_FWD_CASE
     return cudaErrorInvalidValue;
 }
@@ -680,6 +688,8 @@ int attn_fwd_tc_ctas_per_sm(int kind, int d) {
     HSTU_OCC_CASE(HSTU_KIND_MTGR, 64)
     HSTU_OCC_CASE(HSTU_KIND_MFALCON, 128)
     HSTU_OCC_CASE(HSTU_KIND_MFALCON, 64)
+    HSTU_OCC_CASE(HSTU_KIND_MFSEQ, 128)
+    HSTU_OCC_CASE(HSTU_KIND_MFSEQ, 64)
 #undef HSTU_OCC_CASE
     return 1;
 }

@@ -46,13 +46,7 @@ __device__ __forceinline__ SeqCtx seq_ctx(const SimtParams& p, int b) {
     SeqCtx c;
     c.off0 = p.off[b];
     c.L = p.off[b + 1] - c.off0;
-    if (p.kind == HSTU_KIND_MTGR) {
-        c.S = p.n_static[b];
-        c.R = p.n_rt[b];
-    } else {
-        c.S = c.L;
-        c.R = 0;
-    }
+    segment_sizes(p.kind, p.n_static, p.n_rt, b, c.L, &c.S, &c.R);
     return c;
 }
 

@@ -13,10 +13,7 @@ __global__ void debug_indices_kernel(int kind, const int32_t* off, const int64_t
     const int s0 = off[b];
     const int L = off[b + 1] - s0;
     int S = L, R = 0;
-    if (kind == HSTU_KIND_MTGR) {
-        S = ns[b];
-        R = nr[b];
-    }
+    segment_sizes(kind, ns, nr, b, L, &S, &R);
     const long long n = (long long)L * L;
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
          e += (long long)gridDim.x * blockDim.x) {

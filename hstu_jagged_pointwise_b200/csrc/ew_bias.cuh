@@ -22,7 +22,10 @@
 
 namespace hstu {
 
-enum PosMode { kPosUniform = 0, kPosDiag = 1 };
+// kPosUniform: one position index for the block; kPosDiag: index from j - i (a
+// diagonal row of biases); kPosCol: every row of the block sits at one position
+// (M-FALCON candidates), so the index depends on the column alone.
+enum PosMode { kPosUniform = 0, kPosDiag = 1, kPosCol = 2 };
 enum TimeMode { kTimeUniform = 0, kTimeTwo = 1, kTimeBits = 2 };
 
 // Masked scores get this bias: z ~ -1e30, tanh(z/2) = -1 exactly, SiLU = 0 and SiLU' = 0.

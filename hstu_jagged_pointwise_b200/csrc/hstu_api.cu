@@ -19,7 +19,7 @@ namespace {
 struct DevInfo {
     bool ready = false;
     int sms = 0;
-    int occ[3][2] = {{0, 0}, {0, 0}, {0, 0}};   // [kind][d == 128]
+    int occ[4][2] = {{0, 0}, {0, 0}, {0, 0}, {0, 0}};   // [kind][d == 128]
 };
 std::mutex g_mu;
 DevInfo g_dev[64];
@@ -32,7 +32,7 @@ const DevInfo* dev_info() {
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return nullptr;
-        for (int k = 0; k < 3; k++) {
+        for (int k = 0; k < 4; k++) {
             d.occ[k][0] = attn_fwd_tc_ctas_per_sm(k, 64);
             d.occ[k][1] = attn_fwd_tc_ctas_per_sm(k, 128);
         }
@@ -126,6 +126,11 @@ int check_mask(const hstu_mask_spec* m, int* kind) {
     if (m->kind == HSTU_MASK_MTGR) {
         if (!aligned(m->n_static, 4) || !aligned(m->n_realtime, 4)) return HSTU_ERR_INVALID_ARG;
         *kind = HSTU_KIND_MTGR;
+        return HSTU_OK;
+    }
+    if (m->kind == HSTU_MASK_MFALCON_SEQ) {
+        if (!aligned(m->n_realtime, 4)) return HSTU_ERR_INVALID_ARG;
+        *kind = HSTU_KIND_MFSEQ;
         return HSTU_OK;
     }
     return HSTU_ERR_INVALID_ARG;
@@ -241,7 +246,9 @@ const char* hstu_status_string(int s) {
 
 size_t hstu_attn_workspace_bytes(const hstu_dims* dims, int32_t mask_kind, int32_t is_bwd) {
     if (check_dims(dims) != HSTU_OK) return 0;
-    if (mask_kind != HSTU_MASK_CAUSAL && mask_kind != HSTU_MASK_MTGR) return 0;
+    if (mask_kind != HSTU_MASK_CAUSAL && mask_kind != HSTU_MASK_MTGR && mask_kind != HSTU_MASK_MFALCON_SEQ)
+        return 0;
+    if (is_bwd && mask_kind == HSTU_MASK_MFALCON_SEQ) return 0;
     return attn_layout(*dims, is_bwd ? 1 : 0).total;
 }
 
@@ -350,6 +357,7 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     int kind = 0;
     st = check_mask(mask, &kind);
     if (st != HSTU_OK) return st;
+    if (kind == HSTU_KIND_MFSEQ) return HSTU_ERR_UNSUPPORTED;   // scoring pass: forward only
     const hstu_dims& d = *dims;
     const Layout L = attn_layout(d, 1);
     if (!aligned(workspace, 256)) return HSTU_ERR_WORKSPACE;
@@ -584,12 +592,15 @@ int hstu_debug_indices(int32_t B, int32_t mask_kind, const int32_t* seq_offsets,
                        uint8_t* mask_bits, int16_t* pos_idx, int8_t* time_bucket, void* stream) {
     if (B < 0 || n_pos < 1 || n_pos > 16384 || n_tbuckets < 1 || n_tbuckets > 64)
         return HSTU_ERR_INVALID_ARG;
-    if (mask_kind != HSTU_MASK_CAUSAL && mask_kind != HSTU_MASK_MTGR) return HSTU_ERR_INVALID_ARG;
+    if (mask_kind != HSTU_MASK_CAUSAL && mask_kind != HSTU_MASK_MTGR && mask_kind != HSTU_MASK_MFALCON_SEQ)
+        return HSTU_ERR_INVALID_ARG;
     if (B == 0) return HSTU_OK;
     if (!seq_offsets || !timestamps || !pair_offsets || !mask_bits || !pos_idx || !time_bucket)
         return HSTU_ERR_INVALID_ARG;
     if (mask_kind == HSTU_MASK_MTGR && (!n_static || !n_realtime)) return HSTU_ERR_INVALID_ARG;
-    const int kind = mask_kind == HSTU_MASK_MTGR ? HSTU_KIND_MTGR : HSTU_KIND_CAUSAL;
+    if (mask_kind == HSTU_MASK_MFALCON_SEQ && !n_realtime) return HSTU_ERR_INVALID_ARG;
+    const int kind = mask_kind == HSTU_MASK_MTGR ? HSTU_KIND_MTGR
+                   : (mask_kind == HSTU_MASK_MFALCON_SEQ ? HSTU_KIND_MFSEQ : HSTU_KIND_CAUSAL);
     return cuda_status(launch_debug_indices(B, kind, seq_offsets, timestamps, n_static, n_realtime,
                                             n_pos, n_tbuckets, pair_offsets, 0, mask_bits, pos_idx,
                                             time_bucket, static_cast<cudaStream_t>(stream)));

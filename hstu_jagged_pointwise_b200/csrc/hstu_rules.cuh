@@ -10,14 +10,33 @@
 //   MTGR dynamic mixed mask (MTGR deep-dive, section 2; MTGR arXiv report,
 //   section 3.1): static tokens bidirectional, real-time causal, candidates
 //   see themselves plus non-candidates with a strictly earlier timestamp.
+//   Full-sequence M-FALCON (HSTU blog, section 4.2): [history ; candidates] in
+//   one row, history causal, every candidate sees all history and itself (no
+//   timestamp filter); it is the MTGR layout with no static part.
 #pragma once
 #include <stdint.h>
 
 #define HSTU_KIND_CAUSAL 0
 #define HSTU_KIND_MTGR 1
 #define HSTU_KIND_MFALCON 2
+#define HSTU_KIND_MFSEQ 3
 
 namespace hstu {
+
+// Segment sizes of row b: S static tokens, R real-time / history tokens, the rest candidates.
+__device__ __forceinline__ void segment_sizes(int kind, const int32_t* n_static, const int32_t* n_rt, int b,
+                                              int L, int* S, int* R) {
+    if (kind == HSTU_KIND_MTGR) {
+        *S = n_static[b];
+        *R = n_rt[b];
+    } else if (kind == HSTU_KIND_MFSEQ) {
+        *S = 0;
+        *R = n_rt[b];
+    } else {
+        *S = L;
+        *R = 0;
+    }
+}
 
 // 0 static, 1 real-time, 2 candidate (MTGR rows); causal rows are all "static-causal".
 __device__ __forceinline__ int token_class(int i, int S, int R) {
@@ -26,7 +45,7 @@ __device__ __forceinline__ int token_class(int i, int S, int R) {
 
 // Position used by rab_pos.  MTGR candidates share the slot right after the history.
 __device__ __forceinline__ int token_pos(int kind, int i, int S, int R) {
-    return (kind == HSTU_KIND_MTGR && i >= S + R) ? S + R : i;
+    return ((kind == HSTU_KIND_MTGR || kind == HSTU_KIND_MFSEQ) && i >= S + R) ? S + R : i;
 }
 
 __device__ __forceinline__ int pos_index(int pos_i, int pos_j, int P) {
@@ -51,22 +70,22 @@ __device__ __forceinline__ int time_bucket(int64_t ti, int64_t tj, int nb) {
     return time_bucket_of_delta(abs_diff_u64(ti, tj), nb);
 }
 
-// Mask for causal and MTGR rows (i, j local to the sequence).
+// Mask of causal, MTGR and full-sequence M-FALCON rows (i, j local to the sequence).
 __device__ __forceinline__ bool visible(int kind, int i, int j, int S, int R, int64_t ts_i,
                                         int64_t ts_j) {
     if (kind == HSTU_KIND_CAUSAL) return j <= i;
     int ci = token_class(i, S, R), cj = token_class(j, S, R);
     if (ci == 0) return cj == 0;
     if (ci == 1) return cj == 0 || (cj == 1 && j <= i);
-    return j == i || (cj != 2 && ts_j < ts_i);
+    return j == i || (cj != 2 && (kind == HSTU_KIND_MFSEQ || ts_j < ts_i));
 }
 
 // Tile-level classification of a (query tile, key tile) pair from segment
 // sizes alone.  Rows [qa, qb] and columns [ka, kb] are clipped to [0, L).
 // Returns 0 when no pair can be visible, 1 when some may be (evaluate the
 // mask per element), 2 when every pair with j < L is visible.
-// Candidate rows against history are "partial": their timestamp filter is
-// applied per element.
+// MTGR candidate rows against history are "partial": their timestamp filter is
+// applied per element; full-sequence M-FALCON candidates see all history.
 __device__ __forceinline__ int tile_class(int kind, int qa, int qb, int ka, int kb, int S, int R) {
     if (kind == HSTU_KIND_CAUSAL) {
         if (ka > qb) return 0;
@@ -94,6 +113,7 @@ __device__ __forceinline__ int tile_class(int kind, int qa, int qb, int ka, int 
     // every column at or before the first row (static or earlier real-time)
     if (qb < S && kb < S) return 2;
     if (qa >= S && qb < H && kb <= qa) return 2;
+    if (kind == HSTU_KIND_MFSEQ && qa >= H && kb < H) return 2;   // candidates x history: no filter
     return 1;
 }
 

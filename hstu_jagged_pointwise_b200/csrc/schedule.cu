@@ -92,8 +92,9 @@ __global__ void __launch_bounds__(kThreads) schedule_kernel(SchedParams p) {
             const int Lk = p.kv_off[b + 1] - p.kv_off[b];
             if (Lk < 0 || Lk > p.max_kv_len) bad = 1;
         }
-        if (p.kind == HSTU_KIND_MTGR) {
-            const int S = p.n_static[b], R = p.n_rt[b];
+        if (p.kind == HSTU_KIND_MTGR || p.kind == HSTU_KIND_MFSEQ) {
+            int S = 0, R = 0;
+            segment_sizes(p.kind, p.n_static, p.n_rt, b, Lq, &S, &R);
             if (S < 0 || R < 0 || (long long)S + R > Lq) bad = 1;
         }
     }

@@ -54,6 +54,11 @@ def make_mask(kind: str = "causal", n_static: Optional[torch.Tensor] = None,
         _need(n_realtime, "n_realtime", torch.int32)
         return capi.HstuMaskSpec(kind=capi.HSTU_MASK_MTGR, n_static=n_static.data_ptr(),
                                  n_realtime=n_realtime.data_ptr())
+    if kind == "mfalcon_seq":
+        # n_realtime[b] is the history length of row b; the rest of the row are candidates
+        _need(n_realtime, "n_realtime", torch.int32)
+        return capi.HstuMaskSpec(kind=capi.HSTU_MASK_MFALCON_SEQ, n_static=None,
+                                 n_realtime=n_realtime.data_ptr())
     raise ValueError(f"unknown mask kind {kind!r}")
 
 
@@ -90,8 +95,9 @@ class Layer:
         self.dims = make_dims(self.T, self.B, H, d, dtype, alpha, max_seq_len, n_pos, n_tbuckets, ln_eps)
         self.mask = make_mask(mask_kind, n_static, n_realtime)
         self.device = seq_offsets.device
-        n = max(attn_workspace_bytes(self.dims, self.mask.kind, False),
-                attn_workspace_bytes(self.dims, self.mask.kind, True))
+        n = attn_workspace_bytes(self.dims, self.mask.kind, False)
+        if self.mask.kind != capi.HSTU_MASK_MFALCON_SEQ:   # the full-sequence M-FALCON mask is forward only
+            n = max(n, attn_workspace_bytes(self.dims, self.mask.kind, True))
         self.ws = workspace(n, self.device)
 
     @property
@@ -188,7 +194,8 @@ def debug_indices(seq_offsets, timestamps, mask_kind: str = "causal", n_static=N
     m = torch.zeros(n, dtype=torch.uint8, device=seq_offsets.device)
     pi = torch.zeros(n, dtype=torch.int16, device=seq_offsets.device)
     tb = torch.zeros(n, dtype=torch.int8, device=seq_offsets.device)
-    kind = capi.HSTU_MASK_MTGR if mask_kind == "mtgr" else capi.HSTU_MASK_CAUSAL
+    kind = {"causal": capi.HSTU_MASK_CAUSAL, "mtgr": capi.HSTU_MASK_MTGR,
+            "mfalcon_seq": capi.HSTU_MASK_MFALCON_SEQ}[mask_kind]
     st = capi.LIB.hstu_debug_indices(L.numel(), kind, _p(seq_offsets), _p(timestamps), _p(n_static),
                                      _p(n_realtime), n_pos, n_tbuckets, _p(po), _p(m), _p(pi), _p(tb), _stream())
     capi.check(st, "hstu_debug_indices")

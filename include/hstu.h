@@ -10,7 +10,8 @@
  *
  *   pidx(i, j) = clamp(pos(j) - pos(i), -(P-1), P-1) + (P-1)    (rab_pos has 2P-1 entries)
  *   tb(i, j)   = min(nb - 1, bit_length(|ts(i) - ts(j)|))       (rab_time has nb entries)
- *   pos(i)     = i, except MTGR candidates, which all sit at pos = S + R
+ *   pos(i)     = i, except candidates (MTGR, full-sequence M-FALCON), which all
+ *                sit at pos = S + R
  *
  * Masks: HSTU_MASK_CAUSAL (j <= i; MTGR deep-dive section 2, "classic GR causal
  * mask") and HSTU_MASK_MTGR, the dynamic mixed mask (MTGR deep-dive section 2;
@@ -20,6 +21,11 @@
  * non-candidate whose timestamp is strictly smaller than its own.
  * hstu_mfalcon_score is the M-FALCON candidate mask over cached history K/V
  * (HSTU blog, sections 4.2-4.3): candidates see all history and themselves.
+ * HSTU_MASK_MFALCON_SEQ is the same candidate mask with history and
+ * candidates in one row [R history | K candidates] (HSTU blog, section 4.2:
+ * one pass scores the candidates against a causal history): history tokens are
+ * causal, a candidate sees every history token and itself, and all candidates
+ * sit at pos = R.  It is forward only (a scoring pass).
  *
  * Conventions shared by every entry point:
  *  - Tensor pointers are DEVICE pointers owned by the caller.  Host structs
@@ -73,12 +79,15 @@ typedef enum {
 
 typedef enum { HSTU_BF16 = 0, HSTU_F32 = 1 } hstu_dtype;
 
-typedef enum { HSTU_MASK_CAUSAL = 0, HSTU_MASK_MTGR = 1 } hstu_mask_kind;
+typedef enum { HSTU_MASK_CAUSAL = 0, HSTU_MASK_MTGR = 1, HSTU_MASK_MFALCON_SEQ = 2 } hstu_mask_kind;
 
 /* Mask description.  For HSTU_MASK_MTGR, n_static[b] (profile + long-term
  * tokens, seen bidirectionally) and n_realtime[b] are DEVICE int32 [B]; the
  * remaining L_b - n_static[b] - n_realtime[b] tokens of row b are candidates.
- * Both pointers are ignored for HSTU_MASK_CAUSAL. */
+ * For HSTU_MASK_MFALCON_SEQ, n_realtime[b] is the history length of row b (the
+ * rest are candidates) and n_static is ignored (may be NULL).  Both pointers
+ * are ignored for HSTU_MASK_CAUSAL.  Segment sizes outside [0, L_b] set the
+ * device status word (HSTU_ERR_DEVICE_BOUNDS) and the launch writes nothing. */
 typedef struct {
     int32_t kind;                /* hstu_mask_kind */
     const int32_t* n_static;     /* device [B] */
@@ -100,7 +109,8 @@ typedef struct {
 } hstu_dims;
 
 /* Bytes of workspace hstu_attn_fwd (is_bwd = 0) or hstu_attn_bwd (is_bwd = 1)
- * needs for these dims and mask kind; 0 when the arguments are invalid. */
+ * needs for these dims and mask kind; 0 when the arguments are invalid, and 0
+ * for is_bwd = 1 with HSTU_MASK_MFALCON_SEQ (no backward for that mask). */
 HSTU_API size_t hstu_attn_workspace_bytes(const hstu_dims* dims, int32_t mask_kind, int32_t is_bwd);
 
 /* Forward of one HSTU attention layer (formula above).
@@ -158,7 +168,8 @@ HSTU_API int hstu_attn_fwd_noalloc(const hstu_dims* dims, const hstu_mask_spec* 
  * Out: dq, dk [T, H*d_qk]; dv, du [T, H*d_v] (element type dims.dtype);
  *      d_rab_pos fp32 [2P-1], d_rab_time fp32 [nb], d_gamma, d_beta fp32 [H*d_v].
  * Every output is overwritten, not accumulated.  y, ln_mean and ln_rstd are the
- * forward's outputs for the same inputs. */
+ * forward's outputs for the same inputs.  HSTU_MASK_MFALCON_SEQ returns
+ * HSTU_ERR_UNSUPPORTED (a scoring pass: forward only). */
 HSTU_API int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask,
                   const void* q, const void* k, const void* v, const void* u,
                   const int32_t* seq_offsets, const int64_t* timestamps,

@@ -93,6 +93,24 @@ def test_fwd_rejects_bad_arguments_before_launch():
     assert capi.LIB.hstu_attn_fwd(C.byref(d0), C.byref(m), *args, 2048, None) == capi.HSTU_OK
 
 
+def test_full_sequence_mfalcon_mask_is_forward_only():
+    """The [history ; candidates] mask has a forward workspace, no backward, and needs n_realtime."""
+    d = dims()
+    assert capi.LIB.hstu_attn_workspace_bytes(C.byref(d), capi.HSTU_MASK_MFALCON_SEQ, 0) > 0
+    assert capi.LIB.hstu_attn_workspace_bytes(C.byref(d), capi.HSTU_MASK_MFALCON_SEQ, 1) == 0
+    buf = (C.c_int32 * 8)()
+    m = capi.HstuMaskSpec(kind=capi.HSTU_MASK_MFALCON_SEQ, n_static=None, n_realtime=C.addressof(buf))
+    nulls = [None] * 23
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), C.byref(m), *nulls, 0, None) == capi.HSTU_ERR_UNSUPPORTED
+    # without the history lengths the forward is refused before any launch
+    m0 = capi.HstuMaskSpec(kind=capi.HSTU_MASK_MFALCON_SEQ, n_static=None, n_realtime=None)
+    assert capi.LIB.hstu_attn_fwd(C.byref(d), C.byref(m0), *([None] * 15), 0, None) == \
+        capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_debug_indices(1, capi.HSTU_MASK_MFALCON_SEQ, C.addressof(buf), C.addressof(buf), None,
+                                       None, 256, 64, C.addressof(buf), C.addressof(buf), C.addressof(buf),
+                                       C.addressof(buf), None) == capi.HSTU_ERR_INVALID_ARG
+
+
 def test_mfalcon_rejects_bad_arguments():
     d = capi.HstuMfalconDims(B=2, T_hist=10, T_cand=4, H=2, d_qk=128, d_v=128, dtype=capi.HSTU_BF16,
                              n_pos=256, n_tbuckets=64, max_hist_len=8, max_cand_len=4, alpha=9.0,

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from hstu_jagged_pointwise_b200 import workloads as W
-from parity import (assert_bf16, assert_f32, run_layer, run_mfalcon, storage_bwd, storage_fwd,
+from parity import (assert_bf16, assert_f32, errors, run_layer, run_mfalcon, storage_bwd, storage_fwd,
                     storage_mfalcon)
 
 pytestmark = pytest.mark.gpu
@@ -38,12 +38,17 @@ def test_debug_indices_bit_exact():
     u2 = W.mtgr_user(rng, 2, 280, 0, 30)
     u3 = W.mtgr_user(rng, 5, 20, 0, 0)
     cases.append(("mtgr", [hand, u1, u2, u3], [3, 43, 282, 25], [2, 8, 0, 0]))
+    # full-sequence M-FALCON: candidates before, at and after the history's last timestamp,
+    # a history longer than the position clamp, no history, no candidates
+    h1 = W.increasing_ts(rng, 300)
+    c1 = np.concatenate([h1[-1] + np.array([0, 5, 1]), h1[:2]])
+    cases.append(("mfalcon_seq", [np.concatenate([h1, c1]), ts_a[:6], ts_b[:40]], None, [300, 0, 40]))
     for kind, ts_list, ns, nr in cases:
         lens = [len(t) for t in ts_list]
         off = np.zeros(len(lens) + 1, np.int32)
         off[1:] = np.cumsum(lens)
         ts = np.concatenate(ts_list)
-        k = oracle.MASK_MTGR if kind == "mtgr" else oracle.MASK_CAUSAL
+        k = {"causal": oracle.MASK_CAUSAL, "mtgr": oracle.MASK_MTGR, "mfalcon_seq": oracle.MASK_MFSEQ}[kind]
         m0, p0, t0, _ = oracle.indices(off, ts, k, ns, nr)
         dn = lambda a, dt: torch.as_tensor(np.asarray(a, dt)).cuda()
         m1, p1, t1, _ = ops.debug_indices(dn(off, np.int32), dn(ts, np.int64), kind,
@@ -166,6 +171,57 @@ def test_mfalcon_permutation_equivariance():
     w.cand_ts = w.cand_ts[perm]
     out2, _ = run_mfalcon(w)
     assert torch.equal(out2["y"], out["y"][pt.cuda()])
+
+
+# ----------------------------------------------------------------------------
+# full-sequence M-FALCON: [history ; candidates] in one jagged row
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_mfalcon_seq_forward_small(d):
+    # empty row, no history, one history token, splits off the 128-row tile grid, no candidates
+    w = W.make_mfalcon([0, 0, 1, 200, 300, 129, 64], [0, 3, 5, 130, 300, 1, 0], H=2, d=d, seed=13,
+                       alpha=301.0)
+    ws = W.mfalcon_seq_from(w, seed=14)
+    out, _, _ = run_layer(ws)
+    y, o, _, _ = oracle.layer_fwd(ws)
+    st = storage_fwd(ws)
+    assert_bf16(out["y"], y, "y", st["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", st["o_pre"])
+    if d == 128:
+        # the candidate rows score like the cached-history kernel on the same users
+        cand = np.concatenate([np.arange(ws.offsets[b] + ws.n_realtime[b], ws.offsets[b + 1])
+                               for b in range(ws.B)]).astype(np.int64)
+        oc, _ = run_mfalcon(w)
+        rel, _, _ = errors(out["y"][torch.as_tensor(cand).cuda()], oc["y"])
+        assert rel < 5e-3, f"cached-history and one-row candidate scores differ: rel {rel:.2e}"
+
+
+def _seq_slice(w, b):
+    """Row b of a full-sequence M-FALCON workload alone (rows are independent)."""
+    import dataclasses
+    s0, s1 = int(w.offsets[b]), int(w.offsets[b + 1])
+    sub = dataclasses.replace(w, offsets=np.array([0, s1 - s0], np.int32), ts=w.ts[s0:s1],
+                              n_realtime=np.asarray(w.n_realtime[b:b + 1], np.int32),
+                              q=w.q[s0:s1], k=w.k[s0:s1], v=w.v[s0:s1], u=w.u[s0:s1])
+    return sub, s0
+
+
+def test_mfalcon_ranking_full_sequence_sampled_rows():
+    """256 users x [2048 history ; 1024 candidates] in one launch; sampled rows of four users."""
+    ws = W.mfalcon_seq_from(W.mfalcon_ranking(seed=0), seed=1)
+    out, _, _ = run_layer(ws)
+    rng = np.random.default_rng(5)
+    for b in (0, 97, 200, 255):
+        sub, s0 = _seq_slice(ws, b)
+        nh = int(sub.n_realtime[0])
+        rows = np.unique(np.concatenate([rng.integers(0, nh, 6), [0, nh - 1, nh, sub.T - 1],
+                                         rng.integers(nh, sub.T, 6)])).astype(np.int64)
+        y, o, _, _ = oracle.layer_fwd(sub, rows)
+        st = storage_fwd(sub, rows)
+        rt = torch.as_tensor(rows + s0).cuda()
+        assert_bf16(out["y"][rt], y, f"y[user {b}]", st["y"])
+        assert_bf16(out["o_pre"][rt], o, f"o_pre[user {b}]", st["o_pre"])
 
 
 # ----------------------------------------------------------------------------
