@@ -522,7 +522,7 @@ def run_mfalcon_seq(args, world, w, dev):
     """The same users as one jagged row each, [history ; candidates], through the
     attention forward with the full-sequence M-FALCON mask: history rows causal,
     candidates against all history and themselves."""
-    from hstu_jagged_pointwise_b200 import ops
+    from hstu_jagged_pointwise_b200 import capi, ops
     ws = W.mfalcon_seq_from(w, seed=args.seed + 1)
     t = {n: getattr(ws, n).to(dev) for n in ("q", "k", "v", "u", "rab_pos", "rab_time", "gamma", "beta")}
     off = torch.as_tensor(ws.offsets).to(dev)
@@ -554,9 +554,35 @@ def run_mfalcon_seq(args, world, w, dev):
     pairs = int(w.H * np.sum(nh * (nh + 1) // 2 + nc * (nh + 1)))
     pk, _ = peaks()
     tfl = 4 * w.d * pairs / (ms * 1e-3) / 1e12
+    del out, layer
+
+    # the KV-cache producer on the same batch: history rows of k, v, ts packed for the scorer
+    hist_rows = int(nh.sum())
+    cache = ops.mfalcon_cache_history(off, ts, nr, t["k"], t["v"], hist_rows=hist_rows)
+    for _ in range(args.warmup):
+        ops.mfalcon_cache_history(off, ts, nr, t["k"], t["v"], out=cache)
+    torch.cuda.synchronize()
+    barrier(world)
+    capi.profile_enable(True)
+    e0.record(s)
+    for _ in range(args.steps):
+        ops.mfalcon_cache_history(off, ts, nr, t["k"], t["v"], out=cache)
+    e1.record(s)
+    torch.cuda.synchronize()
+    prof = capi.profile_read()
+    capi.profile_enable(False)
+    ms_c = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    if int(cache["status"].item()) != 0:
+        raise RuntimeError("device status set in the KV-cache producer")
+    nb = hist_rows * (4 * ws.D * 2 + 16)     # read and write k, v rows (bf16) and the int64 timestamp
+    n_copy, t_copy = prof.get("cache_copy_kernel", (1, ms_c))
+    gbs = nb / (t_copy / n_copy * 1e-3) / 1e9
     return {"workload": f"{w.name}_one_row", "tokens": int(ws.T), "cands_per_s": round(world * w.T / (ms * 1e-3), 1),
             "ms_per_pass": round(ms, 4), "tflops": round(world * tfl, 3),
-            "pct_bf16_peak": round(tfl / pk["bf16_tflops_sustained"], 4)}
+            "pct_bf16_peak": round(tfl / pk["bf16_tflops_sustained"], 4),
+            "kv_cache_producer": {"rows": hist_rows, "ms_per_call": round(ms_c, 4),
+                                  "copy_kernel_ms": round(t_copy / n_copy, 4), "bytes_per_call": nb,
+                                  "copy_kernel_gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}}
 
 
 # ----------------------------------------------------------------------------

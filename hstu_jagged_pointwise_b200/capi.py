@@ -30,7 +30,7 @@ EXPORTS = (
     "hstu_attn_workspace_bytes", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_mfalcon_workspace_bytes",
     "hstu_mfalcon_score", "hstu_debug_indices", "hstu_check_device_error", "hstu_status_string",
     "hstu_version", "hstu_profile_enable", "hstu_profile_read", "hstu_profile_kind_name",
-    "hstu_attn_fwd_noalloc",
+    "hstu_attn_fwd_noalloc", "hstu_mfalcon_cache_history",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20   # HSTU_NOALLOC_SCRATCH_BYTES
@@ -81,6 +81,8 @@ def load():
     lib.hstu_mfalcon_workspace_bytes.restype = S
     lib.hstu_mfalcon_score.argtypes = [C.POINTER(HstuMfalconDims)] + [P] * 14 + [i32] + [P] * 3 + [S, P]
     lib.hstu_mfalcon_score.restype = C.c_int
+    lib.hstu_mfalcon_cache_history.argtypes = [i32, i32, i32, i32, P, P, P, P, P, C.c_int64, P, P, P, P, P, P]
+    lib.hstu_mfalcon_cache_history.restype = C.c_int
     lib.hstu_debug_indices.argtypes = [i32, i32, P, P, P, P, i32, i32, P, P, P, P, P]
     lib.hstu_debug_indices.restype = C.c_int
     lib.hstu_check_device_error.argtypes = [P, P]

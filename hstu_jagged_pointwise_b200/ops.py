@@ -182,6 +182,36 @@ class MFalcon:
         return int(capi.LIB.hstu_check_device_error(_p(self.ws), _stream()))
 
 
+def mfalcon_cache_history(seq_offsets, timestamps, n_history, k, v, hist_rows: Optional[int] = None,
+                          out: Optional[dict] = None) -> dict:
+    """KV cache for MFalcon.score from a full-sequence M-FALCON batch: the first
+    n_history[b] rows of every user's [history ; candidates] row of k, v and
+    timestamps, packed, with their offsets.  hist_rows (rows to allocate) defaults
+    to sum(n_history), read on the host.  out["status"] (device int32) is nonzero
+    when the batch was invalid or did not fit; nothing else is written then."""
+    _need(seq_offsets, "seq_offsets", torch.int32)
+    _need(timestamps, "timestamps", torch.int64)
+    _need(n_history, "n_history", torch.int32)
+    if k.dtype != v.dtype or k.shape != v.shape or k.dim() != 2 or not k.is_contiguous() or not v.is_contiguous():
+        raise ValueError("k and v must be contiguous [T, H*d] tensors of one dtype")
+    B = seq_offsets.numel() - 1
+    if hist_rows is None:
+        hist_rows = int(n_history.sum().item()) if B > 0 else 0
+    dev = k.device
+    if out is None:
+        out = dict(hist_offsets=torch.empty(B + 1, dtype=torch.int32, device=dev),
+                   hist_ts=torch.empty(hist_rows, dtype=torch.int64, device=dev),
+                   hist_k=torch.empty(hist_rows, k.shape[1], dtype=k.dtype, device=dev),
+                   hist_v=torch.empty(hist_rows, k.shape[1], dtype=k.dtype, device=dev),
+                   status=torch.zeros(1, dtype=torch.int32, device=dev))
+    st = capi.LIB.hstu_mfalcon_cache_history(
+        B, k.shape[0], k.shape[1], _DTYPES[k.dtype], _p(seq_offsets), _p(timestamps), _p(n_history), _p(k),
+        _p(v), out["hist_k"].shape[0], _p(out["hist_offsets"]), _p(out["hist_ts"]), _p(out["hist_k"]),
+        _p(out["hist_v"]), _p(out["status"]), _stream())
+    capi.check(st, "hstu_mfalcon_cache_history")
+    return out
+
+
 def debug_indices(seq_offsets, timestamps, mask_kind: str = "causal", n_static=None, n_realtime=None,
                   n_pos: int = 256, n_tbuckets: int = 64):
     """Per-pair (mask, rab_pos index, time bucket) from the kernels' own device functions."""

@@ -216,6 +216,34 @@ HSTU_API int hstu_mfalcon_score(const hstu_mfalcon_dims* dims,
                        const float* ln_gamma, const float* ln_beta, int32_t b_m,
                        void* y, void* o_pre, void* workspace, size_t workspace_bytes, void* stream);
 
+/* KV-cache producer for hstu_mfalcon_score (HSTU blog, section 4.3 "KV caching":
+ * a user's history keys and values are computed once and reused by every later
+ * candidate microbatch).  Input is a full-sequence M-FALCON batch, one row
+ * [R_b history ; candidates] per user (section 4.2); output is the compact
+ * history layout hstu_mfalcon_score reads.
+ * In:  B users; T rows; row_elems elements per row of k and v (H*d), element
+ *      type dtype (HSTU_BF16 or HSTU_F32; row_elems * elem_size a multiple of
+ *      16); seq_offsets int32 [B+1], timestamps int64 [T], n_history int32 [B]
+ *      (R_b, the mask's n_realtime), k, v [T, row_elems]; hist_capacity = rows
+ *      allocated in hist_ts / hist_k / hist_v.
+ * Out: hist_offsets int32 [B+1] = exclusive prefix sums of R_b; for i < R_b,
+ *      row hist_offsets[b] + i of hist_ts / hist_k / hist_v is row
+ *      seq_offsets[b] + i of timestamps / k / v (exact copies).  Rows past
+ *      hist_offsets[B] are not written.
+ * device_status: DEVICE int32, required.  Set on `stream` to 0 on success, or
+ *      to 1 when seq_offsets is not a valid jagged layout of T rows, some R_b
+ *      lies outside [0, L_b], or sum(R_b) exceeds hist_capacity; then nothing
+ *      else is written.
+ * Returns HSTU_ERR_INVALID_ARG for negative sizes, a bad dtype, or a missing or
+ * misaligned pointer (16 bytes for k, v, hist_k, hist_v; 8 for the timestamps;
+ * 4 for the int32 arrays), HSTU_ERR_UNSUPPORTED for rows that are not whole
+ * 16-byte vectors, each time before any launch. */
+HSTU_API int hstu_mfalcon_cache_history(int32_t B, int32_t T, int32_t row_elems, int32_t dtype,
+                       const int32_t* seq_offsets, const int64_t* timestamps, const int32_t* n_history,
+                       const void* k, const void* v, int64_t hist_capacity,
+                       int32_t* hist_offsets, int64_t* hist_ts, void* hist_k, void* hist_v,
+                       int32_t* device_status, void* stream);
+
 /* Integer decisions of the fused kernels, written through the same device
  * functions they use, for exact comparison in tests.  For every sequence b and
  * pair (i, j) of it, entry pair_offsets[b] + i*L_b + j (pair_offsets: device

@@ -18,7 +18,7 @@ def header_functions():
 
 def test_exports_match_header():
     names = header_functions()
-    assert len(names) == 13, names
+    assert len(names) == 14, names
     assert set(names) == set(capi.EXPORTS)
     for n in names:
         assert hasattr(capi.LIB, n), n
@@ -109,6 +109,20 @@ def test_full_sequence_mfalcon_mask_is_forward_only():
     assert capi.LIB.hstu_debug_indices(1, capi.HSTU_MASK_MFALCON_SEQ, C.addressof(buf), C.addressof(buf), None,
                                        None, 256, 64, C.addressof(buf), C.addressof(buf), C.addressof(buf),
                                        C.addressof(buf), None) == capi.HSTU_ERR_INVALID_ARG
+
+
+def test_cache_producer_rejects_bad_arguments_before_launch():
+    f = capi.LIB.hstu_mfalcon_cache_history
+    buf = (C.c_int64 * 64)()
+    a = C.addressof(buf)
+    ok = [a] * 5   # seq_offsets, timestamps, n_history, k, v
+    outs = [a] * 5  # hist_offsets, hist_ts, hist_k, hist_v, device_status
+    assert f(-1, 0, 64, capi.HSTU_BF16, *ok, 0, *outs, None) == capi.HSTU_ERR_INVALID_ARG
+    assert f(1, 4, 64, 7, *ok, 4, *outs, None) == capi.HSTU_ERR_INVALID_ARG            # dtype
+    assert f(1, 4, 4, capi.HSTU_BF16, *ok, 4, *outs, None) == capi.HSTU_ERR_UNSUPPORTED  # 8-byte rows
+    assert f(1, 4, 64, capi.HSTU_BF16, *ok, 4, a, a, a, a, None, None) == capi.HSTU_ERR_INVALID_ARG  # no status
+    assert f(1, 4, 64, capi.HSTU_BF16, a, a, a, a + 8, a, 4, *outs, None) == capi.HSTU_ERR_INVALID_ARG  # k misaligned
+    assert f(1, 4, 64, capi.HSTU_BF16, a, a, a, a, a, -1, *outs, None) == capi.HSTU_ERR_INVALID_ARG
 
 
 def test_mfalcon_rejects_bad_arguments():

@@ -197,6 +197,66 @@ def test_mfalcon_seq_forward_small(d):
         assert rel < 5e-3, f"cached-history and one-row candidate scores differ: rel {rel:.2e}"
 
 
+def test_mfalcon_seq_forward_fp32():
+    w = W.make_mfalcon([0, 5, 70, 40], [2, 0, 9, 33], H=2, d=32, dtype=torch.float32, seed=19, alpha=71.0)
+    ws = W.mfalcon_seq_from(w, seed=20)
+    out, _, _ = run_layer(ws)
+    y, o, _, _ = oracle.layer_fwd(ws)
+    assert_f32(out["y"], y, "y")
+    assert_f32(out["o_pre"], o, "o_pre")
+
+
+def _cache_from_one_row(ws, dtype=None):
+    from hstu_jagged_pointwise_b200 import ops
+    cast = (lambda t: t.cuda()) if dtype is None else (lambda t: t.to(dtype).cuda())
+    off = torch.as_tensor(ws.offsets).cuda()
+    ts = torch.as_tensor(ws.ts).cuda()
+    nh = torch.as_tensor(np.asarray(ws.n_realtime, np.int32)).cuda()
+    out = ops.mfalcon_cache_history(off, ts, nh, cast(ws.k), cast(ws.v))
+    torch.cuda.synchronize()
+    return out
+
+
+def test_mfalcon_cache_producer_exact_and_scores_identically():
+    """The history rows of the one-row layout, packed, are the cache the scorer reads: bit-exact."""
+    w = W.make_mfalcon([0, 0, 1, 200, 300, 129, 64, 3], [0, 3, 5, 130, 300, 1, 0, 2], H=2, d=128, seed=15,
+                       alpha=301.0)
+    ws = W.mfalcon_seq_from(w, seed=16)
+    c = _cache_from_one_row(ws)
+    assert int(c["status"].item()) == 0
+    np.testing.assert_array_equal(c["hist_offsets"].cpu().numpy(), np.asarray(w.hist_offsets, np.int32))
+    np.testing.assert_array_equal(c["hist_ts"].cpu().numpy(), np.asarray(w.hist_ts, np.int64))
+    assert torch.equal(c["hist_k"].cpu(), w.hist_k) and torch.equal(c["hist_v"].cpu(), w.hist_v)
+    # fp32 rows take the same path
+    c32 = _cache_from_one_row(ws, torch.float32)
+    assert torch.equal(c32["hist_k"].cpu(), w.hist_k.float()) and torch.equal(c32["hist_v"].cpu(), w.hist_v.float())
+    # scoring from the produced cache is the scoring from the original one
+    ref, d = run_mfalcon(w)
+    d2 = dict(d, hist_k=c["hist_k"], hist_v=c["hist_v"], hist_offsets=c["hist_offsets"], hist_ts=c["hist_ts"])
+    got, _ = run_mfalcon(w, d=d2)
+    assert torch.equal(got["y"], ref["y"]) and torch.equal(got["o_pre"], ref["o_pre"])
+
+
+def test_mfalcon_cache_producer_rejects_bad_batches():
+    from hstu_jagged_pointwise_b200 import ops
+    w = W.make_mfalcon([10, 20], [4, 5], H=2, d=64, seed=17, alpha=21.0)
+    ws = W.mfalcon_seq_from(w, seed=18)
+    off = torch.as_tensor(ws.offsets).cuda()
+    ts = torch.as_tensor(ws.ts).cuda()
+    k, v = ws.k.cuda(), ws.v.cuda()
+    for nh, rows in (([10, 26], 36), ([-1, 20], 30), ([10, 20], 29)):   # R > L, R < 0, no room
+        out = dict(hist_offsets=torch.full((3,), -7, dtype=torch.int32, device="cuda"),
+                   hist_ts=torch.full((rows,), -7, dtype=torch.int64, device="cuda"),
+                   hist_k=torch.full((rows, k.shape[1]), -7.0, dtype=k.dtype, device="cuda"),
+                   hist_v=torch.full((rows, k.shape[1]), -7.0, dtype=k.dtype, device="cuda"),
+                   status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+        ops.mfalcon_cache_history(off, ts, torch.tensor(nh, dtype=torch.int32, device="cuda"), k, v, out=out)
+        torch.cuda.synchronize()
+        assert int(out["status"].item()) == 1, nh
+        assert bool((out["hist_offsets"] == -7).all()) and bool((out["hist_ts"] == -7).all())
+        assert bool((out["hist_k"] == -7).all()) and bool((out["hist_v"] == -7).all())
+
+
 def _seq_slice(w, b):
     """Row b of a full-sequence M-FALCON workload alone (rows are independent)."""
     import dataclasses
@@ -209,8 +269,15 @@ def _seq_slice(w, b):
 
 def test_mfalcon_ranking_full_sequence_sampled_rows():
     """256 users x [2048 history ; 1024 candidates] in one launch; sampled rows of four users."""
-    ws = W.mfalcon_seq_from(W.mfalcon_ranking(seed=0), seed=1)
+    w = W.mfalcon_ranking(seed=0)
+    ws = W.mfalcon_seq_from(w, seed=1)
     out, _, _ = run_layer(ws)
+    # the KV cache produced from this batch is the ranking workload's cache, exactly
+    c = _cache_from_one_row(ws)
+    assert int(c["status"].item()) == 0
+    assert torch.equal(c["hist_k"].cpu(), w.hist_k) and torch.equal(c["hist_v"].cpu(), w.hist_v)
+    np.testing.assert_array_equal(c["hist_ts"].cpu().numpy(), np.asarray(w.hist_ts, np.int64))
+    del c
     rng = np.random.default_rng(5)
     for b in (0, 97, 200, 255):
         sub, s0 = _seq_slice(ws, b)
