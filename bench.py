@@ -359,9 +359,15 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     ms_fwd = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
 
+    # Group LayerNorm variant of the same layer (LayerNorm kernels only differ)
+    extra = {}
+    if not args.no_gln:
+        extra["gln"] = run_gln(args, world, w, dv, off, ts, rp, rt, fwd_out, bwd_out)
+
     # ---- end to end through the C ABI with host buffers
     if args.no_e2e:
-        return finish(args, world, w, kernels, ms, ms_max, ms_fwd, None, None, None, None, clocks, f_fwd, f_bwd, P, d)
+        return finish(args, world, w, kernels, ms, ms_max, ms_fwd, None, None, None, None, clocks, f_fwd, f_bwd, P, d,
+                      extra)
     pin = {n: t.pin_memory() for n, t in host.items()}
     small_in = {n: t.pin_memory() for n, t in (("rp", w.rab_pos), ("rt", w.rab_time), ("g", w.gamma),
                                                 ("b", w.beta))}
@@ -403,10 +409,55 @@ def run_ours(args, world, rank, local):
     if not args.no_mfalcon:
         del pin, outs_h
         mf = run_mfalcon(args, world, rank, local)
-    return finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d)
+    return finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d,
+                  extra)
 
 
-def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d):
+def run_gln(args, world, w, dv, off, ts, rp, rt, fwd_out, bwd_out):
+    """The layer with Group LayerNorm (4 groups, seeded random token ids, one gamma/beta row
+    per group): forward + backward steps timed, and the LayerNorm kernels' HBM rates."""
+    from hstu_jagged_pointwise_b200 import capi, ops
+    G = 4
+    dev = dv["q"].device
+    gen = torch.Generator().manual_seed(args.seed + 77)
+    tg = torch.randint(0, G, (w.T,), generator=gen, dtype=torch.uint8).to(dev)
+    g = (1 + 0.1 * torch.randn(G, w.D, generator=gen)).to(dev)
+    b = (0.1 * torch.randn(G, w.D, generator=gen)).to(dev)
+    layer = ops.Layer(off, ts, w.H, w.d, torch.bfloat16, w.alpha, w.max_len, n_groups=G, token_group=tg)
+    bo = dict(bwd_out, d_gamma=torch.empty_like(g), d_beta=torch.empty_like(b))
+
+    def step():
+        layer.forward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, out=fwd_out)
+        layer.backward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, fwd_out, dv["grad"], out=bo)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    capi.profile_enable(True)
+    e0.record(s)
+    for _ in range(args.steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    prof = capi.profile_read()
+    capi.profile_enable(False)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    if layer.check_device_error() != 0:
+        raise RuntimeError("device status set in the Group LayerNorm step")
+    pk, _ = peaks()
+    out = {"groups": G, "token_groups": "uniform random", "ms_per_step": round(ms, 4)}
+    for name, nbytes in (("ln_fwd_kernel", (6 * w.D + 9) * w.T), ("ln_bwd_kernel", (10 * w.D + 9) * w.T)):
+        n, t = prof[name]
+        gbs = nbytes / (t / n * 1e-3) / 1e9
+        out[name] = {"ms_per_launch": round(t / n, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    return out
+
+
+def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d,
+           extra=None):
     H = w.H
     # ---- roofline of the dominant kernel
     pk, pk_src = peaks()
@@ -471,6 +522,7 @@ def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, cl
     }
     if mf is not None:
         line["mfalcon"] = mf
+    line.update(extra or {})
     return line, w
 
 
@@ -624,6 +676,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-mfalcon", action="store_true")
+    ap.add_argument("--no-gln", action="store_true", help="skip the Group LayerNorm variant")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--tokens", type=int, default=262144,

@@ -30,7 +30,8 @@ EXPORTS = (
     "hstu_attn_workspace_bytes", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_mfalcon_workspace_bytes",
     "hstu_mfalcon_score", "hstu_debug_indices", "hstu_check_device_error", "hstu_status_string",
     "hstu_version", "hstu_profile_enable", "hstu_profile_read", "hstu_profile_kind_name",
-    "hstu_attn_fwd_noalloc", "hstu_mfalcon_cache_history",
+    "hstu_attn_fwd_noalloc", "hstu_mfalcon_cache_history", "hstu_attn_fwd_gln", "hstu_attn_bwd_gln",
+    "hstu_attn_workspace_bytes_gln",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20   # HSTU_NOALLOC_SCRATCH_BYTES
@@ -45,6 +46,10 @@ class HstuDims(C.Structure):
 
 class HstuMaskSpec(C.Structure):
     _fields_ = [("kind", C.c_int32), ("n_static", C.c_void_p), ("n_realtime", C.c_void_p)]
+
+
+class HstuNormSpec(C.Structure):
+    _fields_ = [("n_groups", C.c_int32), ("token_group", C.c_void_p)]
 
 
 class HstuMfalconDims(C.Structure):
@@ -77,6 +82,13 @@ def load():
     lib.hstu_attn_fwd_noalloc.restype = C.c_int
     lib.hstu_attn_bwd.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec)] + [P] * 23 + [S, P]
     lib.hstu_attn_bwd.restype = C.c_int
+    NS = C.POINTER(HstuNormSpec)
+    lib.hstu_attn_workspace_bytes_gln.argtypes = [C.POINTER(HstuDims), i32, i32, i32]
+    lib.hstu_attn_workspace_bytes_gln.restype = S
+    lib.hstu_attn_fwd_gln.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec), NS] + [P] * 15 + [S, P]
+    lib.hstu_attn_fwd_gln.restype = C.c_int
+    lib.hstu_attn_bwd_gln.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec), NS] + [P] * 23 + [S, P]
+    lib.hstu_attn_bwd_gln.restype = C.c_int
     lib.hstu_mfalcon_workspace_bytes.argtypes = [C.POINTER(HstuMfalconDims), i32]
     lib.hstu_mfalcon_workspace_bytes.restype = S
     lib.hstu_mfalcon_score.argtypes = [C.POINTER(HstuMfalconDims)] + [P] * 14 + [i32] + [P] * 3 + [S, P]

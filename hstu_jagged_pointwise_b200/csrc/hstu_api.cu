@@ -138,12 +138,12 @@ int check_mask(const hstu_mask_spec* m, int* kind) {
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-    size_t items = 0, perm = 0, seq_base = 0, dy = 0, part = 0, dq_acc = 0, rab_part = 0, total = 0;
+    size_t items = 0, perm = 0, seq_base = 0, dy = 0, part = 0, dq_acc = 0, rab_part = 0, gmask = 0, total = 0;
     long long max_items = 0;
     int n_part = 0;
 };
 
-Layout attn_layout(const hstu_dims& d, int is_bwd) {
+Layout attn_layout(const hstu_dims& d, int is_bwd, int n_groups = 1) {
     Layout L;
     size_t off = sizeof(Control);
     L.max_items = (long long)d.H * (((long long)d.T + kTileM - 1) / kTileM + d.B);
@@ -157,9 +157,14 @@ Layout attn_layout(const hstu_dims& d, int is_bwd) {
         const size_t D = (size_t)d.H * d.d_v;
         L.dy = off;
         off = align_up(off + (size_t)d.T * D * elem_size(d.dtype), 256);
-        L.n_part = ln_bwd_partials(d.T);
+        // LayerNorm partial rows: one per block, or one per (block, group) for Group LayerNorm
+        L.n_part = n_groups > 1 ? gln_blocks(d.T) : ln_bwd_partials(d.T);
         L.part = off;
-        off = align_up(off + (size_t)L.n_part * 2 * D * 4, 256);
+        off = align_up(off + (size_t)L.n_part * (n_groups > 1 ? n_groups : 1) * 2 * D * 4, 256);
+        if (n_groups > 1) {
+            L.gmask = off;                       // groups each grouped block holds
+            off = align_up(off + (size_t)L.n_part * 4, 256);
+        }
         if (d.dtype == HSTU_BF16) {
             L.dq_acc = off;                      // fp32 dQ accumulated across key tiles
             off = align_up(off + (size_t)d.T * D * 4, 256);
@@ -252,18 +257,47 @@ size_t hstu_attn_workspace_bytes(const hstu_dims* dims, int32_t mask_kind, int32
     return attn_layout(*dims, is_bwd ? 1 : 0).total;
 }
 
-int hstu_attn_fwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void* q, const void* k,
-                  const void* v, const void* u, const int32_t* seq_offsets, const int64_t* timestamps,
-                  const float* rab_pos, const float* rab_time, const float* ln_gamma,
-                  const float* ln_beta, void* y, void* o_pre, float* ln_mean, float* ln_rstd,
-                  void* workspace, size_t workspace_bytes, void* stream) {
+size_t hstu_attn_workspace_bytes_gln(const hstu_dims* dims, int32_t mask_kind, int32_t n_groups, int32_t is_bwd) {
+    if (n_groups < 1 || n_groups > kLnMaxGroups) return 0;
+    if (hstu_attn_workspace_bytes(dims, mask_kind, is_bwd) == 0) return 0;
+    if ((long long)n_groups * dims->H * dims->d_v > kLnMaxGroupCols) return 0;
+    return attn_layout(*dims, is_bwd ? 1 : 0, n_groups).total;
+}
+
+namespace {
+
+// Group LayerNorm arguments: n_groups in [1, kLnMaxGroups], G * D within the backward's
+// shared-memory sums, and a token_group array whenever G > 1.
+int check_norm(const hstu_norm_spec* n, const hstu_dims& d, int* G, const uint8_t** group) {
+    if (!n) {
+        *G = 1;
+        *group = nullptr;
+        return HSTU_OK;
+    }
+    if (n->n_groups < 1 || n->n_groups > kLnMaxGroups) return HSTU_ERR_INVALID_ARG;
+    if ((long long)n->n_groups * d.H * d.d_v > kLnMaxGroupCols) return HSTU_ERR_UNSUPPORTED;
+    if (n->n_groups > 1 && d.T > 0 && !n->token_group) return HSTU_ERR_INVALID_ARG;
+    *G = n->n_groups;
+    *group = n->n_groups > 1 ? n->token_group : nullptr;
+    return HSTU_OK;
+}
+
+int attn_fwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_norm_spec* norm,
+                  const void* q, const void* k, const void* v, const void* u, const int32_t* seq_offsets,
+                  const int64_t* timestamps, const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta, void* y, void* o_pre, float* ln_mean,
+                  float* ln_rstd, void* workspace, size_t workspace_bytes, void* stream) {
     int st = check_dims(dims);
+    if (st != HSTU_OK) return st;
+    int G = 1;
+    const uint8_t* group = nullptr;
+    st = check_norm(norm, *dims, &G, &group);
     if (st != HSTU_OK) return st;
     int kind = 0;
     st = check_mask(mask, &kind);
     if (st != HSTU_OK) return st;
     const hstu_dims& d = *dims;
-    const Layout L = attn_layout(d, 0);
+    const Layout L = attn_layout(d, 0, G);
     if (!aligned(workspace, 256)) return HSTU_ERR_WORKSPACE;
     if (workspace_bytes < L.total) return HSTU_ERR_WORKSPACE;
     if (d.T == 0) return HSTU_OK;
@@ -342,24 +376,32 @@ int hstu_attn_fwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     lp.o = o_pre;
     lp.mean = ln_mean;
     lp.rstd = ln_rstd;
+    lp.G = G;
+    lp.group = group;
+    lp.status = &ctrl->status;
+    if (G > 1) lp.n_part = gln_blocks(d.T);           // grid of the grouped forward
     return cuda_status(launch_ln_fwd(d.dtype == HSTU_F32, lp, s));
 }
 
-int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void* q, const void* k,
-                  const void* v, const void* u, const int32_t* seq_offsets, const int64_t* timestamps,
-                  const float* rab_pos, const float* rab_time, const float* ln_gamma,
-                  const float* ln_beta, const void* y, const float* ln_mean, const float* ln_rstd,
-                  const void* d_o_pre, void* dq, void* dk, void* dv, void* du, float* d_rab_pos,
-                  float* d_rab_time, float* d_gamma, float* d_beta, void* workspace,
+int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_norm_spec* norm,
+                  const void* q, const void* k, const void* v, const void* u, const int32_t* seq_offsets,
+                  const int64_t* timestamps, const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta, const void* y, const float* ln_mean,
+                  const float* ln_rstd, const void* d_o_pre, void* dq, void* dk, void* dv, void* du,
+                  float* d_rab_pos, float* d_rab_time, float* d_gamma, float* d_beta, void* workspace,
                   size_t workspace_bytes, void* stream) {
     int st = check_dims(dims);
+    if (st != HSTU_OK) return st;
+    int G = 1;
+    const uint8_t* group = nullptr;
+    st = check_norm(norm, *dims, &G, &group);
     if (st != HSTU_OK) return st;
     int kind = 0;
     st = check_mask(mask, &kind);
     if (st != HSTU_OK) return st;
     if (kind == HSTU_KIND_MFSEQ) return HSTU_ERR_UNSUPPORTED;   // scoring pass: forward only
     const hstu_dims& d = *dims;
-    const Layout L = attn_layout(d, 1);
+    const Layout L = attn_layout(d, 1, G);
     if (!aligned(workspace, 256)) return HSTU_ERR_WORKSPACE;
     if (workspace_bytes < L.total) return HSTU_ERR_WORKSPACE;
     if (!aligned(d_rab_pos, 4) || !aligned(d_rab_time, 4) || !aligned(d_gamma, 4) ||
@@ -370,8 +412,8 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * d.n_pos - 1), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * d.n_tbuckets, s);
     if (e == cudaSuccess && d.T == 0) {
-        e = cudaMemsetAsync(d_gamma, 0, sizeof(float) * D, s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(d_beta, 0, sizeof(float) * D, s);
+        e = cudaMemsetAsync(d_gamma, 0, sizeof(float) * D * G, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(d_beta, 0, sizeof(float) * D * G, s);
     }
     if (e != cudaSuccess) return cuda_status(e);
     if (d.T == 0) return HSTU_OK;
@@ -425,6 +467,10 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     lp.n_part = L.n_part;
     lp.d_gamma = d_gamma;
     lp.d_beta = d_beta;
+    lp.G = G;
+    lp.group = group;
+    lp.status = &ctrl->status;
+    if (G > 1) lp.gmask = at<int>(workspace, L.gmask);
     st = cuda_status(launch_ln_bwd(d.dtype == HSTU_F32, lp, s));
     if (st != HSTU_OK) return st;
 
@@ -478,6 +524,52 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     st = cuda_status(launch_rab_reduce(rab_part, grid, d.n_pos, d.n_tbuckets, d_rab_pos, d_rab_time, s));
     if (st != HSTU_OK) return st;
     return cuda_status(launch_f32_to_bf16(dq_acc, static_cast<__nv_bfloat16*>(dq), (long long)d.T * D, s));
+}
+
+}  // namespace
+
+int hstu_attn_fwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void* q, const void* k,
+                  const void* v, const void* u, const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time, const float* ln_gamma,
+                  const float* ln_beta, void* y, void* o_pre, float* ln_mean, float* ln_rstd,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+    return attn_fwd_impl(dims, mask, nullptr, q, k, v, u, seq_offsets, timestamps, rab_pos, rab_time, ln_gamma,
+                         ln_beta, y, o_pre, ln_mean, ln_rstd, workspace, workspace_bytes, stream);
+}
+
+int hstu_attn_fwd_gln(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_norm_spec* norm,
+                      const void* q, const void* k, const void* v, const void* u, const int32_t* seq_offsets,
+                      const int64_t* timestamps, const float* rab_pos, const float* rab_time,
+                      const float* ln_gamma, const float* ln_beta, void* y, void* o_pre, float* ln_mean,
+                      float* ln_rstd, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!norm) return HSTU_ERR_INVALID_ARG;
+    return attn_fwd_impl(dims, mask, norm, q, k, v, u, seq_offsets, timestamps, rab_pos, rab_time, ln_gamma,
+                         ln_beta, y, o_pre, ln_mean, ln_rstd, workspace, workspace_bytes, stream);
+}
+
+int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void* q, const void* k,
+                  const void* v, const void* u, const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time, const float* ln_gamma,
+                  const float* ln_beta, const void* y, const float* ln_mean, const float* ln_rstd,
+                  const void* d_o_pre, void* dq, void* dk, void* dv, void* du, float* d_rab_pos,
+                  float* d_rab_time, float* d_gamma, float* d_beta, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    return attn_bwd_impl(dims, mask, nullptr, q, k, v, u, seq_offsets, timestamps, rab_pos, rab_time, ln_gamma,
+                         ln_beta, y, ln_mean, ln_rstd, d_o_pre, dq, dk, dv, du, d_rab_pos, d_rab_time, d_gamma,
+                         d_beta, workspace, workspace_bytes, stream);
+}
+
+int hstu_attn_bwd_gln(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_norm_spec* norm,
+                      const void* q, const void* k, const void* v, const void* u, const int32_t* seq_offsets,
+                      const int64_t* timestamps, const float* rab_pos, const float* rab_time,
+                      const float* ln_gamma, const float* ln_beta, const void* y, const float* ln_mean,
+                      const float* ln_rstd, const void* d_o_pre, void* dq, void* dk, void* dv, void* du,
+                      float* d_rab_pos, float* d_rab_time, float* d_gamma, float* d_beta, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    if (!norm) return HSTU_ERR_INVALID_ARG;
+    return attn_bwd_impl(dims, mask, norm, q, k, v, u, seq_offsets, timestamps, rab_pos, rab_time, ln_gamma,
+                         ln_beta, y, ln_mean, ln_rstd, d_o_pre, dq, dk, dv, du, d_rab_pos, d_rab_time, d_gamma,
+                         d_beta, workspace, workspace_bytes, stream);
 }
 
 size_t hstu_mfalcon_workspace_bytes(const hstu_mfalcon_dims* dims, int32_t b_m) {

@@ -128,11 +128,21 @@ struct LnParams {
     void* dy;
     float dy_scale;  // dY is written times this (1/(2 alpha) for the tensor-core backward)
     void* du;
-    float* part;     // [n_blocks][2][D]
+    float* part;     // [n_blocks][G][2][D]
     int n_part;
-    float* d_gamma;
-    float* d_beta;
+    float* d_gamma;  // [G][D]
+    float* d_beta;   // [G][D]
+    // Group LayerNorm: gamma / beta (and their gradients) are [G][D], row t uses
+    // group[t]; G <= 1 and group == nullptr is the plain LayerNorm
+    const uint8_t* group;
+    int G;
+    int* status;     // kStatusBounds is set here for a group id >= G (the row then uses G - 1)
+    int* gmask;      // [blocks] groups each grouped backward block left a partial row for
 };
+
+constexpr int kLnMaxGroups = 16;
+constexpr int kGlnMaxBlocks = 148 * 16;   // grouped LayerNorm blocks (each a contiguous chunk of rows)
+constexpr int kLnMaxGroupCols = 16384;   // G * D: bound on the [G][D] affine tables
 
 // ---- opt-in per-kernel timing (profile.cu)
 enum ProfKind {
@@ -166,6 +176,7 @@ cudaError_t launch_rab_reduce(const float* part, int n_part, int P, int nb, floa
 cudaError_t launch_ln_fwd(int dtype_f32, const LnParams& p, cudaStream_t s);
 cudaError_t launch_ln_bwd(int dtype_f32, const LnParams& p, cudaStream_t s);
 int ln_bwd_partials(long long T);
+int gln_blocks(long long T);
 cudaError_t launch_debug_indices(int B, int kind, const int32_t* off, const int64_t* ts,
                                  const int32_t* ns, const int32_t* nr, int P, int nb,
                                  const int64_t* pair_off, int max_len, uint8_t* m, int16_t* pi,

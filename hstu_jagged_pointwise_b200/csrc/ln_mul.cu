@@ -217,24 +217,255 @@ __global__ void __launch_bounds__(32 * WPR) ln_bwd_kernel(LnParams p) {
     }
 }
 
+// ---------------------------------------------------------------- Group LayerNorm
+// MTGR deep-dive, section 2, and the MTGR arXiv report (GLN): tokens from different
+// sources (profile, behaviour, real-time, candidate) are normalised by group so that
+// each keeps its own distribution.  Reading: the statistics stay per token over D;
+// every group has its own affine gamma_g / beta_g.  Row t uses g = group[t].
+//
+// Every block owns a contiguous chunk of rows.  It reads the chunk's group ids once,
+// lists the rows group by group in shared memory (a stable warp-ballot compaction), and
+// then runs the plain row loop once per group present: gamma_g / beta_g and the
+// backward's dgamma_g / dbeta_g sums stay in registers as in the plain kernels.  The
+// backward leaves one partial row per (block, group present) and a bit mask of the groups
+// present; the reduction adds a group's rows in block order (deterministic).
+constexpr int kGlnSeg = 1024;              // rows listed at a time (a chunk may take several)
+
+struct GlnList {
+    uint8_t g[kGlnSeg];
+    int16_t row[kGlnSeg];
+    int start[kLnMaxGroups];
+    int count[kLnMaxGroups];
+};
+
+__device__ __forceinline__ long long gln_chunk(const LnParams& p) {
+    return (p.T + gridDim.x - 1) / gridDim.x;
+}
+
+// Lists rows [r0, r0 + n) group by group: rows of group k are row[start[k] .. + count[k]).
+// A group id >= G sets kStatusBounds and counts as G - 1.
+__device__ void gln_list(const LnParams& p, long long r0, int n, GlnList& L) {
+    int bad = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        int g = p.group[r0 + i];
+        if (g >= p.G) {
+            bad = 1;
+            g = p.G - 1;
+        }
+        L.g[i] = (uint8_t)g;
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(p.status, kStatusBounds);
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int base = 0;
+        for (int k = 0; k < p.G; k++) {
+            const int first = base;
+            for (int i0 = 0; i0 < n; i0 += 32) {
+                const int i = i0 + lane;
+                const bool mine = i < n && L.g[i] == k;
+                const unsigned bal = __ballot_sync(0xffffffffu, mine);
+                if (mine) L.row[base + __popc(bal & ((1u << lane) - 1u))] = (int16_t)i;
+                base += __popc(bal);
+            }
+            if (lane == 0) {
+                L.start[k] = first;
+                L.count[k] = base - first;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+template <typename T, int WPR, int NCW>
+__global__ void __launch_bounds__(32 * WPR) gln_fwd_kernel(LnParams p) {
+    constexpr int V = Vec<T>::N;
+    __shared__ float red[2][4];
+    __shared__ GlnList L;
+    const int nvec = p.D / V;
+    const long long chunk = gln_chunk(p);
+    const long long c0 = (long long)blockIdx.x * chunk, c1 = min(p.T, c0 + chunk);
+    for (long long seg = c0; seg < c1; seg += kGlnSeg) {
+        const int n = (int)min((long long)kGlnSeg, c1 - seg);
+        gln_list(p, seg, n, L);
+        for (int grp = 0; grp < p.G; grp++) {
+            const int cnt = L.count[grp], st = L.start[grp];
+            if (cnt == 0) continue;
+            float gm[NCW][V], bt[NCW][V];
+#pragma unroll
+            for (int k = 0; k < NCW; k++) {
+                const int vi = k * 32 * WPR + threadIdx.x;
+                if (vi < nvec) {
+                    load_f32v(p.gamma + (size_t)grp * p.D, vi * V, V, gm[k]);
+                    load_f32v(p.beta + (size_t)grp * p.D, vi * V, V, bt[k]);
+                }
+            }
+            for (int j = 0; j < cnt; j++) {
+                const long long row = seg + L.row[st + j];
+                const size_t base = (size_t)row * p.D;
+                float x[NCW][V], u[NCW][V];
+                float s = 0.f;
+#pragma unroll
+                for (int k = 0; k < NCW; k++) {
+                    const int vi = k * 32 * WPR + threadIdx.x;
+                    if (vi < nvec) {
+                        Vec<T>::load(p.y, base + (size_t)vi * V, x[k]);
+                        Vec<T>::load(p.u, base + (size_t)vi * V, u[k]);
+#pragma unroll
+                        for (int e = 0; e < V; e++) s += x[k][e];
+                    }
+                }
+                const float mean = block_sum<WPR>(s, red, 0) / p.D;
+                float q = 0.f;
+#pragma unroll
+                for (int k = 0; k < NCW; k++) {
+                    const int vi = k * 32 * WPR + threadIdx.x;
+                    if (vi < nvec) {
+#pragma unroll
+                        for (int e = 0; e < V; e++) {
+                            const float d = x[k][e] - mean;
+                            q += d * d;
+                        }
+                    }
+                }
+                const float rstd = rsqrtf(block_sum<WPR>(q, red, 1) / p.D + p.eps);
+#pragma unroll
+                for (int k = 0; k < NCW; k++) {
+                    const int vi = k * 32 * WPR + threadIdx.x;
+                    if (vi < nvec) {
+                        float o[V];
+#pragma unroll
+                        for (int e = 0; e < V; e++) o[e] = ((x[k][e] - mean) * rstd * gm[k][e] + bt[k][e]) * u[k][e];
+                        Vec<T>::store(p.o, base + (size_t)vi * V, o);
+                    }
+                }
+                if (threadIdx.x == 0) {
+                    if (p.mean) p.mean[row] = mean;
+                    if (p.rstd) p.rstd[row] = rstd;
+                }
+            }
+        }
+        __syncthreads();                                   // L is rebuilt for the next segment
+    }
+}
+
+template <typename T, int WPR, int NCW>
+__global__ void __launch_bounds__(32 * WPR) gln_bwd_kernel(LnParams p) {
+    constexpr int V = Vec<T>::N;
+    __shared__ float red[2][4];
+    __shared__ GlnList L;
+    const int nvec = p.D / V;
+    const long long chunk = gln_chunk(p);
+    const long long c0 = (long long)blockIdx.x * chunk, c1 = min(p.T, c0 + chunk);
+    unsigned present = 0;                                  // groups with a partial row written
+    for (long long seg = c0; seg < c1; seg += kGlnSeg) {
+        const int n = (int)min((long long)kGlnSeg, c1 - seg);
+        gln_list(p, seg, n, L);
+        for (int grp = 0; grp < p.G; grp++) {
+            const int cnt = L.count[grp], st = L.start[grp];
+            if (cnt == 0) continue;
+            float gm[NCW][V], bt[NCW][V], ag[NCW][V], ab[NCW][V];
+#pragma unroll
+            for (int k = 0; k < NCW; k++) {
+                const int vi = k * 32 * WPR + threadIdx.x;
+#pragma unroll
+                for (int e = 0; e < V; e++) ag[k][e] = ab[k][e] = 0.f;
+                if (vi < nvec) {
+                    load_f32v(p.gamma + (size_t)grp * p.D, vi * V, V, gm[k]);
+                    load_f32v(p.beta + (size_t)grp * p.D, vi * V, V, bt[k]);
+                }
+            }
+            for (int j = 0; j < cnt; j++) {
+                const long long row = seg + L.row[st + j];
+                const size_t base = (size_t)row * p.D;
+                const float mean = p.mean[row], rstd = p.rstd[row];
+                float xh[NCW][V], gx[NCW][V];
+                float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+                for (int k = 0; k < NCW; k++) {
+                    const int vi = k * 32 * WPR + threadIdx.x;
+                    if (vi < nvec) {
+                        float y[V], u[V], g[V], du[V];
+                        Vec<T>::load(p.y, base + (size_t)vi * V, y);
+                        Vec<T>::load(p.u, base + (size_t)vi * V, u);
+                        Vec<T>::load(p.g, base + (size_t)vi * V, g);
+#pragma unroll
+                        for (int e = 0; e < V; e++) {
+                            xh[k][e] = (y[e] - mean) * rstd;
+                            du[e] = g[e] * (xh[k][e] * gm[k][e] + bt[k][e]);
+                            const float gl = g[e] * u[e];
+                            ag[k][e] += gl * xh[k][e];
+                            ab[k][e] += gl;
+                            gx[k][e] = gl * gm[k][e];
+                            m1 += gx[k][e];
+                            m2 += gx[k][e] * xh[k][e];
+                        }
+                        Vec<T>::store(p.du, base + (size_t)vi * V, du);
+                    }
+                }
+                m1 = block_sum<WPR>(m1, red, 0) / p.D;
+                m2 = block_sum<WPR>(m2, red, 1) / p.D;
+                const float rs = rstd * p.dy_scale;
+#pragma unroll
+                for (int k = 0; k < NCW; k++) {
+                    const int vi = k * 32 * WPR + threadIdx.x;
+                    if (vi < nvec) {
+                        float dy[V];
+#pragma unroll
+                        for (int e = 0; e < V; e++) dy[e] = rs * (gx[k][e] - m1 - xh[k][e] * m2);
+                        Vec<T>::store(p.dy, base + (size_t)vi * V, dy);
+                    }
+                }
+            }
+            // this block's partial row of group grp: written the first time, then added to
+            // (only this thread ever touches these columns of the row)
+            float* part = p.part + ((size_t)blockIdx.x * p.G + grp) * 2 * p.D;
+            const bool first = !(present & (1u << grp));
+#pragma unroll
+            for (int k = 0; k < NCW; k++) {
+                const int vi = k * 32 * WPR + threadIdx.x;
+                if (vi < nvec) {
+#pragma unroll
+                    for (int e = 0; e < V; e++) {
+                        float* a = part + vi * V + e;
+                        float* c = part + p.D + vi * V + e;
+                        *a = first ? ag[k][e] : *a + ag[k][e];
+                        *c = first ? ab[k][e] : *c + ab[k][e];
+                    }
+                }
+            }
+            present |= 1u << grp;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) p.gmask[blockIdx.x] = (int)present;
+}
+
 // Sums the per-block partials in a fixed order (deterministic): a block owns 32 of the
-// 2D columns; warp w sums the partials w, w+8, w+16, ... of each column (coalesced
-// 128-byte rows), and warp 0 adds the eight warp sums in order.
+// 2D columns of one group (blockIdx.y; the plain LayerNorm is group 0); warp w sums the
+// partial rows of blocks w, w+8, w+16, ... that hold the group (coalesced 128-byte rows),
+// and warp 0 adds the eight warp sums in order.
 __global__ void __launch_bounds__(256) ln_bwd_reduce_kernel(LnParams p) {
     __shared__ float acc[8][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.y;
     const int c = blockIdx.x * 32 + lane;
     float s = 0.f;
-    if (c < 2 * p.D)
-        for (int k = warp; k < p.n_part; k += 8) s += p.part[(size_t)k * 2 * p.D + c];
+    if (c < 2 * p.D) {
+        if (p.G > 1) {
+            for (int k = warp; k < p.n_part; k += 8)
+                if (p.gmask[k] & (1 << g)) s += p.part[((size_t)k * p.G + g) * 2 * p.D + c];
+        } else {
+            for (int k = warp; k < p.n_part; k += 8) s += p.part[(size_t)k * 2 * p.D + c];
+        }
+    }
     acc[warp][lane] = s;
     __syncthreads();
     if (warp == 0 && c < 2 * p.D) {
         float t = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; w++) t += acc[w][lane];
-        if (c < p.D) p.d_gamma[c] = t;
-        else p.d_beta[c - p.D] = t;
+        if (c < p.D) p.d_gamma[(size_t)g * p.D + c] = t;
+        else p.d_beta[(size_t)g * p.D + c - p.D] = t;
     }
 }
 
@@ -260,13 +491,21 @@ bool pick_shape(int D, int* wpr, int* ncw) {
         else KERNEL<T, 4, 8><<<GRID, 128, 0, s>>>(p);                                        \
     } while (0)
 
+#define HSTU_GLN_DISPATCH(KERNEL, GRID, WPR_, NCW_) HSTU_LN_DISPATCH(KERNEL, GRID, WPR_, NCW_)
+
+bool grouped(const LnParams& p) { return p.G > 1; }
+
 template <typename T>
 cudaError_t fwd_t(const LnParams& p, cudaStream_t s) {
     int wpr = 0, ncw = 0;
     if (!pick_shape<T>(p.D, &wpr, &ncw)) return cudaErrorInvalidValue;
-    const unsigned grid = (unsigned)(p.T < kLnMaxBlocks ? p.T : kLnMaxBlocks);
     prof_begin(kProfLnFwd, s);
-    HSTU_LN_DISPATCH(ln_fwd_kernel, grid, wpr, ncw);
+    if (grouped(p)) {
+        HSTU_GLN_DISPATCH(gln_fwd_kernel, (unsigned)p.n_part, wpr, ncw);
+    } else {
+        const unsigned grid = (unsigned)(p.T < kLnMaxBlocks ? p.T : kLnMaxBlocks);
+        HSTU_LN_DISPATCH(ln_fwd_kernel, grid, wpr, ncw);
+    }
     prof_end(kProfLnFwd, s);
     return cudaGetLastError();
 }
@@ -275,24 +514,35 @@ template <typename T>
 cudaError_t bwd_t(const LnParams& p, cudaStream_t s) {
     int wpr = 0, ncw = 0;
     if (!pick_shape<T>(p.D, &wpr, &ncw)) return cudaErrorInvalidValue;
-    const unsigned grid = (unsigned)p.n_part;
     prof_begin(kProfLnBwd, s);
-    HSTU_LN_DISPATCH(ln_bwd_kernel, grid, wpr, ncw);
+    if (grouped(p)) {
+        HSTU_GLN_DISPATCH(gln_bwd_kernel, (unsigned)p.n_part, wpr, ncw);
+    } else {
+        HSTU_LN_DISPATCH(ln_bwd_kernel, (unsigned)p.n_part, wpr, ncw);
+    }
     prof_end(kProfLnBwd, s);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     prof_begin(kProfLnBwdReduce, s);
-    ln_bwd_reduce_kernel<<<(2 * p.D + 31) / 32, 256, 0, s>>>(p);
+    ln_bwd_reduce_kernel<<<dim3((2 * p.D + 31) / 32, grouped(p) ? p.G : 1), 256, 0, s>>>(p);
     prof_end(kProfLnBwdReduce, s);
     return cudaGetLastError();
 }
 
 #undef HSTU_LN_DISPATCH
+#undef HSTU_GLN_DISPATCH
 
 }  // namespace
 
 int ln_bwd_partials(long long T) {
     long long n = T < kLnMaxBlocks ? T : kLnMaxBlocks;   // one block per row, grid-stride beyond
+    return n < 1 ? 1 : (int)n;
+}
+
+// Blocks of the grouped kernels (each takes a contiguous chunk of rows) and the partial
+// rows of [2][D] the grouped backward leaves: one per (block, group).
+int gln_blocks(long long T) {
+    const long long n = T < kGlnMaxBlocks ? T : kGlnMaxBlocks;
     return n < 1 ? 1 : (int)n;
 }
 

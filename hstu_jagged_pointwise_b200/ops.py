@@ -62,8 +62,11 @@ def make_mask(kind: str = "causal", n_static: Optional[torch.Tensor] = None,
     raise ValueError(f"unknown mask kind {kind!r}")
 
 
-def attn_workspace_bytes(dims: capi.HstuDims, mask_kind: int, is_bwd: bool) -> int:
-    n = capi.LIB.hstu_attn_workspace_bytes(C.byref(dims), mask_kind, 1 if is_bwd else 0)
+def attn_workspace_bytes(dims: capi.HstuDims, mask_kind: int, is_bwd: bool, n_groups: int = 1) -> int:
+    if n_groups > 1:
+        n = capi.LIB.hstu_attn_workspace_bytes_gln(C.byref(dims), mask_kind, n_groups, 1 if is_bwd else 0)
+    else:
+        n = capi.LIB.hstu_attn_workspace_bytes(C.byref(dims), mask_kind, 1 if is_bwd else 0)
     if n == 0:
         raise capi.HstuError(capi.HSTU_ERR_INVALID_ARG, "hstu_attn_workspace_bytes")
     return int(n)
@@ -84,7 +87,10 @@ class Layer:
     def __init__(self, seq_offsets: torch.Tensor, timestamps: torch.Tensor, H: int, d: int,
                  dtype: torch.dtype, alpha: float, max_seq_len: int, mask_kind: str = "causal",
                  n_static: Optional[torch.Tensor] = None, n_realtime: Optional[torch.Tensor] = None,
-                 n_pos: int = 256, n_tbuckets: int = 64, ln_eps: float = 1e-5):
+                 n_pos: int = 256, n_tbuckets: int = 64, ln_eps: float = 1e-5, n_groups: int = 1,
+                 token_group: Optional[torch.Tensor] = None):
+        """n_groups > 1 selects Group LayerNorm: token_group (uint8 [T]) names each token's
+        group, and ln_gamma / ln_beta (and their gradients) are [n_groups, H*d]."""
         _need(seq_offsets, "seq_offsets", torch.int32)
         _need(timestamps, "timestamps", torch.int64)
         self.seq_offsets, self.timestamps = seq_offsets, timestamps
@@ -94,10 +100,16 @@ class Layer:
         self.n_static, self.n_realtime = n_static, n_realtime
         self.dims = make_dims(self.T, self.B, H, d, dtype, alpha, max_seq_len, n_pos, n_tbuckets, ln_eps)
         self.mask = make_mask(mask_kind, n_static, n_realtime)
+        self.norm = None
+        if n_groups > 1:
+            _need(token_group, "token_group", torch.uint8)
+            self.token_group = token_group
+            self.norm = capi.HstuNormSpec(n_groups=int(n_groups), token_group=token_group.data_ptr())
         self.device = seq_offsets.device
-        n = attn_workspace_bytes(self.dims, self.mask.kind, False)
+        G = int(n_groups)
+        n = attn_workspace_bytes(self.dims, self.mask.kind, False, G)
         if self.mask.kind != capi.HSTU_MASK_MFALCON_SEQ:   # the full-sequence M-FALCON mask is forward only
-            n = max(n, attn_workspace_bytes(self.dims, self.mask.kind, True))
+            n = max(n, attn_workspace_bytes(self.dims, self.mask.kind, True, G))
         self.ws = workspace(n, self.device)
 
     @property
@@ -113,10 +125,13 @@ class Layer:
             out = dict(y=torch.empty_like(q), o_pre=torch.empty_like(q),
                        mean=torch.empty(self.T, dtype=torch.float32, device=self.device),
                        rstd=torch.empty(self.T, dtype=torch.float32, device=self.device))
-        st = capi.LIB.hstu_attn_fwd(
-            C.byref(self.dims), C.byref(self.mask), _p(q), _p(k), _p(v), _p(u), _p(self.seq_offsets),
-            _p(self.timestamps), _p(rab_pos), _p(rab_time), _p(ln_gamma), _p(ln_beta), _p(out["y"]),
-            _p(out["o_pre"]), _p(out["mean"]), _p(out["rstd"]), _p(self.ws), self.ws.numel(), _stream())
+        args = (_p(q), _p(k), _p(v), _p(u), _p(self.seq_offsets), _p(self.timestamps), _p(rab_pos), _p(rab_time),
+                _p(ln_gamma), _p(ln_beta), _p(out["y"]), _p(out["o_pre"]), _p(out["mean"]), _p(out["rstd"]),
+                _p(self.ws), self.ws.numel(), _stream())
+        if self.norm is None:
+            st = capi.LIB.hstu_attn_fwd(C.byref(self.dims), C.byref(self.mask), *args)
+        else:
+            st = capi.LIB.hstu_attn_fwd_gln(C.byref(self.dims), C.byref(self.mask), C.byref(self.norm), *args)
         capi.check(st, "hstu_attn_fwd")
         return out
 
@@ -128,12 +143,15 @@ class Layer:
                        du=torch.empty_like(u),
                        d_rab_pos=torch.empty_like(rab_pos), d_rab_time=torch.empty_like(rab_time),
                        d_gamma=torch.empty_like(ln_gamma), d_beta=torch.empty_like(ln_beta))
-        st = capi.LIB.hstu_attn_bwd(
-            C.byref(self.dims), C.byref(self.mask), _p(q), _p(k), _p(v), _p(u), _p(self.seq_offsets),
-            _p(self.timestamps), _p(rab_pos), _p(rab_time), _p(ln_gamma), _p(ln_beta), _p(fwd["y"]),
-            _p(fwd["mean"]), _p(fwd["rstd"]), _p(d_o_pre), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
-            _p(out["du"]), _p(out["d_rab_pos"]), _p(out["d_rab_time"]), _p(out["d_gamma"]),
-            _p(out["d_beta"]), _p(self.ws), self.ws.numel(), _stream())
+        args = (_p(q), _p(k), _p(v), _p(u), _p(self.seq_offsets), _p(self.timestamps), _p(rab_pos), _p(rab_time),
+                _p(ln_gamma), _p(ln_beta), _p(fwd["y"]), _p(fwd["mean"]), _p(fwd["rstd"]), _p(d_o_pre),
+                _p(out["dq"]), _p(out["dk"]), _p(out["dv"]), _p(out["du"]), _p(out["d_rab_pos"]),
+                _p(out["d_rab_time"]), _p(out["d_gamma"]), _p(out["d_beta"]), _p(self.ws), self.ws.numel(),
+                _stream())
+        if self.norm is None:
+            st = capi.LIB.hstu_attn_bwd(C.byref(self.dims), C.byref(self.mask), *args)
+        else:
+            st = capi.LIB.hstu_attn_bwd_gln(C.byref(self.dims), C.byref(self.mask), C.byref(self.norm), *args)
         capi.check(st, "hstu_attn_bwd")
         return out
 

@@ -77,6 +77,9 @@ class Workload:
     cand_v: Optional[torch.Tensor] = None
     cand_u: Optional[torch.Tensor] = None
     b_m: int = 0
+    # Group LayerNorm: gamma / beta are [n_groups, D] and token t uses row token_group[t]
+    n_groups: int = 1
+    token_group: Optional[np.ndarray] = None  # uint8 [T]
     meta: dict = field(default_factory=dict)
 
     @property
@@ -289,6 +292,40 @@ def make_mfalcon(n_hist, n_cand, H: int, d: int, dtype=torch.bfloat16, seed: int
                     hist_k=hk, hist_v=hv, cand_offsets=co,
                     cand_ts=np.concatenate(cand_ts) if Tc else np.zeros(0, np.int64),
                     cand_q=cq, cand_k=ck, cand_v=cv, cand_u=cu, b_m=b_m)
+
+
+GLN_PROFILE, GLN_BEHAVIOUR, GLN_REALTIME, GLN_CANDIDATE = 0, 1, 2, 3
+
+
+def with_group_norm(w: Workload, seed: int = 0, groups=None) -> Workload:
+    """Group LayerNorm on a self-attention workload: one gamma/beta row per token
+    source.  MTGR rows [profile | long-term behaviour | real-time | candidates] get
+    groups 0..3 from their segment sizes; other workloads take `groups`, a uint8
+    array [T] or a group count to draw uniform random ids from.  The affine rows are
+    1 + N(0, 0.1) and N(0, 0.1) (distinct per group, so a routing error shows)."""
+    gen = torch.Generator().manual_seed(seed + 505)
+    if groups is None:
+        assert w.kind == "mtgr", "token groups from segments need an MTGR workload"
+        parts = []
+        for b in range(w.B):
+            L = int(w.offsets[b + 1] - w.offsets[b])
+            npf = int(w.meta["n_profile"][b])
+            S, R = int(w.n_static[b]), int(w.n_realtime[b])
+            parts.append(np.concatenate([np.full(npf, GLN_PROFILE), np.full(S - npf, GLN_BEHAVIOUR),
+                                         np.full(R, GLN_REALTIME), np.full(L - S - R, GLN_CANDIDATE)]))
+        tg = np.concatenate(parts) if parts else np.zeros(0)
+        G = 4
+    elif np.isscalar(groups):
+        G = int(groups)
+        tg = np.random.Generator(np.random.PCG64(seed)).integers(0, G, size=w.T)
+    else:
+        tg = np.asarray(groups)
+        G = int(tg.max()) + 1 if tg.size else 1
+    w.n_groups = G
+    w.token_group = tg.astype(np.uint8)
+    w.gamma = 1.0 + randn(gen, (G, w.D), torch.float32, 0.1)
+    w.beta = randn(gen, (G, w.D), torch.float32, 0.1)
+    return w
 
 
 def mfalcon_seq_from(w: Workload, seed: int = 0, name: str = "mfalcon_seq") -> Workload:

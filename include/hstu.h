@@ -108,6 +108,17 @@ typedef struct {
     float ln_eps;         /* LayerNorm epsilon (1e-5 in the workloads) */
 } hstu_dims;
 
+/* Group LayerNorm (MTGR deep-dive, section 2; MTGR arXiv report, GLN): tokens
+ * from different sources (profile, behaviour, real-time, candidate) are
+ * normalised per group so that each keeps its own distribution.  Reading used
+ * here: mean and variance stay per token over D; group g has its own affine
+ * gamma_g, beta_g, so token t gets LN(Y_t) * gamma_{group[t]} + beta_{group[t]}.
+ * n_groups = 1 is the plain LayerNorm (token_group is then ignored). */
+typedef struct {
+    int32_t n_groups;              /* G in [1, 16]; G * H * d_v <= 16384 */
+    const uint8_t* token_group;    /* DEVICE uint8 [T], values in [0, G); required when G > 1 */
+} hstu_norm_spec;
+
 /* Bytes of workspace hstu_attn_fwd (is_bwd = 0) or hstu_attn_bwd (is_bwd = 1)
  * needs for these dims and mask kind; 0 when the arguments are invalid, and 0
  * for is_bwd = 1 with HSTU_MASK_MFALCON_SEQ (no backward for that mask). */
@@ -120,6 +131,29 @@ HSTU_API size_t hstu_attn_workspace_bytes(const hstu_dims* dims, int32_t mask_ki
  *      o_pre [T, H*d_v], ln_mean [T], ln_rstd [T].
  * Rows of y / o_pre that belong to no sequence are not written. */
 HSTU_API int hstu_attn_fwd(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const void* q, const void* k, const void* v, const void* u,
+                  const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta,
+                  void* y, void* o_pre, float* ln_mean, float* ln_rstd,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of hstu_attn_fwd_gln (is_bwd = 0) / hstu_attn_bwd_gln
+ * (is_bwd = 1) with n_groups groups (the backward keeps LayerNorm partial sums
+ * per group); 0 when the arguments are invalid.  n_groups = 1 gives the plain
+ * size. */
+HSTU_API size_t hstu_attn_workspace_bytes_gln(const hstu_dims* dims, int32_t mask_kind, int32_t n_groups,
+                  int32_t is_bwd);
+
+/* hstu_attn_fwd with Group LayerNorm: ln_gamma and ln_beta are fp32 [G, H*d_v]
+ * (row g is group g's affine); the workspace is sized by
+ * hstu_attn_workspace_bytes_gln; everything else as hstu_attn_fwd.  A token whose group id is >= G sets the device status word
+ * (HSTU_ERR_DEVICE_BOUNDS through hstu_check_device_error) and is normalised
+ * with group G - 1.  NULL norm: HSTU_ERR_INVALID_ARG; n_groups outside
+ * [1, 16] or G > 1 without token_group: HSTU_ERR_INVALID_ARG; G * H * d_v >
+ * 16384: HSTU_ERR_UNSUPPORTED. */
+HSTU_API int hstu_attn_fwd_gln(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const hstu_norm_spec* norm,
                   const void* q, const void* k, const void* v, const void* u,
                   const int32_t* seq_offsets, const int64_t* timestamps,
                   const float* rab_pos, const float* rab_time,
@@ -171,6 +205,23 @@ HSTU_API int hstu_attn_fwd_noalloc(const hstu_dims* dims, const hstu_mask_spec* 
  * forward's outputs for the same inputs.  HSTU_MASK_MFALCON_SEQ returns
  * HSTU_ERR_UNSUPPORTED (a scoring pass: forward only). */
 HSTU_API int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const void* q, const void* k, const void* v, const void* u,
+                  const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time,
+                  const float* ln_gamma, const float* ln_beta,
+                  const void* y, const float* ln_mean, const float* ln_rstd,
+                  const void* d_o_pre,
+                  void* dq, void* dk, void* dv, void* du,
+                  float* d_rab_pos, float* d_rab_time, float* d_gamma, float* d_beta,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of hstu_attn_fwd_gln: ln_gamma, ln_beta, d_gamma and d_beta are fp32
+ * [G, H*d_v] (d_gamma[g] and d_beta[g] sum over the tokens of group g only;
+ * they are deterministic); the workspace is sized by
+ * hstu_attn_workspace_bytes_gln; everything else as hstu_attn_bwd.  Argument
+ * errors and bad group ids as hstu_attn_fwd_gln. */
+HSTU_API int hstu_attn_bwd_gln(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const hstu_norm_spec* norm,
                   const void* q, const void* k, const void* v, const void* u,
                   const int32_t* seq_offsets, const int64_t* timestamps,
                   const float* rab_pos, const float* rab_time,

@@ -240,18 +240,63 @@ def mfalcon(w, rows=None):
 # whole-layer conveniences
 # ----------------------------------------------------------------------------
 
+def gln_mul_fwd(y, u, gamma, beta, group, eps=1e-5):
+    """Group LayerNorm times u (MTGR deep-dive section 2; MTGR report, GLN): token t is
+    normalised over D as in ln_mul_fwd, with the affine row gamma[group[t]],
+    beta[group[t]].  Rows of one group go through ln_mul_fwd together."""
+    y = _c(y, np.float64)
+    u, g, b = f32(u), f32(gamma), f32(beta)
+    grp = np.asarray(group).astype(np.int64)
+    n, D = y.shape
+    o, mu, rs = np.zeros((n, D)), np.zeros(n), np.zeros(n)
+    for k in np.unique(grp):
+        r = np.nonzero(grp == k)[0]
+        o[r], mu[r], rs[r] = ln_mul_fwd(y[r], u[r], g[k], b[k], eps)
+    return o, mu, rs
+
+
+def gln_mul_bwd(y, u, gamma, beta, group, grad, eps=1e-5):
+    """Backward of gln_mul_fwd: (dy, du, dgamma [G, D], dbeta [G, D]); group k's affine
+    gradients sum over its own tokens only (zero for a group with no tokens)."""
+    y = _c(y, np.float64)
+    u, g, b, gr = f32(u), f32(gamma), f32(beta), f32(grad)
+    grp = np.asarray(group).astype(np.int64)
+    n, D = y.shape
+    dy, du = np.zeros((n, D)), np.zeros((n, D))
+    dg, db = np.zeros(g.shape), np.zeros(b.shape)
+    for k in np.unique(grp):
+        r = np.nonzero(grp == k)[0]
+        dy[r], du[r], dg[k], db[k] = ln_mul_bwd(y[r], u[r], g[k], b[k], gr[r], eps)
+    return dy, du, dg, db
+
+
+def norm_fwd(w, y, rows=None):
+    """The layer's Norm(y) * u for the listed rows: LayerNorm, or Group LayerNorm when
+    the workload names token groups."""
+    sel = slice(None) if rows is None else np.asarray(rows)
+    u = f32(w.u)[sel]
+    if getattr(w, "n_groups", 1) > 1:
+        return gln_mul_fwd(y, u, w.gamma, w.beta, np.asarray(w.token_group)[sel], w.eps)
+    return ln_mul_fwd(y, u, w.gamma, w.beta, w.eps)
+
+
+def norm_bwd(w, y, grad):
+    if getattr(w, "n_groups", 1) > 1:
+        return gln_mul_bwd(y, w.u, w.gamma, w.beta, w.token_group, grad, w.eps)
+    return ln_mul_bwd(y, w.u, w.gamma, w.beta, grad, w.eps)
+
+
 def layer_fwd(w, rows=None):
-    """(y, o_pre, mean, rstd) for the listed rows: attention, then LayerNorm(y) * u."""
+    """(y, o_pre, mean, rstd) for the listed rows: attention, then Norm(y) * u."""
     y = attn_fwd(w, rows)
-    u = f32(w.u) if rows is None else f32(w.u)[np.asarray(rows)]
-    o, mu, rs = ln_mul_fwd(y, u, w.gamma, w.beta, w.eps)
+    o, mu, rs = norm_fwd(w, y, rows)
     return y, o, mu, rs
 
 
 def layer_bwd(w):
-    """Full backward of o_pre = LN(attn(q,k,v)) * u for the upstream gradient w.grad."""
+    """Full backward of o_pre = Norm(attn(q,k,v)) * u for the upstream gradient w.grad."""
     y = attn_fwd(w)
-    dy, du, dg, db = ln_mul_bwd(y, w.u, w.gamma, w.beta, w.grad, w.eps)
+    dy, du, dg, db = norm_bwd(w, y, w.grad)
     dq, dk, dv, drp, drt = attn_bwd(w, dy)
     return dict(y=y, dy=dy, du=du, dgamma=dg, dbeta=db, dq=dq, dk=dk, dv=dv, d_rab_pos=drp, d_rab_time=drt)
 

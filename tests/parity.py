@@ -62,10 +62,8 @@ def assert_bf16(got, ref, name, storage=None):
 def storage_fwd(w, rows=None):
     """Oracle forward with the bf16 storage points rounded: Y stored, O_pre from the stored Y."""
     import oracle
-    y = oracle.attn_fwd(w, rows)
-    u = oracle.f32(w.u) if rows is None else oracle.f32(w.u)[np.asarray(rows)]
-    yb = bf16(y)
-    o, _, _ = oracle.ln_mul_fwd(yb, u, w.gamma, w.beta, w.eps)
+    yb = bf16(oracle.attn_fwd(w, rows))
+    o, _, _ = oracle.norm_fwd(w, yb, rows)
     return dict(y=yb, o_pre=bf16(o))
 
 
@@ -73,7 +71,7 @@ def storage_bwd(w):
     """Oracle backward with the bf16 storage points rounded (Y, dY, the stored gradients)."""
     import oracle
     yb = bf16(oracle.attn_fwd(w))
-    dy, du, dg, db = oracle.ln_mul_bwd(yb, w.u, w.gamma, w.beta, w.grad, w.eps)
+    dy, du, dg, db = oracle.norm_bwd(w, yb, w.grad)
     dq, dk, dv, drp, drt = oracle.attn_bwd(w, bf16(dy))
     return dict(y=yb, du=bf16(du), dq=bf16(dq), dk=bf16(dk), dv=bf16(dv), d_rab_pos=drp,
                 d_rab_time=drt, dgamma=dg, dbeta=db)
@@ -121,9 +119,13 @@ def dev(w, device="cuda"):
 def run_layer(w, backward=False, device="cuda"):
     from hstu_jagged_pointwise_b200 import ops
     d = dev(w, device)
+    tg = None
+    if w.n_groups > 1:
+        tg = torch.as_tensor(np.asarray(w.token_group, np.uint8)).to(device)
     layer = ops.Layer(d["offsets"], d["ts"], w.H, w.d, w.dtype, w.alpha, max(w.max_len, 1),
                       mask_kind=w.kind, n_static=d.get("n_static"), n_realtime=d.get("n_realtime"),
-                      n_pos=w.n_pos, n_tbuckets=w.n_tbuckets, ln_eps=w.eps)
+                      n_pos=w.n_pos, n_tbuckets=w.n_tbuckets, ln_eps=w.eps, n_groups=w.n_groups,
+                      token_group=tg)
     fwd = layer.forward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"], d["beta"])
     out = dict(fwd)
     if backward:

@@ -18,7 +18,7 @@ def header_functions():
 
 def test_exports_match_header():
     names = header_functions()
-    assert len(names) == 14, names
+    assert len(names) == 17, names
     assert set(names) == set(capi.EXPORTS)
     for n in names:
         assert hasattr(capi.LIB, n), n

@@ -145,6 +145,54 @@ def test_bf16_backward_small(kind, d):
 
 
 # ----------------------------------------------------------------------------
+# Group LayerNorm (one gamma / beta row per token source)
+# ----------------------------------------------------------------------------
+
+def _check_layer_fwd_bwd(w, f32=False):
+    out, _, _ = run_layer(w, backward=True)
+    y, o, _, _ = oracle.layer_fwd(w)
+    ref = oracle.layer_bwd(w)
+    if f32:
+        assert_f32(out["y"], y, "y")
+        assert_f32(out["o_pre"], o, "o_pre")
+        for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+            assert_f32(out[k], ref[k], k)
+        assert_f32(out["d_gamma"], ref["dgamma"], "d_gamma")
+        assert_f32(out["d_beta"], ref["dbeta"], "d_beta")
+        return
+    sf, sb = storage_fwd(w), storage_bwd(w)
+    assert_bf16(out["y"], y, "y", sf["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", sf["o_pre"])
+    for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+        assert_bf16(out[k], ref[k], k, sb[k])
+    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma", sb["dgamma"])
+    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta", sb["dbeta"])
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_gln_mtgr_forward_backward(d):
+    """MTGR rows with groups profile / behaviour / real-time / candidate from the segments."""
+    w = W.make_mtgr([24, 2, 5], [100, 190, 0], [10, 0, 30], [20, 70, 9], H=2, d=d, seed=21, random_affine=True,
+                    with_grad=True)
+    _check_layer_fwd_bwd(W.with_group_norm(w, seed=22))
+
+
+def test_gln_fp32_random_groups():
+    w = W.make_causal([17, 64, 100, 255], H=2, d=32, dtype=torch.float32, seed=23, alpha=255.0, with_grad=True)
+    _check_layer_fwd_bwd(W.with_group_norm(w, seed=24, groups=3), f32=True)
+
+
+def test_gln_bad_group_flagged():
+    from hstu_jagged_pointwise_b200 import capi
+    w = W.with_group_norm(W.make_causal([40, 9], H=2, d=64, seed=25), seed=26, groups=4)
+    out, layer, d = run_layer(w)
+    layer.token_group[5] = 9                                    # no such group
+    layer.forward(d["q"], d["k"], d["v"], d["u"], d["rab_pos"], d["rab_time"], d["gamma"], d["beta"])
+    assert layer.check_device_error() == capi.HSTU_ERR_DEVICE_BOUNDS
+    assert layer.check_device_error() == capi.HSTU_OK
+
+
+# ----------------------------------------------------------------------------
 # M-FALCON
 # ----------------------------------------------------------------------------
 

@@ -352,6 +352,59 @@ def test_ln_moments_closed_form():
     np.testing.assert_allclose(o.var(1), var / (var + 1e-5), rtol=1e-10)
 
 
+def _gln_case(seed=3, n=41, D=64, G=4):
+    rng = np.random.default_rng(seed)
+    y = rng.normal(size=(n, D)) * 2 + 0.5
+    u = rng.normal(size=(n, D)).astype(np.float32)
+    g = (1 + 0.1 * rng.normal(size=(G, D))).astype(np.float32)
+    b = (0.1 * rng.normal(size=(G, D))).astype(np.float32)
+    grp = rng.integers(0, G - 1, size=n).astype(np.uint8)   # group G-1 has no tokens
+    grad = rng.normal(size=(n, D)).astype(np.float32)
+    return y, u, g, b, grp, grad
+
+
+def test_group_layer_norm_matches_torch_autograd():
+    """Group LayerNorm against float64 torch autograd: F.layer_norm without affine, then the
+    per-token rows gamma[group], beta[group]; the affine gradients come back to their groups."""
+    y, u, g, b, grp, grad = _gln_case()
+    o, mu, rs = oracle.gln_mul_fwd(y, u, g, b, grp, 1e-5)
+    dy, du, dg, db = oracle.gln_mul_bwd(y, u, g, b, grp, grad, 1e-5)
+    ty = torch.tensor(y, requires_grad=True)
+    tu = torch.tensor(u, dtype=torch.float64, requires_grad=True)
+    tg = torch.tensor(g, dtype=torch.float64, requires_grad=True)
+    tb = torch.tensor(b, dtype=torch.float64, requires_grad=True)
+    idx = torch.tensor(grp.astype(np.int64))
+    ref = (torch.nn.functional.layer_norm(ty, (y.shape[1],), eps=1e-5) * tg[idx] + tb[idx]) * tu
+    ref.backward(torch.tensor(grad, dtype=torch.float64))
+    np.testing.assert_allclose(o, ref.detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dy, ty.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(du, tu.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dg, tg.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(db, tb.grad.numpy(), rtol=1e-10, atol=1e-11)
+    assert not dg[-1].any() and not db[-1].any()            # the empty group gets exactly zero
+    np.testing.assert_allclose(mu, y.mean(1), rtol=1e-12)
+
+
+def test_group_layer_norm_with_equal_groups_is_layer_norm():
+    y, u, g, b, grp, grad = _gln_case(seed=4)
+    gs, bs = np.repeat(g[:1], len(g), 0), np.repeat(b[:1], len(b), 0)
+    o, _, _ = oracle.gln_mul_fwd(y, u, gs, bs, grp, 1e-5)
+    o1, _, _ = oracle.ln_mul_fwd(y, u, g[0], b[0], 1e-5)
+    np.testing.assert_allclose(o, o1, rtol=1e-13, atol=1e-13)
+    dy, du, dg, db = oracle.gln_mul_bwd(y, u, gs, bs, grp, grad, 1e-5)
+    dy1, du1, dg1, db1 = oracle.ln_mul_bwd(y, u, g[0], b[0], grad, 1e-5)
+    np.testing.assert_allclose(dy, dy1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(du, du1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dg.sum(0), dg1, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(db.sum(0), db1, rtol=1e-11, atol=1e-12)
+
+
+def test_mtgr_token_groups_follow_segments():
+    w = W.with_group_norm(W.make_mtgr([3, 2], [5, 0], [2, 4], [3, 1], H=1, d=32, dtype=torch.float32, seed=5))
+    np.testing.assert_array_equal(w.token_group, [0, 0, 0, 1, 1, 1, 1, 1, 2, 2, 3, 3, 3, 0, 0, 2, 2, 2, 2, 3])
+    assert w.gamma.shape == (4, 32) and w.n_groups == 4
+
+
 # ----------------------------------------------------------------------------
 # backward: central finite differences with Richardson extrapolation
 # ----------------------------------------------------------------------------
