@@ -363,6 +363,8 @@ def run_ours(args, world, rank, local):
     extra = {}
     if not args.no_gln:
         extra["gln"] = run_gln(args, world, w, dv, off, ts, rp, rt, fwd_out, bwd_out)
+    if not args.no_proj:
+        extra["projections"] = run_proj(args, world, rank)
 
     # ---- end to end through the C ABI with host buffers
     if args.no_e2e:
@@ -411,6 +413,81 @@ def run_ours(args, world, rank, local):
         mf = run_mfalcon(args, world, rank, local)
     return finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, clocks, f_fwd, f_bwd, P, d,
                   extra)
+
+
+def run_proj(args, world, rank):
+    """f1 (X -> U, V, Q, K with SiLU) and f2 of the large layer (262,144 tokens, d_model 1024),
+    forward and backward, on the library's tcgen05 GEMM; the same products through
+    torch.matmul (cuBLAS) are timed beside it for reference."""
+    from hstu_jagged_pointwise_b200 import capi, ops
+    dev = f"cuda:{torch.cuda.current_device()}"
+    if args.tokens == 262144:
+        w = W.projection_large(seed=args.seed + rank, device=dev)
+    else:
+        w = W.make_projection(args.tokens, 1024, 1024, 1024, seed=args.seed + rank, device=dev,
+                              name=f"proj_T{args.tokens}_d1024")
+    T, d_in, D, d_out = w.T, w.d_in, w.D, w.d_out
+    blocks = [w.dact[:, i * D:(i + 1) * D].contiguous() for i in range(4)]
+    outs = {}
+
+    def step():
+        outs["f1"] = ops.f1_fwd(w.x, w.w1, w.b1, D, out=outs.get("f1"))
+        outs["f2"] = ops.f2_fwd(w.o_pre, w.w2, w.b2, residual=w.x, out=outs.get("f2"))
+        outs["b1"] = ops.f1_bwd(w.x, w.w1, w.z, *blocks, out=outs.get("b1"))
+        outs["b2"] = ops.f2_bwd(w.o_pre, w.w2, w.g_out, out=outs.get("b2"))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    capi.profile_enable(True)
+    e0.record(s)
+    for _ in range(args.steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    prof = capi.profile_read()
+    capi.profile_enable(False)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    for o in outs.values():
+        if int(o["status"].item()) != 0:
+            raise RuntimeError("device status set in the projections")
+    flops = 2 * T * (d_in * 4 * D + D * d_out) * 3            # forward + two backward products each
+    n_g, t_g = prof["gemm_tc_kernel"]
+    pk, _ = peaks()
+    gemm_tf = flops / (t_g / args.steps * 1e-3) / 1e12
+
+    # the same eight products through cuBLAS (torch.matmul), timed alone
+    z4 = torch.empty(T, 4 * D, dtype=torch.bfloat16, device=w.x.device)
+    dzb = torch.empty_like(z4)
+
+    def lib_step():
+        torch.matmul(w.x, w.w1.t(), out=z4)
+        torch.matmul(w.o_pre, w.w2.t())
+        torch.matmul(dzb, w.w1)
+        torch.matmul(dzb.t(), w.x)
+        torch.matmul(w.g_out, w.w2)
+        torch.matmul(w.g_out.t(), w.o_pre)
+
+    for _ in range(args.warmup):
+        lib_step()
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(args.steps):
+        lib_step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms_lib = e0.elapsed_time(e1) / args.steps
+    return {"workload": w.name, "ms_per_step": round(ms, 4), "gemm_launches_per_step": n_g // args.steps,
+            "gemm_ms_per_step": round(t_g / args.steps, 4), "gemm_tflops": round(gemm_tf, 1),
+            "frac_bf16_sustained": round(gemm_tf / pk["bf16_tflops_sustained"], 4),
+            "frac_bf16_burst": round(gemm_tf / pk["bf16_tflops"], 4),
+            "other_kernels_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in prof.items()
+                                          if k != "gemm_tc_kernel"},
+            "cublas_same_products_ms": round(ms_lib, 4),
+            "cublas_tflops": round(flops / (ms_lib * 1e-3) / 1e12, 1)}
 
 
 def run_gln(args, world, w, dv, off, ts, rp, rt, fwd_out, bwd_out):
@@ -677,10 +754,13 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-mfalcon", action="store_true")
     ap.add_argument("--no-gln", action="store_true", help="skip the Group LayerNorm variant")
+    ap.add_argument("--no-proj", action="store_true", help="skip the f1 / f2 projections")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--tokens", type=int, default=262144,
                     help="total tokens of the large-layer workload (smaller values for profiling)")
+    ap.add_argument("--only-proj", action="store_true",
+                    help="run only the f1 / f2 projections leg and print its JSON (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -690,6 +770,12 @@ def main():
         line = run_reference(args, world, rank)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return
+    if args.only_proj:
+        torch.cuda.set_device(local)
+        line = run_proj(args, world, rank)
+        if rank == 0:
+            print(json.dumps({"projections": line}), flush=True)
         return
     line, w = run_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -31,7 +31,8 @@ EXPORTS = (
     "hstu_mfalcon_score", "hstu_debug_indices", "hstu_check_device_error", "hstu_status_string",
     "hstu_version", "hstu_profile_enable", "hstu_profile_read", "hstu_profile_kind_name",
     "hstu_attn_fwd_noalloc", "hstu_mfalcon_cache_history", "hstu_attn_fwd_gln", "hstu_attn_bwd_gln",
-    "hstu_attn_workspace_bytes_gln",
+    "hstu_attn_workspace_bytes_gln", "hstu_f1_fwd", "hstu_f2_fwd", "hstu_f1_bwd_workspace_bytes",
+    "hstu_f2_bwd_workspace_bytes", "hstu_f1_bwd", "hstu_f2_bwd",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20   # HSTU_NOALLOC_SCRATCH_BYTES
@@ -95,6 +96,18 @@ def load():
     lib.hstu_mfalcon_score.restype = C.c_int
     lib.hstu_mfalcon_cache_history.argtypes = [i32, i32, i32, i32, P, P, P, P, P, C.c_int64, P, P, P, P, P, P]
     lib.hstu_mfalcon_cache_history.restype = C.c_int
+    lib.hstu_f1_fwd.argtypes = [i32, i32, i32] + [P] * 10
+    lib.hstu_f1_fwd.restype = C.c_int
+    lib.hstu_f2_fwd.argtypes = [i32, i32, i32] + [P] * 7
+    lib.hstu_f2_fwd.restype = C.c_int
+    lib.hstu_f1_bwd_workspace_bytes.argtypes = [i32, i32]
+    lib.hstu_f1_bwd_workspace_bytes.restype = S
+    lib.hstu_f2_bwd_workspace_bytes.argtypes = [i32, i32]
+    lib.hstu_f2_bwd_workspace_bytes.restype = S
+    lib.hstu_f1_bwd.argtypes = [i32, i32, i32] + [P] * 11 + [S, P, P]
+    lib.hstu_f1_bwd.restype = C.c_int
+    lib.hstu_f2_bwd.argtypes = [i32, i32, i32] + [P] * 7 + [S, P, P]
+    lib.hstu_f2_bwd.restype = C.c_int
     lib.hstu_debug_indices.argtypes = [i32, i32, P, P, P, P, i32, i32, P, P, P, P, P]
     lib.hstu_debug_indices.restype = C.c_int
     lib.hstu_check_device_error.argtypes = [P, P]

@@ -230,6 +230,32 @@ SimtParams simt_params(const hstu_dims& d, int kind, const hstu_mask_spec& m, co
 }  // namespace
 }  // namespace hstu
 
+namespace hstu {
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+    return make_tmap(m, base, rows, cols, box_rows);
+}
+
+bool make_tmap_f32_sw128(CUtensorMap* m, void* base, long long rows, long long cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int device_sms() {
+    const DevInfo* di = dev_info();
+    return di ? di->sms : 0;
+}
+
+}  // namespace hstu
+
 using namespace hstu;
 
 extern "C" {

@@ -144,11 +144,46 @@ constexpr int kLnMaxGroups = 16;
 constexpr int kGlnMaxBlocks = 148 * 16;   // grouped LayerNorm blocks (each a contiguous chunk of rows)
 constexpr int kLnMaxGroupCols = 16384;   // G * D: bound on the [G][D] affine tables
 
+// ---- dense projections (proj_gemm.cu, proj_api.cu)
+enum GemmEpi { kEpiF1 = 0, kEpiF2 = 1, kEpiBf16 = 2, kEpiAddF32 = 3 };
+
+struct GemmParams {
+    int M, N, K;
+    int k_splits;                       // K split over this many tiles (kEpiAddF32 only)
+    const float* bias;                  // [N] or nullptr
+    const __nv_bfloat16* residual;      // [M, N] or nullptr (kEpiF2)
+    void* out;                          // [M, N]: bf16, or fp32 for kEpiAddF32
+    __nv_bfloat16* out4[4];             // kEpiF1: U, V, Q, K, each [M, D]
+    __nv_bfloat16* z;                   // kEpiF1: pre-activation [M, N] or nullptr
+    int D;                              // kEpiF1: width of each output block
+    int* status;                        // kStatusTimeout is OR-ed here, or nullptr
+};
+
+// Output tensor maps of the epilogue: out[0..3] (kEpiF1: U, V, Q, K; otherwise out[0] only)
+// and z (kEpiF1 pre-activation), each stored from 32-row boxes.
+struct GemmOutMaps {
+    CUtensorMap out[4];
+    CUtensorMap z;
+};
+constexpr int kGemmStoreRows = 32;
+
+cudaError_t launch_gemm_tc(bool a_mn, bool b_mn, int epi, const CUtensorMap& ta, const CUtensorMap& tb,
+                           const GemmOutMaps& to, const GemmParams& p, int grid, cudaStream_t s);
+int gemm_tiles(const GemmParams& p);
+int gemm_k_steps(int K);
+int gemm_box_rows(bool mn_major, bool is_b);
+
+// [rows, cols] bf16 row-major, 128-byte swizzle, box = 64 columns x box_rows rows
+bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows);
+// [rows, cols] fp32 row-major, 128-byte swizzle, box = 32 columns x box_rows rows
+bool make_tmap_f32_sw128(CUtensorMap* m, void* base, long long rows, long long cols, int box_rows);
+int device_sms();
+
 // ---- opt-in per-kernel timing (profile.cu)
 enum ProfKind {
     kProfSchedule = 0, kProfAttnFwdTc, kProfAttnFwdSimt, kProfLnFwd, kProfLnBwd, kProfLnBwdReduce,
     kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfDqConvert,
-    kProfRabReduce, kProfCacheScan, kProfCacheCopy, kProfKinds
+    kProfRabReduce, kProfCacheScan, kProfCacheCopy, kProfGemm, kProfSiluGrad, kProfColSum, kProfKinds
 };
 void prof_begin(int kind, cudaStream_t s);
 void prof_end(int kind, cudaStream_t s);

@@ -200,6 +200,76 @@ class MFalcon:
         return int(capi.LIB.hstu_check_device_error(_p(self.ws), _stream()))
 
 
+# ----------------------------------------------------------------------------
+# the projections around the attention: f1 (X -> U, V, Q, K with SiLU) and f2
+# ----------------------------------------------------------------------------
+
+def _status(dev):
+    return torch.zeros(1, dtype=torch.int32, device=dev)
+
+
+def f1_fwd(x, w1, b1, D: int, save_z: bool = True, out: Optional[dict] = None) -> dict:
+    """U, V, Q, K = split(SiLU(x @ w1.T + b1)), each [T, D]; z (pre-activation) kept for
+    the backward when save_z.  w1 is [4D, d_in]; b1 fp32 [4D] or None."""
+    _need(x, "x", torch.bfloat16)
+    _need(w1, "w1", torch.bfloat16)
+    T, d_in = x.shape
+    if out is None:
+        out = {n: torch.empty(T, D, dtype=torch.bfloat16, device=x.device) for n in ("u", "v", "q", "k")}
+        out["z"] = torch.empty(T, 4 * D, dtype=torch.bfloat16, device=x.device) if save_z else None
+        out["status"] = _status(x.device)
+    st = capi.LIB.hstu_f1_fwd(T, d_in, D, _p(x), _p(w1), _p(b1), _p(out["u"]), _p(out["v"]), _p(out["q"]),
+                              _p(out["k"]), _p(out.get("z")), _p(out.get("status")), _stream())
+    capi.check(st, "hstu_f1_fwd")
+    return out
+
+
+def f2_fwd(o_pre, w2, b2=None, residual=None, out: Optional[dict] = None) -> dict:
+    """out = o_pre @ w2.T + b2 (+ residual); w2 is [d_out, D]."""
+    _need(o_pre, "o_pre", torch.bfloat16)
+    _need(w2, "w2", torch.bfloat16)
+    T, D = o_pre.shape
+    d_out = w2.shape[0]
+    if out is None:
+        out = dict(out=torch.empty(T, d_out, dtype=torch.bfloat16, device=o_pre.device),
+                   status=_status(o_pre.device))
+    st = capi.LIB.hstu_f2_fwd(T, D, d_out, _p(o_pre), _p(w2), _p(b2), _p(residual), _p(out["out"]),
+                              _p(out.get("status")), _stream())
+    capi.check(st, "hstu_f2_fwd")
+    return out
+
+
+def f1_bwd(x, w1, z, du, dv, dq, dk, out: Optional[dict] = None) -> dict:
+    """dx [T, d_in] (bf16), dw1 [4D, d_in] and db1 [4D] (fp32) of f1 for the U, V, Q, K gradients."""
+    T, d_in = x.shape
+    D = du.shape[1]
+    if out is None:
+        n = capi.LIB.hstu_f1_bwd_workspace_bytes(T, D)
+        out = dict(dx=torch.empty_like(x), dw1=torch.empty(4 * D, d_in, dtype=torch.float32, device=x.device),
+                   db1=torch.empty(4 * D, dtype=torch.float32, device=x.device), ws=workspace(n, x.device),
+                   status=_status(x.device))
+    st = capi.LIB.hstu_f1_bwd(T, d_in, D, _p(x), _p(w1), _p(z), _p(du), _p(dv), _p(dq), _p(dk), _p(out["dx"]),
+                              _p(out["dw1"]), _p(out["db1"]), _p(out["ws"]), out["ws"].numel(),
+                              _p(out.get("status")), _stream())
+    capi.check(st, "hstu_f1_bwd")
+    return out
+
+
+def f2_bwd(o_pre, w2, g, out: Optional[dict] = None) -> dict:
+    """d_o_pre [T, D] (bf16), dw2 [d_out, D] and db2 [d_out] (fp32) of f2 for g = dL/d out."""
+    T, D = o_pre.shape
+    d_out = w2.shape[0]
+    if out is None:
+        n = capi.LIB.hstu_f2_bwd_workspace_bytes(T, d_out)
+        out = dict(d_o_pre=torch.empty_like(o_pre), dw2=torch.empty(d_out, D, dtype=torch.float32, device=g.device),
+                   db2=torch.empty(d_out, dtype=torch.float32, device=g.device), ws=workspace(n, g.device),
+                   status=_status(g.device))
+    st = capi.LIB.hstu_f2_bwd(T, D, d_out, _p(o_pre), _p(w2), _p(g), _p(out["d_o_pre"]), _p(out["dw2"]),
+                              _p(out["db2"]), _p(out["ws"]), out["ws"].numel(), _p(out.get("status")), _stream())
+    capi.check(st, "hstu_f2_bwd")
+    return out
+
+
 def mfalcon_cache_history(seq_offsets, timestamps, n_history, k, v, hist_rows: Optional[int] = None,
                           out: Optional[dict] = None) -> dict:
     """KV cache for MFalcon.score from a full-sequence M-FALCON batch: the first

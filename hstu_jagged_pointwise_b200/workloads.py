@@ -128,7 +128,7 @@ def increasing_ts(rng: np.random.Generator, n: int, start: int = T0) -> np.ndarr
 
 
 def randn(gen: torch.Generator, shape, dtype: torch.dtype, std: float = 1.0) -> torch.Tensor:
-    x = torch.randn(*shape, generator=gen, dtype=torch.float32)
+    x = torch.randn(*shape, generator=gen, dtype=torch.float32, device=gen.device)
     if std != 1.0:
         x.mul_(std)
     return x.to(dtype)
@@ -355,6 +355,49 @@ def mfalcon_seq_from(w: Workload, seed: int = 0, name: str = "mfalcon_seq") -> W
                     offsets=_offsets(n_hist + n_cand).astype(np.int32), ts=ts.astype(np.int64),
                     q=cat(hq, w.cand_q), k=cat(w.hist_k, w.cand_k), v=cat(w.hist_v, w.cand_v),
                     u=cat(hu, w.cand_u), n_realtime=n_hist.astype(np.int32))
+
+
+# ----------------------------------------------------------------------------
+# the projections around the attention
+# ----------------------------------------------------------------------------
+
+@dataclass
+class ProjWorkload:
+    """Inputs of f1 (X -> U, V, Q, K) and f2 (O_pre -> out) and their upstream gradients.
+    Weights are [out, in] with N(0, 1/fan_in) entries, so Z and out stay O(1); biases
+    N(0, 0.1); activations and gradients N(0, 1); the residual is X (d_out = d_in)."""
+    T: int
+    d_in: int
+    D: int
+    d_out: int
+    x: torch.Tensor          # [T, d_in]
+    w1: torch.Tensor         # [4D, d_in]
+    b1: torch.Tensor         # [4D] fp32
+    o_pre: torch.Tensor      # [T, D]
+    w2: torch.Tensor         # [d_out, D]
+    b2: torch.Tensor         # [d_out] fp32
+    dact: torch.Tensor       # [T, 4D]: gradients of U, V, Q, K side by side
+    g_out: torch.Tensor      # [T, d_out]
+    z: torch.Tensor          # [T, 4D]: a pre-activation input for the f1 backward
+    name: str = "proj"
+
+
+def make_projection(T: int, d_in: int, D: int, d_out: Optional[int] = None, seed: int = 0,
+                    device: str = "cpu", dtype=torch.bfloat16, name: str = "proj") -> ProjWorkload:
+    d_out = d_in if d_out is None else d_out
+    gen = torch.Generator(device=device).manual_seed(seed + 606)
+    return ProjWorkload(
+        T=T, d_in=d_in, D=D, d_out=d_out,
+        x=randn(gen, (T, d_in), dtype), w1=randn(gen, (4 * D, d_in), dtype, d_in ** -0.5),
+        b1=randn(gen, (4 * D,), torch.float32, 0.1), o_pre=randn(gen, (T, D), dtype),
+        w2=randn(gen, (d_out, D), dtype, D ** -0.5), b2=randn(gen, (d_out,), torch.float32, 0.1),
+        dact=randn(gen, (T, 4 * D), dtype), g_out=randn(gen, (T, d_out), dtype),
+        z=randn(gen, (T, 4 * D), dtype, 2.0), name=name)
+
+
+def projection_large(seed: int = 0, device: str = "cpu") -> ProjWorkload:
+    """The large layer's projections: 262,144 tokens, d_model 1024 = 8 heads x 128."""
+    return make_projection(262144, 1024, 1024, 1024, seed=seed, device=device, name="proj_T262144_d1024")
 
 
 # ----------------------------------------------------------------------------

@@ -295,6 +295,54 @@ HSTU_API int hstu_mfalcon_cache_history(int32_t B, int32_t T, int32_t row_elems,
                        int32_t* hist_offsets, int64_t* hist_ts, void* hist_k, void* hist_v,
                        int32_t* device_status, void* stream);
 
+/* ---- The projections on either side of the attention (Meta HSTU blog, section 3
+ * formula: U(X), V(X), Q(X), K(X) = Split(phi1(f1(X))), phi1 = SiLU, and
+ * O(X) = f2(Norm(A(X)V(X)) (.) U(X))).  f1 and f2 are linear maps with weights
+ * stored [out, in] row-major (bf16) and optional fp32 biases; activations are
+ * bf16 row-major, accumulation fp32 on the tensor cores.
+ * device_status (optional DEVICE int32, NULL to skip) is set to 0 on `stream`,
+ * then gets bit 2 if a bounded wait in the GEMM ran out (outputs then
+ * incomplete).  Argument errors return before any launch:
+ * HSTU_ERR_INVALID_ARG for sizes out of range or missing / misaligned pointers
+ * (16 bytes for tensors and biases, 4 for device_status), HSTU_ERR_UNSUPPORTED
+ * for widths off the multiples stated below. */
+
+/* Z = X W1^T + b1 (X [T, d_in], W1 [4D, d_in], b1 [4D] or NULL);
+ * U, V, Q, K = SiLU(Z) column blocks [0, D), [D, 2D), [2D, 3D), [3D, 4D), each
+ * written to its own [T, D] tensor (the attention's input layout).  z (NULL to
+ * skip) receives Z [T, 4D] for the backward.  d_in a multiple of 8, D of 64. */
+HSTU_API int hstu_f1_fwd(int32_t T, int32_t d_in, int32_t D, const void* x, const void* w1, const float* b1,
+                  void* u, void* v, void* q, void* k, void* z, int32_t* device_status, void* stream);
+
+/* out = O_pre W2^T + b2 (+ residual): O_pre [T, D], W2 [d_out, D], b2 [d_out] or
+ * NULL, residual [T, d_out] or NULL (added when given, e.g. the layer input
+ * of a residual stack), out [T, d_out].  D a multiple of 8, d_out of 32. */
+HSTU_API int hstu_f2_fwd(int32_t T, int32_t D, int32_t d_out, const void* o_pre, const void* w2,
+                  const float* b2, const void* residual, void* out, int32_t* device_status, void* stream);
+
+/* Workspace bytes of hstu_f1_bwd / hstu_f2_bwd; 0 for invalid sizes. */
+HSTU_API size_t hstu_f1_bwd_workspace_bytes(int32_t T, int32_t D);
+HSTU_API size_t hstu_f2_bwd_workspace_bytes(int32_t T, int32_t d_out);
+
+/* Backward of hstu_f1_fwd for the U, V, Q, K gradients du, dv, dq, dk [T, D]
+ * (z = the forward's Z).  dZ = dAct * SiLU'(Z) is kept in bf16 in the
+ * workspace; dx = dZ W1 [T, d_in] (bf16); dw1 = dZ^T X [4D, d_in] and
+ * db1 = column sums of the stored dZ [4D] in fp32, overwritten.  dw1 sums split-K tiles
+ * with atomics (last-bit order effects); db1 is deterministic.  d_in and D
+ * multiples of 32, 4D <= 8192. */
+HSTU_API int hstu_f1_bwd(int32_t T, int32_t d_in, int32_t D, const void* x, const void* w1, const void* z,
+                  const void* du, const void* dv, const void* dq, const void* dk,
+                  void* dx, float* dw1, float* db1, void* workspace, size_t workspace_bytes,
+                  int32_t* device_status, void* stream);
+
+/* Backward of hstu_f2_fwd for d_out_grad = dL/d out [T, d_out]: d_o_pre =
+ * d_out_grad W2 [T, D] (bf16); dw2 = d_out_grad^T O_pre [d_out, D] and db2
+ * [d_out] in fp32, overwritten (dw2 with split-K atomics, db2 deterministic).
+ * The residual's gradient is d_out_grad itself.  D and d_out multiples of 32. */
+HSTU_API int hstu_f2_bwd(int32_t T, int32_t D, int32_t d_out, const void* o_pre, const void* w2,
+                  const void* d_out_grad, void* d_o_pre, float* dw2, float* db2,
+                  void* workspace, size_t workspace_bytes, int32_t* device_status, void* stream);
+
 /* Integer decisions of the fused kernels, written through the same device
  * functions they use, for exact comparison in tests.  For every sequence b and
  * pair (i, j) of it, entry pair_offsets[b] + i*L_b + j (pair_offsets: device

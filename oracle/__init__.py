@@ -286,6 +286,57 @@ def norm_bwd(w, y, grad):
     return ln_mul_bwd(y, w.u, w.gamma, w.beta, grad, w.eps)
 
 
+# ----------------------------------------------------------------------------
+# the projections around the attention (Meta HSTU blog, section 3 formula):
+# U, V, Q, K = Split(phi1(f1(X))) with phi1 = SiLU, O = f2(Norm(A V) * U)
+# ----------------------------------------------------------------------------
+
+def _as_f64(a):
+    """float64 view of an input: bf16/fp32 tensors and arrays exactly, float64 arrays as they are."""
+    if isinstance(a, np.ndarray) and a.dtype == np.float64:
+        return a
+    return np.asarray(f32(a), dtype=np.float64)
+
+
+def sigmoid(z):
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def f1_fwd(x, w1, b1, D):
+    """Z = X W1^T + b1 in float64 (W1 stored [4D, d_in]); returns Z and the four column
+    blocks of SiLU(Z) in the order U, V, Q, K."""
+    z = _as_f64(x) @ _as_f64(w1).T
+    if b1 is not None:
+        z = z + _as_f64(b1)
+    a = z * sigmoid(z)
+    return z, a[:, :D], a[:, D:2 * D], a[:, 2 * D:3 * D], a[:, 3 * D:]
+
+
+def f2_fwd(o_pre, w2, b2=None, residual=None):
+    """out = O_pre W2^T + b2 (+ residual), float64 (W2 stored [d_out, D])."""
+    o = _as_f64(o_pre) @ _as_f64(w2).T
+    if b2 is not None:
+        o = o + _as_f64(b2)
+    if residual is not None:
+        o = o + _as_f64(residual)
+    return o
+
+
+def f1_bwd(x, w1, z, du, dv, dq, dk):
+    """dZ = [dU dV dQ dK] * SiLU'(Z), SiLU'(z) = s (1 + z (1 - s)); dX = dZ W1, dW1 = dZ^T X,
+    db1 = column sums of dZ.  Returns (dz, dx, dw1, db1)."""
+    z = _as_f64(z)
+    s = sigmoid(z)
+    dz = np.concatenate([_as_f64(du), _as_f64(dv), _as_f64(dq), _as_f64(dk)], axis=1) * s * (1 + z * (1 - s))
+    return dz, dz @ _as_f64(w1), dz.T @ _as_f64(x), dz.sum(0)
+
+
+def f2_bwd(o_pre, w2, g):
+    """d_O_pre = G W2, dW2 = G^T O_pre, db2 = column sums of G for G = dL/d out."""
+    g = _as_f64(g)
+    return g @ _as_f64(w2), g.T @ _as_f64(o_pre), g.sum(0)
+
+
 def layer_fwd(w, rows=None):
     """(y, o_pre, mean, rstd) for the listed rows: attention, then Norm(y) * u."""
     y = attn_fwd(w, rows)

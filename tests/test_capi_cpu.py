@@ -18,7 +18,7 @@ def header_functions():
 
 def test_exports_match_header():
     names = header_functions()
-    assert len(names) == 17, names
+    assert len(names) == 23, names
     assert set(names) == set(capi.EXPORTS)
     for n in names:
         assert hasattr(capi.LIB, n), n
@@ -123,6 +123,25 @@ def test_cache_producer_rejects_bad_arguments_before_launch():
     assert f(1, 4, 64, capi.HSTU_BF16, *ok, 4, a, a, a, a, None, None) == capi.HSTU_ERR_INVALID_ARG  # no status
     assert f(1, 4, 64, capi.HSTU_BF16, a, a, a, a + 8, a, 4, *outs, None) == capi.HSTU_ERR_INVALID_ARG  # k misaligned
     assert f(1, 4, 64, capi.HSTU_BF16, a, a, a, a, a, -1, *outs, None) == capi.HSTU_ERR_INVALID_ARG
+
+
+def test_projections_reject_bad_arguments_before_launch():
+    buf = (C.c_uint8 * 4096)()
+    a = (C.addressof(buf) + 255) // 256 * 256          # 256-byte aligned host address (never dereferenced)
+    f1 = capi.LIB.hstu_f1_fwd
+    assert f1(-1, 64, 64, *([a] * 10), None) == capi.HSTU_ERR_INVALID_ARG
+    assert f1(4, 60, 64, *([a] * 10), None) == capi.HSTU_ERR_UNSUPPORTED       # d_in not a multiple of 8
+    assert f1(4, 64, 96, *([a] * 10), None) == capi.HSTU_ERR_UNSUPPORTED       # D not a multiple of 64
+    assert f1(4, 64, 64, a, a, a + 8, *([a] * 7), None) == capi.HSTU_ERR_INVALID_ARG   # misaligned bias
+    assert f1(4, 64, 64, None, *([a] * 7), None, None, None) == capi.HSTU_ERR_INVALID_ARG  # no x
+    f2 = capi.LIB.hstu_f2_fwd
+    assert f2(4, 64, 48, *([a] * 7)) == capi.HSTU_ERR_UNSUPPORTED             # d_out not a multiple of 32
+    assert capi.LIB.hstu_f1_bwd_workspace_bytes(4, 48) == 0
+    assert capi.LIB.hstu_f1_bwd_workspace_bytes(4, 4096) == 0                 # 4D above 8192
+    assert capi.LIB.hstu_f1_bwd_workspace_bytes(4, 64) > 0
+    assert capi.LIB.hstu_f2_bwd_workspace_bytes(4, 64) > 0
+    assert capi.LIB.hstu_f1_bwd(4, 64, 64, *([a] * 11), 16, None, None) == capi.HSTU_ERR_WORKSPACE
+    assert capi.LIB.hstu_f2_bwd(4, 64, 64, *([a] * 7), 16, None, None) == capi.HSTU_ERR_WORKSPACE
 
 
 def test_mfalcon_rejects_bad_arguments():

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from hstu_jagged_pointwise_b200 import workloads as W
-from parity import (assert_bf16, assert_f32, errors, run_layer, run_mfalcon, storage_bwd, storage_fwd,
+from parity import (assert_bf16, assert_f32, bf16, errors, run_layer, run_mfalcon, storage_bwd, storage_fwd,
                     storage_mfalcon)
 
 pytestmark = pytest.mark.gpu
@@ -337,6 +337,105 @@ def test_mfalcon_ranking_full_sequence_sampled_rows():
         rt = torch.as_tensor(rows + s0).cuda()
         assert_bf16(out["y"][rt], y, f"y[user {b}]", st["y"])
         assert_bf16(out["o_pre"][rt], o, f"o_pre[user {b}]", st["o_pre"])
+
+
+# ----------------------------------------------------------------------------
+# projections: f1 (X -> U, V, Q, K with SiLU) and f2, forward and backward
+# ----------------------------------------------------------------------------
+
+def _bf(a):
+    return torch.as_tensor(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def _status_ok(out):
+    assert int(out["status"].item()) == 0
+
+
+def test_projections_small_forward_backward():
+    """Tails everywhere: T = 300 rows (2.3 row tiles), d_in = 224 (K tail of 32, and a partial
+    column tile for dX), d_out = 224 (a partial column tile and half a stored chunk)."""
+    from hstu_jagged_pointwise_b200 import ops
+    w = W.make_projection(300, 224, 64, 224, seed=31)
+    c = {n: getattr(w, n).cuda() for n in ("x", "w1", "b1", "o_pre", "w2", "b2", "g_out")}
+    D = w.D
+    f = ops.f1_fwd(c["x"], c["w1"], c["b1"], D)
+    torch.cuda.synchronize()
+    _status_ok(f)
+    z, u, v, q, k = oracle.f1_fwd(w.x, w.w1, w.b1, D)
+    for name, ref in (("z", z), ("u", u), ("v", v), ("q", q), ("k", k)):
+        assert_bf16(f[name], ref, name, bf16(ref))
+    o = ops.f2_fwd(c["o_pre"], c["w2"], c["b2"], residual=c["x"])
+    torch.cuda.synchronize()
+    _status_ok(o)
+    ref = oracle.f2_fwd(w.o_pre, w.w2, w.b2, w.x)
+    assert_bf16(o["out"], ref, "out", bf16(ref))
+    # backward of f1 from the oracle's Z (rounded to the bf16 the layer stores)
+    zb = _bf(z)
+    dact = w.dact
+    blocks = [dact[:, i * D:(i + 1) * D].contiguous() for i in range(4)]
+    b = ops.f1_bwd(c["x"], c["w1"], zb.cuda(), *[t.cuda() for t in blocks])
+    torch.cuda.synchronize()
+    _status_ok(b)
+    dz, dx, dw1, db1 = oracle.f1_bwd(w.x, w.w1, zb, *blocks)
+    dzb = bf16(dz)                                          # the kernel keeps dZ in bf16
+    assert_bf16(b["dx"], dx, "dx", bf16(dzb @ oracle.f32(w.w1).astype(np.float64)))
+    assert_bf16(b["dw1"], dw1, "dw1", dzb.T @ oracle.f32(w.x).astype(np.float64))
+    assert_bf16(b["db1"], db1, "db1", dzb.sum(0))
+    g = ops.f2_bwd(c["o_pre"], c["w2"], c["g_out"])
+    torch.cuda.synchronize()
+    _status_ok(g)
+    do, dw2, db2 = oracle.f2_bwd(w.o_pre, w.w2, w.g_out)
+    assert_bf16(g["d_o_pre"], do, "d_o_pre", bf16(do))
+    assert_bf16(g["dw2"], dw2, "dw2")
+    assert_bf16(g["db2"], db2, "db2")
+
+
+def test_projections_large_sampled():
+    """The large layer's projections (262,144 tokens, d_model 1024) in the bench's launch
+    configuration: sampled rows of every row-wise output, sampled entries of the weight
+    gradients and bias gradients (each a sum over all tokens)."""
+    from hstu_jagged_pointwise_b200 import ops
+    w = W.projection_large(seed=0, device="cuda")
+    D = w.D
+    f = ops.f1_fwd(w.x, w.w1, w.b1, D)
+    o = ops.f2_fwd(w.o_pre, w.w2, w.b2, residual=w.x)
+    blocks = [w.dact[:, i * D:(i + 1) * D].contiguous() for i in range(4)]
+    b = ops.f1_bwd(w.x, w.w1, w.z, *blocks)
+    g = ops.f2_bwd(w.o_pre, w.w2, w.g_out)
+    torch.cuda.synchronize()
+    for out in (f, o, b, g):
+        _status_ok(out)
+    rng = np.random.default_rng(9)
+    rows = np.unique(np.concatenate([rng.integers(0, w.T, 40), [0, w.T - 1]]))
+    rt = torch.as_tensor(rows).cuda()
+    cpu = lambda t: t[rt].cpu()
+    z, u, v, q, k = oracle.f1_fwd(cpu(w.x), w.w1.cpu(), w.b1.cpu(), D)
+    for name, ref in (("z", z), ("u", u), ("v", v), ("q", q), ("k", k)):
+        assert_bf16(f[name][rt], ref, name, bf16(ref))
+    ref = oracle.f2_fwd(cpu(w.o_pre), w.w2.cpu(), w.b2.cpu(), cpu(w.x))
+    assert_bf16(o["out"][rt], ref, "out", bf16(ref))
+    dz, dx, _, _ = oracle.f1_bwd(cpu(w.x), w.w1.cpu(), cpu(w.z), *[cpu(t) for t in blocks])
+    assert_bf16(b["dx"][rt], dx, "dx", bf16(bf16(dz) @ oracle.f32(w.w1.cpu()).astype(np.float64)))
+    do, _, _ = oracle.f2_bwd(cpu(w.o_pre), w.w2.cpu(), cpu(w.g_out))
+    assert_bf16(g["d_o_pre"][rt], do, "d_o_pre", bf16(do))
+    # weight and bias gradients: sampled columns, sums over all 262,144 tokens
+    ci = np.array([0, 5, 1023, 1024, 2047, 3000, 4095])          # output columns of f1 (all four blocks)
+    cj = np.array([0, 17, 511, 1023])                             # input columns
+    zc = w.z[:, torch.as_tensor(ci).cuda()].cpu()
+    dc = w.dact[:, torch.as_tensor(ci).cuda()].cpu()
+    empty = torch.zeros(w.T, 0, dtype=torch.bfloat16)
+    xs = w.x[:, torch.as_tensor(cj).cuda()].cpu()
+    dz_c, _, dw1_c, db1_c = oracle.f1_bwd(xs, torch.zeros(len(ci), len(cj), dtype=torch.bfloat16), zc, dc, empty,
+                                          empty, empty)
+    got_w1 = b["dw1"][torch.as_tensor(ci).cuda()][:, torch.as_tensor(cj).cuda()]
+    assert_bf16(got_w1, dw1_c, "dw1 (sampled)", bf16(dz_c).T @ oracle.f32(xs).astype(np.float64))
+    assert_bf16(b["db1"][torch.as_tensor(ci).cuda()], db1_c, "db1 (sampled)", bf16(dz_c).sum(0))
+    oi = np.array([0, 300, 1023])
+    gs = w.g_out[:, torch.as_tensor(oi).cuda()].cpu()
+    os_ = w.o_pre[:, torch.as_tensor(cj).cuda()].cpu()
+    _, dw2_c, db2_c = oracle.f2_bwd(os_, torch.zeros(len(oi), len(cj), dtype=torch.bfloat16), gs)
+    assert_bf16(g["dw2"][torch.as_tensor(oi).cuda()][:, torch.as_tensor(cj).cuda()], dw2_c, "dw2 (sampled)")
+    assert_bf16(g["db2"][torch.as_tensor(oi).cuda()], db2_c, "db2 (sampled)")
 
 
 # ----------------------------------------------------------------------------

@@ -406,6 +406,63 @@ def test_mtgr_token_groups_follow_segments():
 
 
 # ----------------------------------------------------------------------------
+# projections: f1 (phi1 = SiLU, split U V Q K) and f2
+# ----------------------------------------------------------------------------
+
+def test_f1_split_order_and_silu_closed_form():
+    """W1 made of four scaled identity blocks: block r of the output is SiLU(c_r x) in the
+    order U, V, Q, K, with SiLU(z) = z * expit(z) from scipy."""
+    T, D = 9, 16
+    x = np.random.default_rng(6).normal(size=(T, D)).astype(np.float32)
+    scales = [1.0, -2.0, 0.5, 3.0]
+    w1 = np.concatenate([c * np.eye(D, dtype=np.float32) for c in scales])
+    z, *blocks = oracle.f1_fwd(x, w1, None, D)
+    for c, blk in zip(scales, blocks):
+        ref = c * x.astype(np.float64)
+        np.testing.assert_allclose(blk, ref * expit(ref), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(z[:, D:2 * D], -2.0 * x, rtol=0, atol=0)
+    b1 = np.arange(4 * D, dtype=np.float32)
+    z0, *_ = oracle.f1_fwd(np.zeros((2, D), np.float32), w1, b1, D)
+    np.testing.assert_array_equal(z0, np.tile(b1, (2, 1)))
+
+
+def test_f2_zero_weight_is_bias_plus_residual():
+    rng = np.random.default_rng(7)
+    o = rng.normal(size=(5, 32)).astype(np.float32)
+    b2 = rng.normal(size=48).astype(np.float32)
+    res = rng.normal(size=(5, 48)).astype(np.float32)
+    out = oracle.f2_fwd(o, np.zeros((48, 32), np.float32), b2, res)
+    np.testing.assert_allclose(out, b2.astype(np.float64) + res, rtol=0, atol=0)
+
+
+def test_projection_gradients_match_torch_autograd():
+    """f1 and f2 backward against float64 torch autograd of the forward definition."""
+    w = W.make_projection(23, 48, 16, 40, seed=8, dtype=torch.float32)
+    x = torch.tensor(w.x.numpy(), dtype=torch.float64, requires_grad=True)
+    w1 = torch.tensor(w.w1.numpy(), dtype=torch.float64, requires_grad=True)
+    b1 = torch.tensor(w.b1.numpy(), dtype=torch.float64, requires_grad=True)
+    z = x @ w1.T + b1
+    a = torch.nn.functional.silu(z)
+    a.backward(torch.tensor(w.dact.numpy(), dtype=torch.float64))
+    D = w.D
+    zo, *_ = oracle.f1_fwd(w.x, w.w1, w.b1, D)
+    dact = w.dact.numpy()
+    dz, dx, dw1, db1 = oracle.f1_bwd(w.x, w.w1, zo, dact[:, :D], dact[:, D:2 * D], dact[:, 2 * D:3 * D],
+                                     dact[:, 3 * D:])
+    np.testing.assert_allclose(dx, x.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dw1, w1.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(db1, b1.grad.numpy(), rtol=1e-11, atol=1e-12)
+    o = torch.tensor(w.o_pre.numpy(), dtype=torch.float64, requires_grad=True)
+    w2 = torch.tensor(w.w2.numpy(), dtype=torch.float64, requires_grad=True)
+    b2 = torch.tensor(w.b2.numpy(), dtype=torch.float64, requires_grad=True)
+    (o @ w2.T + b2).backward(torch.tensor(w.g_out.numpy(), dtype=torch.float64))
+    do, dw2, db2 = oracle.f2_bwd(w.o_pre, w.w2, w.g_out)
+    np.testing.assert_allclose(do, o.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dw2, w2.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(db2, b2.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
 # backward: central finite differences with Richardson extrapolation
 # ----------------------------------------------------------------------------
 
