@@ -337,6 +337,70 @@ def f2_bwd(o_pre, w2, g):
     return g @ _as_f64(w2), g.T @ _as_f64(o_pre), g.sum(0)
 
 
+# ----------------------------------------------------------------------------
+# Stochastic Length (HSTU blog, section 3.4) and token-balanced batches (MTGR
+# deep-dive, section 3, contribution 3)
+# ----------------------------------------------------------------------------
+
+_SM_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+
+
+def splitmix64(state: int, n) -> np.ndarray:
+    """Output n (n >= 1) of SplitMix64 from `state` (Steele, Lea and Flood, OOPSLA 2014):
+    z = state + n * gamma, then the published xor-shift-multiply finaliser."""
+    with np.errstate(over="ignore"):
+        z = np.uint64(state) + np.asarray(n, dtype=np.uint64) * _SM_GAMMA
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+def sl_keys(seed: int, b: int, L: int) -> np.ndarray:
+    """Random key of event i of sequence b: SplitMix64 output number b * 2^32 + i + 1."""
+    return splitmix64(seed, np.uint64(b) * np.uint64(1 << 32) + np.arange(L, dtype=np.uint64) + np.uint64(1))
+
+
+def sl_sample(offsets, cap: int, seed: int):
+    """Stochastic Length: a sequence longer than cap keeps the cap events with the smallest
+    keys (ties by index) -- a uniform random subset -- in their original order.  Returns
+    (new offsets int32 [B+1], gather indices int64 into the input tokens)."""
+    off = np.asarray(offsets, dtype=np.int64)
+    new = [0]
+    idx = []
+    for b in range(len(off) - 1):
+        L = int(off[b + 1] - off[b])
+        if L <= cap:
+            keep = np.arange(L)
+        else:
+            keys = sl_keys(seed, b, L)
+            order = np.lexsort((np.arange(L), keys))      # by key, then by index
+            keep = np.sort(order[:cap])
+        idx.append(off[b] + keep)
+        new.append(new[-1] + len(keep))
+    gather = np.concatenate(idx) if idx else np.zeros(0, np.int64)
+    return np.asarray(new, dtype=np.int32), gather.astype(np.int64)
+
+
+def pack_balanced(offsets, n_bins: int):
+    """Token-balanced contiguous batches: sequence b (tokens [s_b, s_b + L_b) of T) goes to
+    bin floor((s_b + L_b / 2) * n_bins / T), clamped to n_bins - 1.  Returns (bin_seq_start
+    [n_bins+1], bin_tokens [n_bins], weights [n_bins] = sequences in the bin / B, the factor
+    that makes the weighted sum of per-bin mean gradients the mean over all sequences)."""
+    off = np.asarray(offsets, dtype=np.int64)
+    B = len(off) - 1
+    T = int(off[-1])
+    bins = np.zeros(B, np.int64)
+    for b in range(B):
+        mid2 = 2 * off[b] + (off[b + 1] - off[b])        # twice the midpoint, kept integral
+        bins[b] = min(n_bins - 1, (mid2 * n_bins) // (2 * T)) if T > 0 else 0
+    start = np.zeros(n_bins + 1, np.int64)
+    for r in range(n_bins + 1):
+        start[r] = int(np.searchsorted(bins, r, side="left"))
+    tokens = np.array([off[start[r + 1]] - off[start[r]] for r in range(n_bins)], np.int64)
+    weights = np.array([(start[r + 1] - start[r]) / B if B else 0.0 for r in range(n_bins)])
+    return start.astype(np.int32), tokens, weights
+
+
 def layer_fwd(w, rows=None):
     """(y, o_pre, mean, rstd) for the listed rows: attention, then Norm(y) * u."""
     y = attn_fwd(w, rows)

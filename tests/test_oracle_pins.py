@@ -463,6 +463,67 @@ def test_projection_gradients_match_torch_autograd():
 
 
 # ----------------------------------------------------------------------------
+# Stochastic Length sampler and token-balanced batches
+# ----------------------------------------------------------------------------
+
+def test_splitmix64_known_answers():
+    rows = [r.split() for r in read_golden("splitmix64_seed1234567.txt")]
+    n = np.array([int(a) for a, _ in rows], dtype=np.uint64)
+    want = np.array([int(b) for _, b in rows], dtype=np.uint64)
+    np.testing.assert_array_equal(oracle.splitmix64(1234567, n), want)
+
+
+def test_sl_keeps_cap_events_in_order_and_short_rows_whole():
+    lens = [776, 777, 4096, 5, 0, 1000]
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    new, idx = oracle.sl_sample(off, 776, seed=42)
+    np.testing.assert_array_equal(np.diff(new), [776, 776, 776, 5, 0, 776])
+    for b in range(len(lens)):
+        g = idx[new[b]:new[b + 1]]
+        assert np.all(np.diff(g) > 0)                                  # original order, no repeats
+        assert np.all((g >= off[b]) & (g < off[b + 1]))
+    np.testing.assert_array_equal(idx[new[0]:new[1]], np.arange(776))  # at the cap: untouched
+    np.testing.assert_array_equal(idx[new[3]:new[4]], off[3] + np.arange(5))
+    # the 777-event row drops exactly the event with the largest key
+    keys = oracle.sl_keys(42, 1, 777)
+    assert int(np.argmax(keys)) not in set((idx[new[1]:new[2]] - off[1]).tolist())
+
+
+def test_sl_subset_is_uniform():
+    """Each of L = 20 events is kept with probability cap / L = 1/4 (over 4000 seeds),
+    and every 2-subset of positions appears with probability (5*4)/(20*19)."""
+    L, cap, n = 20, 5, 4000
+    off = np.array([0, L], np.int32)
+    hits = np.zeros(L)
+    pair = 0
+    for s in range(n):
+        _, idx = oracle.sl_sample(off, cap, seed=s)
+        hits[idx] += 1
+        pair += (0 in idx) and (19 in idx)
+    p = cap / L
+    sd = np.sqrt(n * p * (1 - p))
+    assert np.all(np.abs(hits - n * p) < 5 * sd), hits
+    p2 = cap * (cap - 1) / (L * (L - 1))
+    assert abs(pair - n * p2) < 5 * np.sqrt(n * p2 * (1 - p2))
+
+
+def test_pack_balanced_contiguous_and_balanced():
+    rng = np.random.default_rng(10)
+    lens = rng.integers(16, 4096, size=300)
+    off = np.concatenate([[0], np.cumsum(lens)])
+    start, tokens, weights = oracle.pack_balanced(off, 8)
+    assert start[0] == 0 and start[-1] == 300 and np.all(np.diff(start) >= 0)
+    assert tokens.sum() == off[-1]
+    assert np.all(np.abs(tokens - off[-1] / 8) <= lens.max())          # within one sequence of even
+    np.testing.assert_allclose(weights.sum(), 1.0)
+    # equal lengths split into equal bins
+    off_eq = np.arange(0, 65 * 100, 100)
+    s2, t2, w2 = oracle.pack_balanced(off_eq, 4)
+    np.testing.assert_array_equal(s2, [0, 16, 32, 48, 64])
+    np.testing.assert_allclose(w2, 0.25)
+
+
+# ----------------------------------------------------------------------------
 # backward: central finite differences with Richardson extrapolation
 # ----------------------------------------------------------------------------
 
