@@ -365,6 +365,8 @@ def run_ours(args, world, rank, local):
         extra["gln"] = run_gln(args, world, w, dv, off, ts, rp, rt, fwd_out, bwd_out)
     if not args.no_proj:
         extra["projections"] = run_proj(args, world, rank)
+    if not args.no_data:
+        extra["data_step"] = run_data_step(args, world, rank, w)
 
     # ---- end to end through the C ABI with host buffers
     if args.no_e2e:
@@ -488,6 +490,56 @@ def run_proj(args, world, rank):
                                           if k != "gemm_tc_kernel"},
             "cublas_same_products_ms": round(ms_lib, 4),
             "cublas_tflops": round(flops / (ms_lib * 1e-3) / 1e12, 1)}
+
+
+def run_data_step(args, world, rank, w):
+    """The data step on the large layer's raw batch: Stochastic Length (cap 776 = 4096^0.8),
+    the gathers of the kept rows (d_model 1024 bf16 features and int64 timestamps), and the
+    token-balanced split into 8 bins."""
+    from hstu_jagged_pointwise_b200 import capi, ops
+    dev = torch.device("cuda", torch.cuda.current_device())
+    off = torch.as_tensor(w.offsets).to(dev)
+    gen = torch.Generator(device=dev).manual_seed(args.seed + 91)
+    feats = torch.randn(w.T, 1024, generator=gen, device=dev).to(torch.bfloat16)
+    ts = torch.as_tensor(w.ts).to(dev)
+    cap = W.stochastic_length_cap(4096, 1.6)
+    n_out = int(np.minimum(np.diff(w.offsets), cap).sum())   # the sampled size does not depend on the seed
+    state = {}
+
+    def step(i):
+        o = ops.sl_sample(off, cap, seed=args.seed + i, out_capacity=w.T)
+        n = n_out
+        state["f"] = ops.gather_rows(feats, o["gather"], n, out=state.get("f"))
+        state["t"] = ops.gather_rows(ts, o["gather"], n, out=state.get("t"))
+        state["p"] = ops.pack_balanced(o["offsets"], 8)
+        state["o"] = o
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if int(state["o"]["offsets"][-1].item()) != n_out:
+        raise RuntimeError("sampled size differs from the sum of min(L, cap)")
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    capi.profile_enable(True)
+    e0.record(s)
+    for i in range(args.steps):
+        step(i)
+    e1.record(s)
+    torch.cuda.synchronize()
+    prof = capi.profile_read()
+    capi.profile_enable(False)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    if int(state["o"]["status"].item()) != 0:
+        raise RuntimeError("device status set by the Stochastic Length sampler")
+    n_g, t_g = prof["gather_rows_kernel"]
+    gbytes = n_out * (2 * (1024 * 2 + 8) + 2 * 4)            # rows read and written, the index read twice
+    pk, _ = peaks()
+    return {"workload": f"{w.name}_raw", "sl_cap": cap, "tokens_in": w.T, "tokens_out": n_out,
+            "ms_per_step": round(ms, 4), "sl_sample_ms": round(prof["sl_sample_kernels"][1] / args.steps, 4),
+            "gather_ms": round(t_g / args.steps, 4),
+            "gather_gbs": round(gbytes / (t_g / args.steps * 1e-3) / 1e9, 1),
+            "gather_frac_hbm": round(gbytes / (t_g / args.steps * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
 
 
 def run_gln(args, world, w, dv, off, ts, rp, rt, fwd_out, bwd_out):
@@ -755,6 +807,7 @@ def main():
     ap.add_argument("--no-mfalcon", action="store_true")
     ap.add_argument("--no-gln", action="store_true", help="skip the Group LayerNorm variant")
     ap.add_argument("--no-proj", action="store_true", help="skip the f1 / f2 projections")
+    ap.add_argument("--no-data", action="store_true", help="skip the Stochastic Length / packing data step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--tokens", type=int, default=262144,

@@ -32,7 +32,8 @@ EXPORTS = (
     "hstu_version", "hstu_profile_enable", "hstu_profile_read", "hstu_profile_kind_name",
     "hstu_attn_fwd_noalloc", "hstu_mfalcon_cache_history", "hstu_attn_fwd_gln", "hstu_attn_bwd_gln",
     "hstu_attn_workspace_bytes_gln", "hstu_f1_fwd", "hstu_f2_fwd", "hstu_f1_bwd_workspace_bytes",
-    "hstu_f2_bwd_workspace_bytes", "hstu_f1_bwd", "hstu_f2_bwd",
+    "hstu_f2_bwd_workspace_bytes", "hstu_f1_bwd", "hstu_f2_bwd", "hstu_sl_sample", "hstu_gather_rows",
+    "hstu_pack_balanced",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20   # HSTU_NOALLOC_SCRATCH_BYTES
@@ -108,6 +109,12 @@ def load():
     lib.hstu_f1_bwd.restype = C.c_int
     lib.hstu_f2_bwd.argtypes = [i32, i32, i32] + [P] * 7 + [S, P, P]
     lib.hstu_f2_bwd.restype = C.c_int
+    lib.hstu_sl_sample.argtypes = [i32, i32, P, i32, C.c_uint64, C.c_int64, P, P, P, P]
+    lib.hstu_sl_sample.restype = C.c_int
+    lib.hstu_gather_rows.argtypes = [C.c_int64, i32, P, C.c_int64, P, P, P]
+    lib.hstu_gather_rows.restype = C.c_int
+    lib.hstu_pack_balanced.argtypes = [i32, P, i32, P, P, P, P]
+    lib.hstu_pack_balanced.restype = C.c_int
     lib.hstu_debug_indices.argtypes = [i32, i32, P, P, P, P, i32, i32, P, P, P, P, P]
     lib.hstu_debug_indices.restype = C.c_int
     lib.hstu_check_device_error.argtypes = [P, P]

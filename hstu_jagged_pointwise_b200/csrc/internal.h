@@ -183,7 +183,7 @@ int device_sms();
 enum ProfKind {
     kProfSchedule = 0, kProfAttnFwdTc, kProfAttnFwdSimt, kProfLnFwd, kProfLnBwd, kProfLnBwdReduce,
     kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfDqConvert,
-    kProfRabReduce, kProfCacheScan, kProfCacheCopy, kProfGemm, kProfSiluGrad, kProfColSum, kProfKinds
+    kProfRabReduce, kProfCacheScan, kProfCacheCopy, kProfGemm, kProfSiluGrad, kProfColSum, kProfSlSample, kProfGather, kProfKinds
 };
 void prof_begin(int kind, cudaStream_t s);
 void prof_end(int kind, cudaStream_t s);

@@ -30,7 +30,8 @@ const char* const kNames[kProfKinds] = {
     "schedule_kernel", "attn_fwd_tc_kernel", "attn_fwd_simt_kernel", "ln_fwd_kernel",
     "ln_bwd_kernel", "ln_bwd_reduce_kernel", "attn_bwd_dkv_simt_kernel", "attn_bwd_dq_simt_kernel",
     "debug_indices_kernel", "attn_bwd_tc_kernel", "dq_convert_kernel", "rab_reduce_kernel",
-    "cache_scan_kernel", "cache_copy_kernel", "gemm_tc_kernel", "silu_grad_kernel", "col_sum_kernel"};
+    "cache_scan_kernel", "cache_copy_kernel", "gemm_tc_kernel", "silu_grad_kernel", "col_sum_kernel",
+    "sl_sample_kernels", "gather_rows_kernel"};
 
 cudaEvent_t take_event() {
     if (!g_pool.empty()) {

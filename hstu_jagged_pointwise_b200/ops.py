@@ -270,6 +270,56 @@ def f2_bwd(o_pre, w2, g, out: Optional[dict] = None) -> dict:
     return out
 
 
+# ----------------------------------------------------------------------------
+# the data step: Stochastic Length sampling, row gathers, token-balanced bins
+# ----------------------------------------------------------------------------
+
+def sl_sample(seq_offsets, cap: int, seed: int, out_capacity: Optional[int] = None) -> dict:
+    """Stochastic Length: sequences longer than cap keep a uniform random subset of cap events
+    in order.  Returns offsets [B+1], gather (input token index per output token, int32) and
+    status (device int32, nonzero for an invalid batch or too small a capacity)."""
+    _need(seq_offsets, "seq_offsets", torch.int32)
+    B = seq_offsets.numel() - 1
+    T = int(seq_offsets[-1].item())
+    cap_out = T if out_capacity is None else int(out_capacity)
+    dev = seq_offsets.device
+    out = dict(offsets=torch.empty(B + 1, dtype=torch.int32, device=dev),
+               gather=torch.empty(max(cap_out, 1), dtype=torch.int32, device=dev), status=_status(dev))
+    st = capi.LIB.hstu_sl_sample(B, T, _p(seq_offsets), int(cap), C.c_uint64(int(seed) & (2**64 - 1)), cap_out,
+                                 _p(out["offsets"]), _p(out["gather"]), _p(out["status"]), _stream())
+    capi.check(st, "hstu_sl_sample")
+    return out
+
+
+def gather_rows(src: torch.Tensor, idx: torch.Tensor, n_rows: Optional[int] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[r] = src[idx[r]] for the first n_rows indices (rows of any contiguous tensor)."""
+    if not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    _need(idx, "idx", torch.int32)
+    n = idx.numel() if n_rows is None else int(n_rows)
+    if out is None:
+        out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] > 0 else out[0].numel() * out.element_size()
+    st = capi.LIB.hstu_gather_rows(n, row_bytes, _p(src), src.shape[0], _p(idx), _p(out), _stream())
+    capi.check(st, "hstu_gather_rows")
+    return out
+
+
+def pack_balanced(seq_offsets, n_bins: int) -> dict:
+    """Token-balanced contiguous bins of sequences and their gradient weights."""
+    _need(seq_offsets, "seq_offsets", torch.int32)
+    B = seq_offsets.numel() - 1
+    dev = seq_offsets.device
+    out = dict(bin_seq_start=torch.empty(n_bins + 1, dtype=torch.int32, device=dev),
+               bin_tokens=torch.empty(n_bins, dtype=torch.int32, device=dev),
+               bin_weight=torch.empty(n_bins, dtype=torch.float32, device=dev))
+    st = capi.LIB.hstu_pack_balanced(B, _p(seq_offsets), int(n_bins), _p(out["bin_seq_start"]),
+                                     _p(out["bin_tokens"]), _p(out["bin_weight"]), _stream())
+    capi.check(st, "hstu_pack_balanced")
+    return out
+
+
 def mfalcon_cache_history(seq_offsets, timestamps, n_history, k, v, hist_rows: Optional[int] = None,
                           out: Optional[dict] = None) -> dict:
     """KV cache for MFalcon.score from a full-sequence M-FALCON batch: the first

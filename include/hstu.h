@@ -343,6 +343,49 @@ HSTU_API int hstu_f2_bwd(int32_t T, int32_t D, int32_t d_out, const void* o_pre,
                   const void* d_out_grad, void* d_o_pre, float* dw2, float* db2,
                   void* workspace, size_t workspace_bytes, int32_t* device_status, void* stream);
 
+/* ---- The data step in front of the attention. */
+
+/* Stochastic Length (HSTU blog, section 3.4: training samples variable-length
+ * subsequences of long-tailed histories; alpha = 1.6 keeps about 776 = 4096^0.8
+ * of 4096 events).  Reading: a sequence longer than `cap` keeps a uniform
+ * random subset of cap events in their original order; shorter ones are kept
+ * whole.  Event i of sequence b draws the key SplitMix64(seed, b * 2^32 + i + 1)
+ * (output number b * 2^32 + i + 1 of the SplitMix64 generator started at
+ * `seed`); the cap smallest keys, ties by index, are kept.
+ * In:  seq_offsets DEVICE int32 [B+1] of a jagged batch of T tokens.
+ * Out: out_offsets DEVICE int32 [B+1] of the sampled batch; gather_idx DEVICE
+ *      int32 [out_capacity]: input token index of each output token (apply it
+ *      with hstu_gather_rows to features, timestamps, ...).  Positions are
+ *      re-indexed implicitly: an output token's position is its index in its
+ *      output sequence.
+ * device_status: DEVICE int32, required; set to 0, or 1 when seq_offsets is not
+ *      a valid layout of T tokens or the output exceeds out_capacity (then
+ *      nothing else is written).
+ * Returns HSTU_ERR_INVALID_ARG for negative sizes, cap < 1 or a missing /
+ * misaligned pointer, before any launch. */
+HSTU_API int hstu_sl_sample(int32_t B, int32_t T, const int32_t* seq_offsets, int32_t cap, uint64_t seed,
+                  int64_t out_capacity, int32_t* out_offsets, int32_t* gather_idx,
+                  int32_t* device_status, void* stream);
+
+/* dst row r = src row idx[r] for r < n_rows (rows of row_bytes bytes; src has
+ * n_src rows; an index outside [0, n_src) gives a zero row).  16-byte rows use
+ * one warp per row with 16-byte vectors. */
+HSTU_API int hstu_gather_rows(int64_t n_rows, int32_t row_bytes, const void* src, int64_t n_src,
+                  const int32_t* idx, void* dst, void* stream);
+
+/* Token-balanced batches (MTGR deep-dive, section 3, contribution 3: batch sizes
+ * adapt so that every GPU gets the same token count, and gradient aggregation
+ * is weighted).  Sequence b, tokens [s_b, s_b + L_b) of T, goes to bin
+ * floor((2 s_b + L_b) n_bins / (2 T)): bins are contiguous sequence ranges
+ * [bin_seq_start[r], bin_seq_start[r+1]) (DEVICE int32 [n_bins+1]) holding
+ * bin_tokens[r] tokens (int32 [n_bins]), each within one sequence length of
+ * T / n_bins; bin_weight[r] (fp32 [n_bins]) = sequences in bin r / B, the
+ * factor that turns per-bin mean gradients into the batch mean.  seq_offsets
+ * must be a valid jagged layout (results are unspecified otherwise, reads stay
+ * in bounds). */
+HSTU_API int hstu_pack_balanced(int32_t B, const int32_t* seq_offsets, int32_t n_bins, int32_t* bin_seq_start,
+                  int32_t* bin_tokens, float* bin_weight, void* stream);
+
 /* Integer decisions of the fused kernels, written through the same device
  * functions they use, for exact comparison in tests.  For every sequence b and
  * pair (i, j) of it, entry pair_offsets[b] + i*L_b + j (pair_offsets: device

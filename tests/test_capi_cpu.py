@@ -18,7 +18,7 @@ def header_functions():
 
 def test_exports_match_header():
     names = header_functions()
-    assert len(names) == 23, names
+    assert len(names) == 26, names
     assert set(names) == set(capi.EXPORTS)
     for n in names:
         assert hasattr(capi.LIB, n), n
@@ -142,6 +142,23 @@ def test_projections_reject_bad_arguments_before_launch():
     assert capi.LIB.hstu_f2_bwd_workspace_bytes(4, 64) > 0
     assert capi.LIB.hstu_f1_bwd(4, 64, 64, *([a] * 11), 16, None, None) == capi.HSTU_ERR_WORKSPACE
     assert capi.LIB.hstu_f2_bwd(4, 64, 64, *([a] * 7), 16, None, None) == capi.HSTU_ERR_WORKSPACE
+
+
+def test_data_step_rejects_bad_arguments_before_launch():
+    buf = (C.c_uint8 * 4096)()
+    a = (C.addressof(buf) + 255) // 256 * 256
+    f = capi.LIB.hstu_sl_sample
+    assert f(-1, 0, a, 8, 1, 0, a, a, a, None) == capi.HSTU_ERR_INVALID_ARG
+    assert f(1, 4, a, 0, 1, 4, a, a, a, None) == capi.HSTU_ERR_INVALID_ARG      # cap < 1
+    assert f(1, 4, a, 8, 1, 4, a, a, None, None) == capi.HSTU_ERR_INVALID_ARG   # no status word
+    assert f(1, 4, a + 2, 8, 1, 4, a, a, a, None) == capi.HSTU_ERR_INVALID_ARG  # misaligned offsets
+    g = capi.LIB.hstu_gather_rows
+    assert g(-1, 16, a, 4, a, a, None) == capi.HSTU_ERR_INVALID_ARG
+    assert g(4, 0, a, 4, a, a, None) == capi.HSTU_ERR_INVALID_ARG
+    assert g(0, 16, None, 0, None, None, None) == capi.HSTU_OK                  # nothing to gather
+    p = capi.LIB.hstu_pack_balanced
+    assert p(4, a, 0, a, a, a, None) == capi.HSTU_ERR_INVALID_ARG               # no bins
+    assert p(4, a, 2, a, None, a, None) == capi.HSTU_ERR_INVALID_ARG
 
 
 def test_mfalcon_rejects_bad_arguments():

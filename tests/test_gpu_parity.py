@@ -439,6 +439,72 @@ def test_projections_large_sampled():
 
 
 # ----------------------------------------------------------------------------
+# the data step: Stochastic Length sampling, gathers, token-balanced bins (bit-exact)
+# ----------------------------------------------------------------------------
+
+def _sl_check(lens, cap, seed, width=256):
+    from hstu_jagged_pointwise_b200 import ops
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    new_ref, idx_ref = oracle.sl_sample(off, cap, seed)
+    o = ops.sl_sample(torch.as_tensor(off).cuda(), cap, seed)
+    torch.cuda.synchronize()
+    assert int(o["status"].item()) == 0
+    np.testing.assert_array_equal(o["offsets"].cpu().numpy(), new_ref)
+    n = int(new_ref[-1])
+    np.testing.assert_array_equal(o["gather"][:n].cpu().numpy(), idx_ref)
+    return off, o, n, idx_ref
+
+
+def test_sl_sample_small_bit_exact():
+    lens = [0, 1, 775, 776, 777, 4096, 8192, 3, 1500, 0]
+    for seed in (0, 1, 2**63 + 12345):
+        off, o, n, idx_ref = _sl_check(lens, 776, seed)
+    # gathers: features (16-byte rows) and timestamps (8-byte rows) of the kept tokens
+    from hstu_jagged_pointwise_b200 import ops
+    T = int(off[-1])
+    gen = torch.Generator().manual_seed(3)
+    feats = torch.randn(T, 256, generator=gen).to(torch.bfloat16)
+    ts = torch.as_tensor(W.increasing_ts(np.random.default_rng(4), T))
+    gf = ops.gather_rows(feats.cuda(), o["gather"], n)
+    gt = ops.gather_rows(ts.cuda(), o["gather"], n)
+    torch.cuda.synchronize()
+    assert torch.equal(gf.cpu(), feats[torch.as_tensor(idx_ref)])
+    assert torch.equal(gt.cpu(), ts[torch.as_tensor(idx_ref)])
+
+
+def test_sl_sample_training_and_large_batches_bit_exact():
+    rng = np.random.default_rng(11)
+    _sl_check(W.zipf_lengths(rng, 64), W.stochastic_length_cap(4096, 1.6), seed=5)     # raw training batch
+    _sl_check(W.lognormal_lengths(rng, 262144), 776, seed=6)                            # 262,144 tokens
+
+
+def test_sl_sample_flags_bad_batches():
+    from hstu_jagged_pointwise_b200 import ops
+    bad = torch.tensor([0, 10, 5, 20], dtype=torch.int32, device="cuda")       # a negative length
+    o = ops.sl_sample(bad, 8, 1, out_capacity=100)
+    torch.cuda.synchronize()
+    assert int(o["status"].item()) == 1
+    ok = torch.tensor([0, 10, 30], dtype=torch.int32, device="cuda")
+    o = ops.sl_sample(ok, 8, 1, out_capacity=15)                              # needs 16 rows
+    torch.cuda.synchronize()
+    assert int(o["status"].item()) == 1
+
+
+def test_pack_balanced_matches_oracle():
+    from hstu_jagged_pointwise_b200 import ops
+    rng = np.random.default_rng(12)
+    for lens, R in ((rng.integers(16, 4096, size=300), 8), (np.full(64, 100), 4), (np.array([5]), 3),
+                    (np.zeros(0, np.int64), 2), (W.lognormal_lengths(rng, 262144), 16)):
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        start, tokens, weights = oracle.pack_balanced(off, R)
+        o = ops.pack_balanced(torch.as_tensor(off).cuda(), R)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(o["bin_seq_start"].cpu().numpy(), start)
+        np.testing.assert_array_equal(o["bin_tokens"].cpu().numpy(), tokens)
+        np.testing.assert_allclose(o["bin_weight"].cpu().numpy(), weights, rtol=1e-6, atol=0)
+
+
+# ----------------------------------------------------------------------------
 # the named workloads at full size
 # ----------------------------------------------------------------------------
 
