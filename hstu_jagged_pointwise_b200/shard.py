@@ -46,11 +46,21 @@ def shard_rows(offsets: np.ndarray, seqs: Sequence[int]):
     return new.astype(np.int32), rows
 
 
-def allreduce_param_grads(grads: Dict[str, torch.Tensor], group=None) -> None:
-    """Sum the parameter gradients over the process group in place (one flat all-reduce)."""
+def bin_sequences(bin_seq_start, rank: int) -> List[int]:
+    """The sequences of token-balanced bin `rank` (contiguous: [start[rank], start[rank + 1]))."""
+    a, z = int(bin_seq_start[rank]), int(bin_seq_start[rank + 1])
+    return list(range(a, z))
+
+
+def allreduce_param_grads(grads: Dict[str, torch.Tensor], group=None, weight: float = 1.0) -> None:
+    """Sum weight * (parameter gradients) over the process group in place (one flat all-reduce).
+    With token-balanced bins, each rank's per-sample mean gradient carries weight = its samples /
+    all samples (MTGR's re-weighted aggregation), so the sum is the mean over the whole batch."""
     import torch.distributed as dist
     ts = [grads[k] for k in PARAM_GRADS]
     flat = torch.cat([t.reshape(-1) for t in ts])
+    if weight != 1.0:
+        flat.mul_(weight)
     dist.all_reduce(flat, group=group)
     o = 0
     for t in ts:

@@ -93,3 +93,52 @@ def test_two_rank_gloo_matches_single_process():
         for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (du, "du")):
             np.testing.assert_allclose(got, ref[name][rows], rtol=1e-12, atol=1e-14)
     assert sorted(covered) == list(range(w.T))
+
+
+def _balanced_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import oracle
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = _global_batch()
+        start, tokens, weights = oracle.pack_balanced(w.offsets, world)
+        seqs = shard.bin_sequences(start, rank)
+        s, rows = _sub(w, seqs)
+        g = oracle.layer_bwd(s)
+        n = max(len(seqs), 1)
+        # this rank's per-sample mean of the parameter gradients, re-weighted by its share of samples
+        grads = {"d_rab_pos": torch.tensor(g["d_rab_pos"]) / n, "d_rab_time": torch.tensor(g["d_rab_time"]) / n,
+                 "d_gamma": torch.tensor(g["dgamma"]) / n, "d_beta": torch.tensor(g["dbeta"]) / n}
+        shard.allreduce_param_grads(grads, weight=float(weights[rank]))
+        q.put((rank, seqs, int(tokens[rank]), {k: v.numpy() for k, v in grads.items()}))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_token_balanced_bins_give_the_batch_mean_gradient():
+    """MTGR's dynamic batches: each rank takes one token-balanced bin (different sample
+    counts), and the weighted all-reduce of per-rank mean gradients is the batch mean."""
+    import oracle
+    w = _global_batch()
+    ref = oracle.layer_bwd(w)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_balanced_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    seqs = sorted(b for _, sq, _, _ in res for b in sq)
+    assert seqs == list(range(w.B))
+    assert len({len(sq) for _, sq, _, _ in res}) == 2            # the bins hold different sample counts
+    for _, _, tok, grads in res:
+        assert abs(tok - w.T / 2) <= w.lengths.max()
+        for k, rk in (("d_rab_pos", "d_rab_pos"), ("d_rab_time", "d_rab_time"), ("d_gamma", "dgamma"),
+                      ("d_beta", "dbeta")):
+            np.testing.assert_allclose(grads[k], ref[rk] / w.B, rtol=1e-12, atol=1e-14)
