@@ -367,6 +367,8 @@ def run_ours(args, world, rank, local):
         extra["projections"] = run_proj(args, world, rank)
     if not args.no_data:
         extra["data_step"] = run_data_step(args, world, rank, w)
+    if not args.no_layer:
+        extra["full_layer"] = run_full_layer(args, world, w, f_fwd + f_bwd)
 
     # ---- end to end through the C ABI with host buffers
     if args.no_e2e:
@@ -490,6 +492,55 @@ def run_proj(args, world, rank):
                                           if k != "gemm_tc_kernel"},
             "cublas_same_products_ms": round(ms_lib, 4),
             "cublas_tflops": round(flops / (ms_lib * 1e-3) / 1e12, 1)}
+
+
+def run_full_layer(args, world, w, attn_flops):
+    """The whole layer on the same batch (d_model 1024): f1 -> attention -> Norm * U -> f2 + X,
+    forward and backward, through ops.HSTULayer."""
+    from hstu_jagged_pointwise_b200 import capi, ops
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gen = torch.Generator(device=dev).manual_seed(args.seed + 55)
+    dm, D = 1024, w.D
+    x = torch.randn(w.T, dm, generator=gen, device=dev).to(torch.bfloat16)
+    g_out = torch.randn(w.T, dm, generator=gen, device=dev).to(torch.bfloat16)
+    prm = dict(w1=(torch.randn(4 * D, dm, generator=gen, device=dev) * dm ** -0.5).to(torch.bfloat16),
+               b1=0.1 * torch.randn(4 * D, generator=gen, device=dev),
+               w2=(torch.randn(dm, D, generator=gen, device=dev) * D ** -0.5).to(torch.bfloat16),
+               b2=0.1 * torch.randn(dm, generator=gen, device=dev),
+               rab_pos=w.rab_pos.to(dev), rab_time=w.rab_time.to(dev), ln_gamma=w.gamma.to(dev),
+               ln_beta=w.beta.to(dev))
+    layer = ops.HSTULayer(torch.as_tensor(w.offsets).to(dev), torch.as_tensor(w.ts).to(dev), dm, w.H, w.d,
+                          w.alpha, w.max_len)
+
+    def step():
+        f = layer.forward(x, prm)
+        layer.backward(f, g_out, prm)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    capi.profile_enable(True)
+    e0.record(s)
+    for _ in range(args.steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    prof = capi.profile_read()
+    capi.profile_enable(False)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    if layer.check_device_error() != 0:
+        raise RuntimeError("device status set in the full layer")
+    proj_flops = 3 * 2 * w.T * (dm * 4 * D + D * dm)
+    flops = attn_flops + proj_flops
+    pk, _ = peaks()
+    tf = world * flops / (ms * 1e-3) / 1e12
+    return {"workload": f"{w.name}_dmodel{dm}", "ms_per_step": round(ms, 4), "tflops": round(tf, 1),
+            "pct_bf16_sustained": round(tf / world / pk["bf16_tflops_sustained"], 4),
+            "kernel_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in sorted(prof.items(),
+                                                                                      key=lambda kv: -kv[1][1])}}
 
 
 def run_data_step(args, world, rank, w):
@@ -808,6 +859,7 @@ def main():
     ap.add_argument("--no-gln", action="store_true", help="skip the Group LayerNorm variant")
     ap.add_argument("--no-proj", action="store_true", help="skip the f1 / f2 projections")
     ap.add_argument("--no-data", action="store_true", help="skip the Stochastic Length / packing data step")
+    ap.add_argument("--no-layer", action="store_true", help="skip the whole-layer (f1, attention, f2) step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--tokens", type=int, default=262144,

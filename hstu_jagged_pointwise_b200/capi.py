@@ -105,7 +105,7 @@ def load():
     lib.hstu_f1_bwd_workspace_bytes.restype = S
     lib.hstu_f2_bwd_workspace_bytes.argtypes = [i32, i32]
     lib.hstu_f2_bwd_workspace_bytes.restype = S
-    lib.hstu_f1_bwd.argtypes = [i32, i32, i32] + [P] * 11 + [S, P, P]
+    lib.hstu_f1_bwd.argtypes = [i32, i32, i32] + [P] * 12 + [S, P, P]
     lib.hstu_f1_bwd.restype = C.c_int
     lib.hstu_f2_bwd.argtypes = [i32, i32, i32] + [P] * 7 + [S, P, P]
     lib.hstu_f2_bwd.restype = C.c_int

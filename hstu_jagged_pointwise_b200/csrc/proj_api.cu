@@ -259,12 +259,13 @@ size_t hstu_f2_bwd_workspace_bytes(int32_t T, int32_t d_out) {
 }
 
 int hstu_f1_bwd(int32_t T, int32_t d_in, int32_t D, const void* x, const void* w1, const void* z, const void* du,
-                const void* dv, const void* dq, const void* dk, void* dx, float* dw1, float* db1, void* workspace,
-                size_t workspace_bytes, int32_t* device_status, void* stream) {
+                const void* dv, const void* dq, const void* dk, const void* dx_add, void* dx, float* dw1, float* db1,
+                void* workspace, size_t workspace_bytes, int32_t* device_status, void* stream) {
     if (T < 0 || d_in < 32 || D < 32 || (long long)4 * D > (1 << 20) || d_in > (1 << 20))
         return HSTU_ERR_INVALID_ARG;
     if (d_in % 32 || D % 32 || 4 * D > 8 * kSiluGradThreads * kSiluGradCols) return HSTU_ERR_UNSUPPORTED;
-    if (!al(dw1, 16) || !al(db1, 16) || !al_or_null(device_status, 4)) return HSTU_ERR_INVALID_ARG;
+    if (!al(dw1, 16) || !al(db1, 16) || !al_or_null(device_status, 4) || !al_or_null(dx_add, 16))
+        return HSTU_ERR_INVALID_ARG;
     if (!al(workspace, 256) || workspace_bytes < hstu_f1_bwd_workspace_bytes(T, D)) return HSTU_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (device_status && cudaMemsetAsync(device_status, 0, 4, s) != cudaSuccess) return HSTU_ERR_CUDA;
@@ -291,10 +292,11 @@ int hstu_f1_bwd(int32_t T, int32_t d_in, int32_t D, const void* x, const void* w
         col_sum_reduce_kernel<<<(4 * D + 255) / 256, 256, 0, s>>>(part, 4 * D, gblocks, db1);
     prof_end(kProfSiluGrad, s);
     if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
-    // 2. dX = dZ W1 (W1 [4D, d_in] read as the MN-major B operand)
+    // 2. dX = dZ W1 (+ dx_add) (W1 [4D, d_in] read as the MN-major B operand)
     GemmParams p = gemm_params(T, d_in, 4 * D, device_status);
     p.out = dx;
-    int st = run_gemm(false, true, kEpiBf16, dz, w1, p, s);
+    p.residual = static_cast<const __nv_bfloat16*>(dx_add);
+    int st = run_gemm(false, true, dx_add ? kEpiF2 : kEpiBf16, dz, w1, p, s);
     if (st != HSTU_OK) return st;
     // 3. dW1 = dZ^T X (both operands MN-major), split over the tokens
     GemmParams pw = gemm_params(4 * D, d_in, T, device_status);

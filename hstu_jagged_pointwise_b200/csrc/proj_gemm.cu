@@ -420,6 +420,7 @@ cudaError_t launch_gemm_tc(bool a_mn, bool b_mn, int epi, const CUtensorMap& ta,
     HSTU_GEMM_CASE(false, false, kEpiF1)
     else HSTU_GEMM_CASE(false, false, kEpiF2)
     else HSTU_GEMM_CASE(false, true, kEpiBf16)
+    else HSTU_GEMM_CASE(false, true, kEpiF2)
     else HSTU_GEMM_CASE(true, true, kEpiAddF32)
     else HSTU_GEMM_CASE(false, false, kEpiBf16)
 #undef HSTU_GEMM_CASE

@@ -159,6 +159,61 @@ class Layer:
         return int(capi.LIB.hstu_check_device_error(_p(self.ws), _stream()))
 
 
+class HSTULayer:
+    """One HSTU layer end to end on the library's kernels (Meta HSTU blog, section 3 formula):
+        U, V, Q, K = Split(SiLU(X W1^T + b1))            (f1, phi1 = SiLU)
+        Y = (SiLU(Q K^T + rab) * mask) V / alpha         (jagged pointwise attention)
+        O_pre = Norm(Y) * U                              (LayerNorm or Group LayerNorm)
+        out = O_pre W2^T + b2 (+ X when residual)        (f2)
+    Parameters are passed per call as a dict: w1 [4D, d_model], b1 [4D] or None, w2 [d_model, D],
+    b2 [d_model] or None, rab_pos, rab_time, ln_gamma, ln_beta (bf16 weights, fp32 the rest)."""
+
+    def __init__(self, seq_offsets, timestamps, d_model: int, H: int, d: int, alpha: float, max_seq_len: int,
+                 mask_kind: str = "causal", n_static=None, n_realtime=None, n_groups: int = 1, token_group=None,
+                 residual: bool = True, n_pos: int = 256, n_tbuckets: int = 64, ln_eps: float = 1e-5):
+        self.attn = Layer(seq_offsets, timestamps, H, d, torch.bfloat16, alpha, max_seq_len, mask_kind=mask_kind,
+                          n_static=n_static, n_realtime=n_realtime, n_pos=n_pos, n_tbuckets=n_tbuckets,
+                          ln_eps=ln_eps, n_groups=n_groups, token_group=token_group)
+        self.d_model, self.D, self.residual = d_model, H * d, residual
+        self._status = []
+
+    def forward(self, x, params: dict) -> dict:
+        """Returns out and the tensors the backward needs."""
+        _need(x, "x", torch.bfloat16)
+        f = f1_fwd(x, params["w1"], params.get("b1"), self.D)
+        a = self.attn.forward(f["q"], f["k"], f["v"], f["u"], params["rab_pos"], params["rab_time"],
+                              params["ln_gamma"], params["ln_beta"])
+        o = f2_fwd(a["o_pre"], params["w2"], params.get("b2"), residual=x if self.residual else None)
+        self._status = [f["status"], o["status"]]
+        return dict(out=o["out"], x=x, f1=f, attn=a)
+
+    def backward(self, saved: dict, d_out, params: dict) -> dict:
+        """Gradients of every input and parameter for d_out = dL/d out."""
+        _need(d_out, "d_out", torch.bfloat16)
+        f, a = saved["f1"], saved["attn"]
+        g2 = f2_bwd(a["o_pre"], params["w2"], d_out)
+        ga = self.attn.backward(f["q"], f["k"], f["v"], f["u"], params["rab_pos"], params["rab_time"],
+                                params["ln_gamma"], params["ln_beta"], a, g2["d_o_pre"])
+        g1 = f1_bwd(saved["x"], params["w1"], f["z"], ga["du"], ga["dv"], ga["dq"], ga["dk"],
+                    dx_add=d_out if self.residual else None)
+        self._status += [g2["status"], g1["status"]]
+        return dict(dx=g1["dx"], dw1=g1["dw1"], db1=g1["db1"], dw2=g2["dw2"], db2=g2["db2"],
+                    d_rab_pos=ga["d_rab_pos"], d_rab_time=ga["d_rab_time"], d_ln_gamma=ga["d_gamma"],
+                    d_ln_beta=ga["d_beta"], d_o_pre=g2["d_o_pre"], dq=ga["dq"], dk=ga["dk"], dv=ga["dv"],
+                    du=ga["du"])
+
+    def check_device_error(self) -> int:
+        """0, or the first nonzero status of the attention workspace or the projections' words."""
+        st = self.attn.check_device_error()
+        if st != 0:
+            return st
+        for t in self._status:
+            v = int(t.item())
+            if v != 0:
+                return capi.HSTU_ERR_DEVICE_TIMEOUT if v & 2 else capi.HSTU_ERR_DEVICE_BOUNDS
+        return 0
+
+
 class MFalcon:
     """M-FALCON candidate scoring against cached history K/V (microbatch b_m)."""
 
@@ -239,8 +294,9 @@ def f2_fwd(o_pre, w2, b2=None, residual=None, out: Optional[dict] = None) -> dic
     return out
 
 
-def f1_bwd(x, w1, z, du, dv, dq, dk, out: Optional[dict] = None) -> dict:
-    """dx [T, d_in] (bf16), dw1 [4D, d_in] and db1 [4D] (fp32) of f1 for the U, V, Q, K gradients."""
+def f1_bwd(x, w1, z, du, dv, dq, dk, out: Optional[dict] = None, dx_add=None) -> dict:
+    """dx [T, d_in] (bf16; plus dx_add when given), dw1 [4D, d_in] and db1 [4D] (fp32) of f1 for
+    the U, V, Q, K gradients."""
     T, d_in = x.shape
     D = du.shape[1]
     if out is None:
@@ -248,7 +304,8 @@ def f1_bwd(x, w1, z, du, dv, dq, dk, out: Optional[dict] = None) -> dict:
         out = dict(dx=torch.empty_like(x), dw1=torch.empty(4 * D, d_in, dtype=torch.float32, device=x.device),
                    db1=torch.empty(4 * D, dtype=torch.float32, device=x.device), ws=workspace(n, x.device),
                    status=_status(x.device))
-    st = capi.LIB.hstu_f1_bwd(T, d_in, D, _p(x), _p(w1), _p(z), _p(du), _p(dv), _p(dq), _p(dk), _p(out["dx"]),
+    st = capi.LIB.hstu_f1_bwd(T, d_in, D, _p(x), _p(w1), _p(z), _p(du), _p(dv), _p(dq), _p(dk), _p(dx_add),
+                              _p(out["dx"]),
                               _p(out["dw1"]), _p(out["db1"]), _p(out["ws"]), out["ws"].numel(),
                               _p(out.get("status")), _stream())
     capi.check(st, "hstu_f1_bwd")

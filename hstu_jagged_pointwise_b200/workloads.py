@@ -395,6 +395,32 @@ def make_projection(T: int, d_in: int, D: int, d_out: Optional[int] = None, seed
         z=randn(gen, (T, 4 * D), dtype, 2.0), name=name)
 
 
+@dataclass
+class LayerWorkload:
+    """Inputs of a whole HSTU layer: the attention workload (offsets, timestamps, masks, rab
+    tables, LayerNorm affine) plus X [T, d_model], the f1 / f2 weights and dL/d out."""
+    attn: Workload
+    d_model: int
+    x: torch.Tensor           # [T, d_model] bf16
+    w1: torch.Tensor          # [4D, d_model] bf16
+    b1: torch.Tensor          # [4D] fp32
+    w2: torch.Tensor          # [d_model, D] bf16
+    b2: torch.Tensor          # [d_model] fp32
+    g_out: torch.Tensor       # [T, d_model] bf16
+
+
+def make_layer(attn: Workload, d_model: int, seed: int = 0) -> LayerWorkload:
+    """Adds layer inputs to an attention workload (its q, k, v, u are then produced by f1)."""
+    gen = torch.Generator().manual_seed(seed + 707)
+    D = attn.D
+    return LayerWorkload(attn=attn, d_model=d_model, x=randn(gen, (attn.T, d_model), torch.bfloat16),
+                         w1=randn(gen, (4 * D, d_model), torch.bfloat16, d_model ** -0.5),
+                         b1=randn(gen, (4 * D,), torch.float32, 0.1),
+                         w2=randn(gen, (d_model, D), torch.bfloat16, D ** -0.5),
+                         b2=randn(gen, (d_model,), torch.float32, 0.1),
+                         g_out=randn(gen, (attn.T, d_model), torch.bfloat16))
+
+
 def projection_large(seed: int = 0, device: str = "cpu") -> ProjWorkload:
     """The large layer's projections: 262,144 tokens, d_model 1024 = 8 heads x 128."""
     return make_projection(262144, 1024, 1024, 1024, seed=seed, device=device, name="proj_T262144_d1024")

@@ -326,12 +326,13 @@ HSTU_API size_t hstu_f2_bwd_workspace_bytes(int32_t T, int32_t d_out);
 
 /* Backward of hstu_f1_fwd for the U, V, Q, K gradients du, dv, dq, dk [T, D]
  * (z = the forward's Z).  dZ = dAct * SiLU'(Z) is kept in bf16 in the
- * workspace; dx = dZ W1 [T, d_in] (bf16); dw1 = dZ^T X [4D, d_in] and
+ * workspace; dx = dZ W1 (+ dx_add [T, d_in] when not NULL, e.g. the gradient
+ * arriving through a residual connection) [T, d_in] (bf16); dw1 = dZ^T X [4D, d_in] and
  * db1 = column sums of the stored dZ [4D] in fp32, overwritten.  dw1 sums split-K tiles
  * with atomics (last-bit order effects); db1 is deterministic.  d_in and D
  * multiples of 32, 4D <= 8192. */
 HSTU_API int hstu_f1_bwd(int32_t T, int32_t d_in, int32_t D, const void* x, const void* w1, const void* z,
-                  const void* du, const void* dv, const void* dq, const void* dk,
+                  const void* du, const void* dv, const void* dq, const void* dk, const void* dx_add,
                   void* dx, float* dw1, float* db1, void* workspace, size_t workspace_bytes,
                   int32_t* device_status, void* stream);
 

@@ -11,7 +11,9 @@ Tolerances.
   with only those roundings already reaches 0.05-0.12 x RMS on heavy-tailed
   elements (o_pre = LN(Y) * U reaches ~16 x RMS, where one bf16 rounding is
   0.06; dK of a key seen by 300 queries inherits the cancellation of dY.V).
-  The allowance is computed from the oracle alone, never from the CUDA path.
+  The allowance is computed from the oracle alone, never from the CUDA path.  A composed
+  layer (f1 -> attention -> f2) compounds the storage points of its steps; its relative
+  bound is 5e-3 plus twice the storage chain's own relative deviation from the exact one.
 Integer work (offsets, masks, index decisions) is compared bit-exactly.
 """
 from __future__ import annotations
@@ -46,13 +48,18 @@ def bf16(x) -> np.ndarray:
     return torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
 
 
-def assert_bf16(got, ref, name, storage=None):
+def assert_bf16(got, ref, name, storage=None, chain=False):
+    """chain=True (composed layers, where the bf16 storage points of several steps compound):
+    the relative bound also gets twice the storage chain's own relative deviation."""
     rel, mx, rms = errors(got, ref)
     allowance = 0.0
+    rel_bound = BF16_REL
     if storage is not None:
         allowance = 2.0 * float(np.abs(_np(storage) - _np(ref)).max()) if np.asarray(ref).size else 0.0
+        if chain:
+            rel_bound += 2.0 * errors(storage, ref)[0]
     assert np.all(np.isfinite(_np(got))), f"{name}: non-finite output"
-    assert rel <= BF16_REL, f"{name}: rel Frobenius {rel:.3e} > {BF16_REL}"
+    assert rel <= rel_bound, f"{name}: rel Frobenius {rel:.3e} > {rel_bound:.3e}"
     bound = BF16_MAXABS_RMS * rms + allowance + 1e-30
     assert mx <= bound, (f"{name}: max abs {mx:.3e} > 3e-2 x RMS {rms:.3e} + storage allowance "
                          f"{allowance:.3e}")

@@ -140,7 +140,7 @@ def test_projections_reject_bad_arguments_before_launch():
     assert capi.LIB.hstu_f1_bwd_workspace_bytes(4, 4096) == 0                 # 4D above 8192
     assert capi.LIB.hstu_f1_bwd_workspace_bytes(4, 64) > 0
     assert capi.LIB.hstu_f2_bwd_workspace_bytes(4, 64) > 0
-    assert capi.LIB.hstu_f1_bwd(4, 64, 64, *([a] * 11), 16, None, None) == capi.HSTU_ERR_WORKSPACE
+    assert capi.LIB.hstu_f1_bwd(4, 64, 64, *([a] * 12), 16, None, None) == capi.HSTU_ERR_WORKSPACE
     assert capi.LIB.hstu_f2_bwd(4, 64, 64, *([a] * 7), 16, None, None) == capi.HSTU_ERR_WORKSPACE
 
 

@@ -439,6 +439,69 @@ def test_projections_large_sampled():
 
 
 # ----------------------------------------------------------------------------
+# a whole HSTU layer: f1 -> attention -> Norm * U -> f2 (+ X), forward and backward
+# ----------------------------------------------------------------------------
+
+def _layer_chain(lw, store):
+    """The layer through the oracle.  store=False: exact (float64 between the steps);
+    store=True: the values rounded to bf16 wherever the library stores them."""
+    import copy
+    r = bf16 if store else (lambda a: np.asarray(a, np.float64))
+    a = lw.attn
+    D = a.D
+    z, u, v, q, k = oracle.f1_fwd(lw.x, lw.w1, lw.b1, D)
+    aw = copy.copy(a)
+    aw.q, aw.k, aw.v, aw.u = (torch.as_tensor(r(t)) for t in (q, k, v, u))
+    if store:
+        sf = storage_fwd(aw)
+        o_pre = sf["o_pre"]
+    else:
+        _, o_pre, _, _ = oracle.layer_fwd(aw)
+    out = r(oracle.f2_fwd(o_pre, lw.w2, lw.b2, lw.x))
+    d_o_pre, dw2, db2 = oracle.f2_bwd(o_pre, lw.w2, lw.g_out)
+    aw.grad = torch.as_tensor(r(d_o_pre))
+    g = storage_bwd(aw) if store else oracle.layer_bwd(aw)
+    dz, dx, dw1, db1 = oracle.f1_bwd(lw.x, lw.w1, r(z), g["du"], g["dv"], g["dq"], g["dk"])
+    if store:
+        dzb = bf16(dz)
+        w1 = oracle.f32(lw.w1).astype(np.float64)
+        dx = dzb @ w1
+        dw1 = dzb.T @ oracle.f32(lw.x).astype(np.float64)
+        db1 = dzb.sum(0)
+    dx = r(dx + oracle.f32(lw.g_out))
+    return dict(out=out, dx=dx, dw1=dw1, db1=db1, dw2=dw2, db2=db2, d_rab_pos=g["d_rab_pos"],
+                d_rab_time=g["d_rab_time"], d_ln_gamma=g["dgamma"], d_ln_beta=g["dbeta"])
+
+
+@pytest.mark.parametrize("kind", ["causal", "mtgr"])
+def test_full_layer_forward_backward(kind):
+    from hstu_jagged_pointwise_b200 import ops
+    if kind == "causal":
+        a = W.make_causal([1, 127, 129, 300], H=2, d=64, seed=41, random_affine=True, with_grad=True)
+    else:
+        a = W.with_group_norm(W.make_mtgr([24, 2], [100, 190], [10, 0], [20, 70], H=2, d=64, seed=42,
+                                          random_affine=True, with_grad=True), seed=43)
+    lw = W.make_layer(a, d_model=96, seed=44)
+    c = {n: getattr(lw, n).cuda() for n in ("x", "w1", "b1", "w2", "b2", "g_out")}
+    prm = dict(w1=c["w1"], b1=c["b1"], w2=c["w2"], b2=c["b2"], rab_pos=a.rab_pos.cuda(),
+               rab_time=a.rab_time.cuda(), ln_gamma=a.gamma.cuda(), ln_beta=a.beta.cuda())
+    tg = torch.as_tensor(np.asarray(a.token_group, np.uint8)).cuda() if a.n_groups > 1 else None
+    layer = ops.HSTULayer(torch.as_tensor(a.offsets).cuda(), torch.as_tensor(a.ts).cuda(), 96, a.H, a.d, a.alpha,
+                          a.max_len, mask_kind=a.kind,
+                          n_static=None if a.n_static is None else torch.as_tensor(a.n_static).cuda(),
+                          n_realtime=None if a.n_realtime is None else torch.as_tensor(a.n_realtime).cuda(),
+                          n_groups=a.n_groups, token_group=tg)
+    fwd = layer.forward(c["x"], prm)
+    grads = layer.backward(fwd, c["g_out"], prm)
+    torch.cuda.synchronize()
+    assert layer.check_device_error() == 0
+    ref, st = _layer_chain(lw, False), _layer_chain(lw, True)
+    assert_bf16(fwd["out"], ref["out"], "out", st["out"], chain=True)
+    for k in ("dx", "dw1", "db1", "dw2", "db2", "d_rab_pos", "d_rab_time", "d_ln_gamma", "d_ln_beta"):
+        assert_bf16(grads[k], ref[k], k, st[k], chain=True)
+
+
+# ----------------------------------------------------------------------------
 # the data step: Stochastic Length sampling, gathers, token-balanced bins (bit-exact)
 # ----------------------------------------------------------------------------
 
