@@ -866,6 +866,8 @@ def main():
                     help="total tokens of the large-layer workload (smaller values for profiling)")
     ap.add_argument("--only-proj", action="store_true",
                     help="run only the f1 / f2 projections leg and print its JSON (profiling aid)")
+    ap.add_argument("--only-layer", action="store_true",
+                    help="run only the whole-layer leg and print its JSON (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -881,6 +883,14 @@ def main():
         line = run_proj(args, world, rank)
         if rank == 0:
             print(json.dumps({"projections": line}), flush=True)
+        return
+    if args.only_layer:
+        torch.cuda.set_device(local)
+        w = W.large_layer(seed=args.seed + rank, total=args.tokens)
+        P = causal_pairs(w.lengths) * w.H
+        line = run_full_layer(args, world, w, 12 * w.d * P)
+        if rank == 0:
+            print(json.dumps({"full_layer": line}), flush=True)
         return
     line, w = run_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -72,9 +72,12 @@ def attn_workspace_bytes(dims: capi.HstuDims, mask_kind: int, is_bwd: bool, n_gr
     return int(n)
 
 
-def workspace(nbytes: int, device) -> torch.Tensor:
-    """A zeroed byte buffer usable as workspace (torch allocations are 256-byte aligned)."""
-    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+def workspace(nbytes: int, device, zero: bool = True) -> torch.Tensor:
+    """A byte buffer usable as workspace (torch allocations are 256-byte aligned); zeroed for
+    the attention workspaces, whose control block must start clear."""
+    if zero:
+        return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
 class Layer:
@@ -166,7 +169,9 @@ class HSTULayer:
         O_pre = Norm(Y) * U                              (LayerNorm or Group LayerNorm)
         out = O_pre W2^T + b2 (+ X when residual)        (f2)
     Parameters are passed per call as a dict: w1 [4D, d_model], b1 [4D] or None, w2 [d_model, D],
-    b2 [d_model] or None, rab_pos, rab_time, ln_gamma, ln_beta (bf16 weights, fp32 the rest)."""
+    b2 [d_model] or None, rab_pos, rab_time, ln_gamma, ln_beta (bf16 weights, fp32 the rest).
+    Outputs and workspaces are allocated on the first call and reused by later calls, so the
+    tensors a call returns are overwritten by the next call of the same kind."""
 
     def __init__(self, seq_offsets, timestamps, d_model: int, H: int, d: int, alpha: float, max_seq_len: int,
                  mask_kind: str = "causal", n_static=None, n_realtime=None, n_groups: int = 1, token_group=None,
@@ -176,14 +181,17 @@ class HSTULayer:
                           ln_eps=ln_eps, n_groups=n_groups, token_group=token_group)
         self.d_model, self.D, self.residual = d_model, H * d, residual
         self._status = []
+        self._buf = {}                                     # outputs reused from step to step
 
     def forward(self, x, params: dict) -> dict:
         """Returns out and the tensors the backward needs."""
         _need(x, "x", torch.bfloat16)
-        f = f1_fwd(x, params["w1"], params.get("b1"), self.D)
-        a = self.attn.forward(f["q"], f["k"], f["v"], f["u"], params["rab_pos"], params["rab_time"],
-                              params["ln_gamma"], params["ln_beta"])
-        o = f2_fwd(a["o_pre"], params["w2"], params.get("b2"), residual=x if self.residual else None)
+        b = self._buf
+        f = b["f1"] = f1_fwd(x, params["w1"], params.get("b1"), self.D, out=b.get("f1"))
+        a = b["attn"] = self.attn.forward(f["q"], f["k"], f["v"], f["u"], params["rab_pos"], params["rab_time"],
+                                          params["ln_gamma"], params["ln_beta"], out=b.get("attn"))
+        o = b["f2"] = f2_fwd(a["o_pre"], params["w2"], params.get("b2"), residual=x if self.residual else None,
+                             out=b.get("f2"))
         self._status = [f["status"], o["status"]]
         return dict(out=o["out"], x=x, f1=f, attn=a)
 
@@ -191,11 +199,13 @@ class HSTULayer:
         """Gradients of every input and parameter for d_out = dL/d out."""
         _need(d_out, "d_out", torch.bfloat16)
         f, a = saved["f1"], saved["attn"]
-        g2 = f2_bwd(a["o_pre"], params["w2"], d_out)
-        ga = self.attn.backward(f["q"], f["k"], f["v"], f["u"], params["rab_pos"], params["rab_time"],
-                                params["ln_gamma"], params["ln_beta"], a, g2["d_o_pre"])
-        g1 = f1_bwd(saved["x"], params["w1"], f["z"], ga["du"], ga["dv"], ga["dq"], ga["dk"],
-                    dx_add=d_out if self.residual else None)
+        b = self._buf
+        g2 = b["b2"] = f2_bwd(a["o_pre"], params["w2"], d_out, out=b.get("b2"))
+        ga = b["battn"] = self.attn.backward(f["q"], f["k"], f["v"], f["u"], params["rab_pos"], params["rab_time"],
+                                             params["ln_gamma"], params["ln_beta"], a, g2["d_o_pre"],
+                                             out=b.get("battn"))
+        g1 = b["b1"] = f1_bwd(saved["x"], params["w1"], f["z"], ga["du"], ga["dv"], ga["dq"], ga["dk"],
+                              dx_add=d_out if self.residual else None, out=b.get("b1"))
         self._status += [g2["status"], g1["status"]]
         return dict(dx=g1["dx"], dw1=g1["dw1"], db1=g1["db1"], dw2=g2["dw2"], db2=g2["db2"],
                     d_rab_pos=ga["d_rab_pos"], d_rab_time=ga["d_rab_time"], d_ln_gamma=ga["d_gamma"],
@@ -260,7 +270,7 @@ class MFalcon:
 # ----------------------------------------------------------------------------
 
 def _status(dev):
-    return torch.zeros(1, dtype=torch.int32, device=dev)
+    return torch.empty(1, dtype=torch.int32, device=dev)    # the entry points set it to 0 first
 
 
 def f1_fwd(x, w1, b1, D: int, save_z: bool = True, out: Optional[dict] = None) -> dict:
@@ -302,7 +312,7 @@ def f1_bwd(x, w1, z, du, dv, dq, dk, out: Optional[dict] = None, dx_add=None) ->
     if out is None:
         n = capi.LIB.hstu_f1_bwd_workspace_bytes(T, D)
         out = dict(dx=torch.empty_like(x), dw1=torch.empty(4 * D, d_in, dtype=torch.float32, device=x.device),
-                   db1=torch.empty(4 * D, dtype=torch.float32, device=x.device), ws=workspace(n, x.device),
+                   db1=torch.empty(4 * D, dtype=torch.float32, device=x.device), ws=workspace(n, x.device, False),
                    status=_status(x.device))
     st = capi.LIB.hstu_f1_bwd(T, d_in, D, _p(x), _p(w1), _p(z), _p(du), _p(dv), _p(dq), _p(dk), _p(dx_add),
                               _p(out["dx"]),
@@ -319,7 +329,7 @@ def f2_bwd(o_pre, w2, g, out: Optional[dict] = None) -> dict:
     if out is None:
         n = capi.LIB.hstu_f2_bwd_workspace_bytes(T, d_out)
         out = dict(d_o_pre=torch.empty_like(o_pre), dw2=torch.empty(d_out, D, dtype=torch.float32, device=g.device),
-                   db2=torch.empty(d_out, dtype=torch.float32, device=g.device), ws=workspace(n, g.device),
+                   db2=torch.empty(d_out, dtype=torch.float32, device=g.device), ws=workspace(n, g.device, False),
                    status=_status(g.device))
     st = capi.LIB.hstu_f2_bwd(T, D, d_out, _p(o_pre), _p(w2), _p(g), _p(out["d_o_pre"]), _p(out["dw2"]),
                               _p(out["db2"]), _p(out["ws"]), out["ws"].numel(), _p(out.get("status")), _stream())
