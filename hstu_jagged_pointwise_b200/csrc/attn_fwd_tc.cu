@@ -499,7 +499,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                         for (int e = 0; e < 2; e++) w_crel[lane + 32 * e] = (int32_t)(tj[e] - cmin);
                     }
-                } else {
+                } else if (wcls != 0) {
 #pragma unroll
                     for (int e = 0; e < 2; e++) w_cts[lane + 32 * e] = tj[e];
                 }
@@ -512,10 +512,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll 1
                 for (int cc = 0; cc < 2; cc++) {
                     const int c = 2 * g + cc;                // 32-column chunk of the tile
+                    uint32_t pk[16];
+                    if (wcls == 0) {
+                        // nothing visible (masked or past the sequence): P = 0, S is never read
+#pragma unroll
+                        for (int e = 0; e < 16; e++) pk[e] = 0u;
+                        tmem_st16(tmem + lane_base + kSCol + 32 * c, pk);
+                        continue;
+                    }
                     uint32_t v[32];
                     tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
                     tmem_ld_wait(v);
-                    uint32_t pk[16];
                     const float* dg = w_diag + 31 - (KIND != HSTU_KIND_CAUSAL && pm == kPosCol ? 0 : lane) + 32 * cc;
                     const int32_t* cr = w_crel + 32 * cc;
                     if (pm == kPosUniform && tm == kTimeUniform) fwd_block<kBiasConst>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
