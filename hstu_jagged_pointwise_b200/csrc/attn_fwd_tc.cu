@@ -107,15 +107,18 @@ __device__ __forceinline__ void flag_timeout(const FwdParams& p, volatile int* a
 // BM = kBiasConst: one bias c0 for the whole block; kBiasRow: bias from the
 // diagonal row (dg points at this lane's entry for the chunk's first key);
 // kBiasRowTime: diagonal row plus a per-element time bucket from cr, the chunk's
-// 32-bit key times relative to the tile's smallest one.  Three variants only, so
-// that the elementwise code stays small enough for the instruction cache.
-enum { kBiasConst = 0, kBiasRow = 1, kBiasRowTime = 2 };
+// 32-bit key times relative to the tile's smallest one.  kBiasRowTwo: the block spans
+// two time buckets, told apart by one compare against thr (t_lo / t_hi are their half
+// biases).  Four small variants, so that the elementwise code stays small enough for
+// the instruction cache.
+enum { kBiasConst = 0, kBiasRow = 1, kBiasRowTime = 2, kBiasRowTwo = 3 };
 
 template <int BM>
 __device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* dg, const int32_t* cr, int32_t a_i,
-                                          float c0, const float* rth, int nbm1, uint32_t (&pk)[16]) {
+                                          float c0, const float* rth, int nbm1, uint32_t (&pk)[16],
+                                          uint32_t thr = 0, float t_lo = 0.f, float t_hi = 0.f) {
     int32_t b[32];
-    if (BM == kBiasRowTime) {
+    if (BM == kBiasRowTime || BM == kBiasRowTwo) {
         const int4* b4 = reinterpret_cast<const int4*>(cr);
 #pragma unroll
         for (int e = 0; e < 8; e++) {
@@ -131,6 +134,7 @@ __device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* 
             const int k = e + f;
             float hb = BM == kBiasConst ? c0 : dg[k];
             if (BM == kBiasRowTime) hb += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
+            if (BM == kBiasRowTwo) hb += (uint32_t)abs(b[k] - a_i) >= thr ? t_hi : t_lo;
             const float h = fmaf(__uint_as_float(v[k]), 0.5f, hb);
             pv[f] = fmaf(h, tanh_approx(h), h);
         }
@@ -527,6 +531,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const int32_t* cr = w_crel + 32 * cc;
                     if (pm == kPosUniform && tm == kTimeUniform) fwd_block<kBiasConst>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else if (pm >= 0 && tm == kTimeUniform) fwd_block<kBiasRow>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                    else if (pm >= 0 && tm == kTimeTwo)
+                        fwd_block<kBiasRowTwo>(v, dg, cr, a_i, c0, s_rth, nbm1, pk, tc.thr, s_rth[tc.tb_lo], s_rth[tc.tb_hi]);
                     else if (pm >= 0 && tm >= 0) fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else {
                         // element by element: MTGR candidates, ragged key tiles, int64-wide time spans
