@@ -424,24 +424,49 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int n_done = 0;
             int t = next_tile(-1);
             load_tj(t);
-            for (; t < n_kt; t = next_tile(t)) {
+            for (int t_next; t < n_kt; t = t_next) {
                 const int n0 = t * kTileN + 64 * g;         // first key of this warp's half
                 __syncwarp();
                 int64_t tj[2] = {tj_next[0], tj_next[1]};
-                load_tj(next_tile(t));
-                int64_t cmin = INT64_MAX, cmax = INT64_MIN;
+                t_next = next_tile(t);
+                load_tj(t_next);
+                // time range of the warp's keys: 32-bit offsets from the first key's time and
+                // two warp reductions; the 64-bit shuffle tree only when the span needs it
+                const int64_t ref = __shfl_sync(kFull, (long long)tj[0], 0);
+                int32_t dmn = INT32_MAX, dmx = INT32_MIN;
+                bool fits = true;
 #pragma unroll
                 for (int e = 0; e < 2; e++) {
                     const int j = n0 + lane + 32 * e;
                     if (j < s.Lk) {
-                        cmin = min(cmin, tj[e]);
-                        cmax = max(cmax, tj[e]);
+                        const int64_t dt = tj[e] - ref;
+                        fits = fits && dt > INT32_MIN && dt < INT32_MAX;
+                        dmn = min(dmn, (int32_t)dt);
+                        dmx = max(dmx, (int32_t)dt);
                     }
                 }
+                int64_t cmin, cmax;
+                if (__all_sync(kFull, fits)) {
+                    dmn = __reduce_min_sync(kFull, dmn);
+                    dmx = __reduce_max_sync(kFull, dmx);
+                    cmin = dmn == INT32_MAX ? INT64_MAX : ref + dmn;
+                    cmax = dmx == INT32_MIN ? INT64_MIN : ref + dmx;
+                } else {
+                    cmin = INT64_MAX;
+                    cmax = INT64_MIN;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    cmin = min(cmin, (int64_t)__shfl_xor_sync(kFull, (long long)cmin, o));
-                    cmax = max(cmax, (int64_t)__shfl_xor_sync(kFull, (long long)cmax, o));
+                    for (int e = 0; e < 2; e++) {
+                        const int j = n0 + lane + 32 * e;
+                        if (j < s.Lk) {
+                            cmin = min(cmin, tj[e]);
+                            cmax = max(cmax, tj[e]);
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        cmin = min(cmin, (int64_t)__shfl_xor_sync(kFull, (long long)cmin, o));
+                        cmax = max(cmax, (int64_t)__shfl_xor_sync(kFull, (long long)cmax, o));
+                    }
                 }
                 // ---- classify this warp's block: 32 rows x 64 columns
                 int pm = -1, tm = -1;
