@@ -196,8 +196,9 @@ def test_gln_bad_group_flagged():
 # M-FALCON
 # ----------------------------------------------------------------------------
 
-def test_mfalcon_small_and_microbatch_invariance():
-    w = W.make_mfalcon([0, 1, 200, 300, 129], [3, 5, 130, 300, 1], H=2, d=128, seed=11, b_m=256,
+@pytest.mark.parametrize("head_dim", [128, 64])
+def test_mfalcon_small_and_microbatch_invariance(head_dim):
+    w = W.make_mfalcon([0, 1, 200, 300, 129], [3, 5, 130, 300, 1], H=2, d=head_dim, seed=11, b_m=256,
                        alpha=301.0)
     y_ref, o_ref = oracle.mfalcon_layer(w)
     st = storage_mfalcon(w)
