@@ -152,6 +152,9 @@ __device__ __forceinline__ void diag_sums(const float (&zf)[C], float& dlo, floa
 // times relative to the warp's smallest key time.  Two variants only, so that the
 // elementwise code stays small enough for the instruction cache.  CONST: one bias c0
 // for the whole block (position and time bias uniform), no diagonal row.
+//
+// Queries go in pairs through packed fp32 arithmetic.  With h = z / 2, t = tanh(h) and
+// p = 1 + t:  SiLU(z) = h p  and  2 SiLU'(z) = p + SiLU(z) (1 - t).
 template <bool TV, int C, bool CONST = false>
 __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_t (&dp)[C], const float* dg, float c0,
                                           bool pos_diag, float& dlo, float& dhi, const int32_t* qr, int32_t a_j,
@@ -166,44 +169,52 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_
             q[4 * e] = v.x; q[4 * e + 1] = v.y; q[4 * e + 2] = v.z; q[4 * e + 3] = v.w;
         }
     }
-    // pass 1: independent per-element chains (no cross-lane operations)
+    const float2 one2 = make_float2(1.f, 1.f);
     float zf[C];
+    float2 acc2 = make_float2(0.f, 0.f);
+    // TV: run-length sums of the time-bias gradient along the row (the bucket changes
+    // rarely), each run sent to its bucket by a predicated reduction when it ends
+    int cur_t = 0;
+    float acc_t = 0.f;
 #pragma unroll
     for (int e = 0; e < C; e += 2) {
-        float av[2];
-#pragma unroll
-        for (int f = 0; f < 2; f++) {
-            const int k = e + f;
-            float hb = CONST ? c0 : dg[-k];
-            if (TV) hb += rth[time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1)];
-            const float h = fmaf(__uint_as_float(sv[k]), 0.5f, hb);
-            const float th = tanh_approx(h);
-            av[f] = fmaf(h, th, h);                                        // SiLU(z)
-            const float g2 = fmaf(h, fmaf(-th, th, 1.f), th + 1.f);        // 2 SiLU'(z)
-            zf[k] = __uint_as_float(dp[k]) * g2;
+        float2 hb = CONST ? make_float2(c0, c0) : make_float2(dg[-e], dg[-e - 1]);
+        int tb0 = 0, tb1 = 0;
+        if (TV) {
+            tb0 = time_bucket_u32((uint32_t)abs(q[e] - a_j), nbm1);
+            tb1 = time_bucket_u32((uint32_t)abs(q[e + 1] - a_j), nbm1);
+            hb.x += rth[tb0];
+            hb.y += rth[tb1];
         }
-        pa[e >> 1] = pack_bf16x2(av[0], av[1]);
-        pz[e >> 1] = pack_bf16x2(zf[e], zf[e + 1]);
-    }
-    // pass 2: gradient bookkeeping on finished values
-#pragma unroll
-    for (int k = 0; k < C; k++) acc += zf[k];
-    if (TV) {
-        // the bucket changes rarely along a row: run-length sums, flushed on change
-        int cur_t = time_bucket_u32((uint32_t)abs(q[0] - a_j), nbm1);
-        float acc_t = 0.f;
-#pragma unroll
-        for (int k = 0; k < C; k++) {
-            const int tb = time_bucket_u32((uint32_t)abs(q[k] - a_j), nbm1);
-            if (tb != cur_t) {
-                red_add_f32(&g_rt[cur_t], acc_t);
-                cur_t = tb;
-                acc_t = 0.f;
+        const float2 h = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), make_float2(0.5f, 0.5f), hb);
+        const float2 t = make_float2(tanh_approx(h.x), tanh_approx(h.y));
+        const float2 p1 = add2(t, one2);
+        const float2 av = mul2(h, p1);                                  // SiLU(z)
+        const float2 g2 = fma2(av, sub2(one2, t), p1);                 // 2 SiLU'(z)
+        const float2 z2 = mul2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), g2);
+        zf[e] = z2.x;
+        zf[e + 1] = z2.y;
+        acc2 = add2(acc2, z2);
+        pa[e >> 1] = pack_bf16x2(av.x, av.y);
+        pz[e >> 1] = pack_bf16x2(z2.x, z2.y);
+        if (TV) {
+            if (e == 0) {
+                cur_t = tb0;
+                acc_t = z2.x;
+            } else {
+                const bool f0 = tb0 != cur_t;
+                red_add_f32_if(f0, &g_rt[cur_t], acc_t);
+                acc_t = f0 ? z2.x : acc_t + z2.x;
+                cur_t = tb0;
             }
-            acc_t += zf[k];
+            const bool f1 = tb1 != cur_t;
+            red_add_f32_if(f1, &g_rt[cur_t], acc_t);
+            acc_t = f1 ? z2.y : acc_t + z2.y;
+            cur_t = tb1;
         }
-        red_add_f32(&g_rt[cur_t], acc_t);
     }
+    if (TV) red_add_f32(&g_rt[cur_t], acc_t);
+    acc += acc2.x + acc2.y;
     if (pos_diag) diag_sums<C>(zf, dlo, dhi);
 }
 
