@@ -543,18 +543,34 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int32_t a_j = (int32_t)(ts_j - kmin);
             const int n_qt = (s.L + kTileM - 1) / kTileM;
             int n_done = 0;
-            for (int t = next_visible<KIND>(s, -1, n_qt); ok && t < n_qt; t = next_visible<KIND>(s, t, n_qt)) {
+            int t = next_visible<KIND>(s, -1, n_qt);
+            while (ok && t < n_qt) {
+                const int t_nx = next_visible<KIND>(s, t, n_qt);
                 for (int hh = 0; hh < 2; hh++) {
                     const int i0 = t * kTileM + 64 * hh + C * g;    // first query of this warp's block
                     __syncwarp();
                     const int iq = i0 + lane % C;                  // lanes past C repeat the block
-                    const int64_t tq = iq < s.L ? p.ts[s.off0 + iq] : 0;
+                    const bool q_ok = iq < s.L;
+                    const int64_t tq = q_ok ? p.ts[s.off0 + iq] : 0;
                     if (lane < C) w_qts[lane] = tq;
-                    int64_t qmin = iq < s.L ? tq : INT64_MAX, qmax = iq < s.L ? tq : INT64_MIN;
+                    // time range of the block's queries: 32-bit offsets from the warp's smallest
+                    // key time and two warp reductions; the 64-bit shuffle tree only when the
+                    // span needs it
+                    const int64_t dq = (int64_t)((uint64_t)tq - (uint64_t)kmin);
+                    int64_t qmin, qmax;
+                    if (__all_sync(kFull, !q_ok || (dq > INT32_MIN && dq < INT32_MAX))) {
+                        const int32_t rmn = __reduce_min_sync(kFull, q_ok ? (int32_t)dq : INT32_MAX);
+                        const int32_t rmx = __reduce_max_sync(kFull, q_ok ? (int32_t)dq : INT32_MIN);
+                        qmin = rmn == INT32_MAX ? INT64_MAX : kmin + rmn;
+                        qmax = rmx == INT32_MIN ? INT64_MIN : kmin + rmx;
+                    } else {
+                        qmin = q_ok ? tq : INT64_MAX;
+                        qmax = q_ok ? tq : INT64_MIN;
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
-                        qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
+                        for (int o = 16; o > 0; o >>= 1) {
+                            qmin = min(qmin, (int64_t)__shfl_xor_sync(kFull, (long long)qmin, o));
+                            qmax = max(qmax, (int64_t)__shfl_xor_sync(kFull, (long long)qmax, o));
+                        }
                     }
                     // ---- classify this warp's block: 32 keys x C queries
                     int wcls = 0;
@@ -587,7 +603,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 w_diag[k] = masked ? kMaskedHalfBias
                                                    : 0.5f * s_rp[min(max(dl, -(p.P - 1)), p.P - 1) + p.P - 1] + tadd;
                             }
-                            if (tm != kTimeUniform && lane < C) w_qrel[lane] = (int32_t)(tq - kmin);
+                            if (tm != kTimeUniform && lane < C) w_qrel[lane] = (int32_t)dq;
                         }
                     }
                     __syncwarp();
@@ -723,6 +739,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                 }
                 n_done++;
+                t = t_nx;
             }
             if (!ok) break;
             // ---------------- epilogue: dV, dK rows of this key tile (D / kEwGroups columns per warp)
