@@ -154,7 +154,8 @@ __device__ __forceinline__ void diag_sums(const float (&zf)[C], float& dlo, floa
 // for the whole block (position and time bias uniform), no diagonal row.
 //
 // Queries go in pairs through packed fp32 arithmetic.  With h = z / 2, t = tanh(h) and
-// p = 1 + t:  SiLU(z) = h p  and  2 SiLU'(z) = p + SiLU(z) (1 - t).
+// p = 1 + t:  SiLU(z) = h + h t = h p  and  2 SiLU'(z) = p + SiLU(z) (1 - t).  SiLU is
+// rounded as in the forward (one fused multiply-add), so A matches the forward's P.
 template <bool TV, int C, bool CONST = false>
 __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_t (&dp)[C], const float* dg, float c0,
                                           bool pos_diag, float& dlo, float& dhi, const int32_t* qr, int32_t a_j,
@@ -189,7 +190,7 @@ __device__ __forceinline__ void bwd_block(const uint32_t (&sv)[C], const uint32_
         const float2 h = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), make_float2(0.5f, 0.5f), hb);
         const float2 t = make_float2(tanh_approx(h.x), tanh_approx(h.y));
         const float2 p1 = add2(t, one2);
-        const float2 av = mul2(h, p1);                                  // SiLU(z)
+        const float2 av = fma2(h, t, h);                                // SiLU(z)
         const float2 g2 = fma2(av, sub2(one2, t), p1);                 // 2 SiLU'(z)
         const float2 z2 = mul2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), g2);
         zf[e] = z2.x;

@@ -126,19 +126,21 @@ __device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* 
             b[4 * e] = x.x; b[4 * e + 1] = x.y; b[4 * e + 2] = x.z; b[4 * e + 3] = x.w;
         }
     }
+    // key pairs through packed fp32 arithmetic: h = z / 2, SiLU(z) = h + h tanh(h)
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        float pv[2];
+        float hb[2];
 #pragma unroll
         for (int f = 0; f < 2; f++) {
             const int k = e + f;
-            float hb = BM == kBiasConst ? c0 : dg[k];
-            if (BM == kBiasRowTime) hb += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
-            if (BM == kBiasRowTwo) hb += (uint32_t)abs(b[k] - a_i) >= thr ? t_hi : t_lo;
-            const float h = fmaf(__uint_as_float(v[k]), 0.5f, hb);
-            pv[f] = fmaf(h, tanh_approx(h), h);
+            hb[f] = BM == kBiasConst ? c0 : dg[k];
+            if (BM == kBiasRowTime) hb[f] += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
+            if (BM == kBiasRowTwo) hb[f] += (uint32_t)abs(b[k] - a_i) >= thr ? t_hi : t_lo;
         }
-        pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+        const float2 h = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), make_float2(0.5f, 0.5f),
+                              make_float2(hb[0], hb[1]));
+        const float2 a = fma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
+        pk[e >> 1] = pack_bf16x2(a.x, a.y);
     }
 }
 
