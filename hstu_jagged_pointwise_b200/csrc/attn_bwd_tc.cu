@@ -541,7 +541,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 kmax = max(kmax, (int64_t)__shfl_xor_sync(kFull, (long long)kmax, o));
                 warp_keys += __shfl_xor_sync(kFull, warp_keys, o);
             }
-            const int32_t a_j = (int32_t)(ts_j - kmin);
+            const int32_t a_j = (int32_t)(uint32_t)((uint64_t)ts_j - (uint64_t)kmin);
+            // |kmin| < 2^62: then tq - kmin cannot wrap to a small value unless it is small
+            const bool kmin_ok = (uint64_t)kmin + (1ull << 62) < (1ull << 63);
             const int n_qt = (s.L + kTileM - 1) / kTileM;
             int n_done = 0;
             int t = next_visible<KIND>(s, -1, n_qt);
@@ -559,7 +561,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     // span needs it
                     const int64_t dq = (int64_t)((uint64_t)tq - (uint64_t)kmin);
                     int64_t qmin, qmax;
-                    if (__all_sync(kFull, !q_ok || (dq > INT32_MIN && dq < INT32_MAX))) {
+                    if (__all_sync(kFull, kmin_ok && (!q_ok || (dq > INT32_MIN && dq < INT32_MAX)))) {
                         const int32_t rmn = __reduce_min_sync(kFull, q_ok ? (int32_t)dq : INT32_MAX);
                         const int32_t rmx = __reduce_max_sync(kFull, q_ok ? (int32_t)dq : INT32_MIN);
                         qmin = rmn == INT32_MAX ? INT64_MAX : kmin + rmn;

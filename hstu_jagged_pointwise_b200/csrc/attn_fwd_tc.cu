@@ -436,12 +436,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // two warp reductions; the 64-bit shuffle tree only when the span needs it
                 const int64_t ref = __shfl_sync(kFull, (long long)tj[0], 0);
                 int32_t dmn = INT32_MAX, dmx = INT32_MIN;
-                bool fits = true;
+                // |ref| < 2^62: then tj - ref cannot wrap to a small value unless it is small
+                bool fits = (uint64_t)ref + (1ull << 62) < (1ull << 63);
 #pragma unroll
                 for (int e = 0; e < 2; e++) {
                     const int j = n0 + lane + 32 * e;
                     if (j < s.Lk) {
-                        const int64_t dt = tj[e] - ref;
+                        const int64_t dt = (int64_t)((uint64_t)tj[e] - (uint64_t)ref);
                         fits = fits && dt > INT32_MIN && dt < INT32_MAX;
                         dmn = min(dmn, (int32_t)dt);
                         dmx = max(dmx, (int32_t)dt);
@@ -528,14 +529,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (pm >= 0) {
                     if (tm != kTimeUniform) {
 #pragma unroll
-                        for (int e = 0; e < 2; e++) w_crel[lane + 32 * e] = (int32_t)(tj[e] - cmin);
+                        for (int e = 0; e < 2; e++) w_crel[lane + 32 * e] = (int32_t)(uint32_t)((uint64_t)tj[e] - (uint64_t)cmin);
                     }
                 } else if (wcls != 0) {
 #pragma unroll
                     for (int e = 0; e < 2; e++) w_cts[lane + 32 * e] = tj[e];
                 }
                 __syncwarp();
-                const int32_t a_i = (int32_t)(ts_i - cmin);
+                const int32_t a_i = (int32_t)(uint32_t)((uint64_t)ts_i - (uint64_t)cmin);
                 ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
                 if (!__all_sync(kFull, ok)) { ok = false; break; }
                 s_use++;

@@ -169,6 +169,24 @@ def _check_layer_fwd_bwd(w, f32=False):
     assert_bf16(out["d_beta"], ref["dbeta"], "d_beta", sb["dbeta"])
 
 
+def test_bf16_extreme_timestamps_forward_backward():
+    """Timestamps near both ends of int64 inside every warp's keys and queries, so 64-bit time
+    differences wrap around: the kernels' 32-bit time offsets must fall back to 64 bits.  The
+    time-bias table is large and q, k small, so one wrong bucket shows far above tolerance."""
+    lo, hi = np.iinfo(np.int64).min, np.iinfo(np.int64).max
+    i = np.arange(300)
+    ts_a = np.where(i % 2 == 0, hi - (i % 7), lo + (i % 5)).astype(np.int64)
+    ts_b = W.increasing_ts(np.random.default_rng(3), 200)
+    ts_b[::37] = lo + 3
+    ts_c = np.where(i[:150] % 3 == 0, hi, -(i[:150] % 11)).astype(np.int64)
+    w = W.make_causal([300, 200, 150], H=2, d=128, seed=31, ts_list=[ts_a, ts_b, ts_c], random_affine=True,
+                      with_grad=True)
+    w.q = (w.q.float() * 0.25).to(w.dtype)
+    w.k = (w.k.float() * 0.25).to(w.dtype)
+    w.rab_time = torch.randn(w.rab_time.shape, generator=torch.Generator().manual_seed(32)) * 4.0
+    _check_layer_fwd_bwd(w)
+
+
 @pytest.mark.parametrize("d", [128, 64])
 def test_gln_mtgr_forward_backward(d):
     """MTGR rows with groups profile / behaviour / real-time / candidate from the segments."""
