@@ -476,10 +476,3 @@ def large_layer(seed: int = 0, total: int = 262144, with_grad: bool = True) -> W
     lengths = lognormal_lengths(rng, total)
     return make_causal(lengths, H=8, d=128, dtype=torch.bfloat16, seed=seed + 404,
                        with_grad=with_grad, name=f"large_layer_T{total}_H8_d128")
-
-
-CONFIGS = {0: tiny_fp32, 1: training_sl, 2: mtgr_medium, 3: mfalcon_ranking, 4: large_layer}
-
-
-def make_config(k: int, seed: int = 0, **kw) -> Workload:
-    return CONFIGS[k](seed=seed, **kw)
