@@ -86,3 +86,57 @@ def test_pins_catch_planted_mistake(name, old, new, tmp_path, monkeypatch):
         except AssertionError:
             return
     pytest.fail(f"no pin caught the planted mistake {name}")
+
+
+# ----------------------------------------------------------------------------
+# the oracle's Python functions (Group LayerNorm, projections, Stochastic Length, packer)
+# ----------------------------------------------------------------------------
+
+PY_MUTATIONS = [
+    ("gln_forward_one_affine_row", "o[r], mu[r], rs[r] = ln_mul_fwd(y[r], u[r], g[k], b[k], eps)",
+     "o[r], mu[r], rs[r] = ln_mul_fwd(y[r], u[r], g[0], b[0], eps)"),
+    ("gln_backward_one_affine_row", "dy[r], du[r], dg[k], db[k] = ln_mul_bwd(y[r], u[r], g[k], b[k], gr[r], eps)",
+     "dy[r], du[r], dg[k], db[k] = ln_mul_bwd(y[r], u[r], g[0], b[0], gr[r], eps)"),
+    ("norm_ignores_groups", 'if getattr(w, "n_groups", 1) > 1:\n        return gln_mul_fwd',
+     'if False:\n        return gln_mul_fwd'),
+    ("f1_split_q_k_swapped", "return z, a[:, :D], a[:, D:2 * D], a[:, 2 * D:3 * D], a[:, 3 * D:]",
+     "return z, a[:, :D], a[:, D:2 * D], a[:, 3 * D:], a[:, 2 * D:3 * D]"),
+    ("f1_bias_dropped", "z = z + _as_f64(b1)", "z = z"),
+    ("f1_silu_grad_wrong", "* s * (1 + z * (1 - s))", "* s * (1 + z * s)"),
+    ("f2_residual_dropped", "o = o + _as_f64(residual)", "o = o"),
+    ("f2_bias_grad_mean", "return g @ _as_f64(w2), g.T @ _as_f64(o_pre), g.sum(0)",
+     "return g @ _as_f64(w2), g.T @ _as_f64(o_pre), g.mean(0)"),
+    ("splitmix64_constant", "np.uint64(0xBF58476D1CE4E5B9)", "np.uint64(0xBF58476D1CE4E5B8)"),
+    ("sl_kept_events_out_of_order", "keep = np.sort(order[:cap])", "keep = order[:cap]"),
+    ("pack_bin_by_start", "mid2 = 2 * off[b] + (off[b + 1] - off[b])", "mid2 = 2 * off[b]"),
+    ("pack_weights_by_tokens", "weights = np.array([(start[r + 1] - start[r]) / B if B else 0.0",
+     "weights = np.array([(tokens[r]) / T if B else 0.0"),
+]
+
+
+def _mutated_module(src: str):
+    import types
+    mod = types.ModuleType("oracle_mutated")
+    mod.__file__ = oracle.__file__
+    exec(compile(src, oracle.__file__, "exec"), mod.__dict__)
+    mod._lib = oracle.lib()
+    return mod
+
+
+def test_unmodified_python_copy_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(pins, "oracle", _mutated_module(open(oracle.__file__).read()))
+    for name, call in _pin_calls():
+        call()
+
+
+@pytest.mark.parametrize("name,old,new", PY_MUTATIONS, ids=[m[0] for m in PY_MUTATIONS])
+def test_pins_catch_planted_python_mistake(name, old, new, monkeypatch):
+    src = open(oracle.__file__).read()
+    assert src.count(old) == 1, f"the text to mutate for {name} is not unique in the oracle"
+    monkeypatch.setattr(pins, "oracle", _mutated_module(src.replace(old, new)))
+    for pin_name, call in _pin_calls():
+        try:
+            call()
+        except Exception:
+            return
+    pytest.fail(f"no pin caught the planted mistake {name}")

@@ -399,6 +399,28 @@ def test_group_layer_norm_with_equal_groups_is_layer_norm():
     np.testing.assert_allclose(db.sum(0), db1, rtol=1e-11, atol=1e-12)
 
 
+def test_layer_norm_step_uses_each_tokens_group_row():
+    """The layer's Norm step with token groups, against float64 torch autograd of layer_norm with
+    each token's own affine row, applied to the oracle's attention output."""
+    w = W.with_group_norm(W.make_causal([7, 20, 13], H=2, d=16, dtype=torch.float32, seed=21, with_grad=True),
+                          seed=22, groups=3)
+    y, o, _, _ = oracle.layer_fwd(w)
+    ref = oracle.layer_bwd(w)
+    ty = torch.tensor(np.asarray(y, dtype=np.float64))
+    tu = torch.tensor(oracle.f32(w.u), dtype=torch.float64, requires_grad=True)
+    tg = torch.tensor(oracle.f32(w.gamma), dtype=torch.float64, requires_grad=True)
+    tb = torch.tensor(oracle.f32(w.beta), dtype=torch.float64, requires_grad=True)
+    ty.requires_grad_(True)
+    idx = torch.tensor(np.asarray(w.token_group).astype(np.int64))
+    out = (torch.nn.functional.layer_norm(ty, (w.D,), eps=w.eps) * tg[idx] + tb[idx]) * tu
+    out.backward(torch.tensor(oracle.f32(w.grad), dtype=torch.float64))
+    np.testing.assert_allclose(o, out.detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ref["dy"], ty.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(ref["du"], tu.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(ref["dgamma"], tg.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(ref["dbeta"], tb.grad.numpy(), rtol=1e-10, atol=1e-11)
+
+
 def test_mtgr_token_groups_follow_segments():
     w = W.with_group_norm(W.make_mtgr([3, 2], [5, 0], [2, 4], [3, 1], H=1, d=32, dtype=torch.float32, seed=5))
     np.testing.assert_array_equal(w.token_group, [0, 0, 0, 1, 1, 1, 1, 1, 2, 2, 3, 3, 3, 0, 0, 2, 2, 2, 2, 3])
@@ -521,6 +543,26 @@ def test_pack_balanced_contiguous_and_balanced():
     s2, t2, w2 = oracle.pack_balanced(off_eq, 4)
     np.testing.assert_array_equal(s2, [0, 16, 32, 48, 64])
     np.testing.assert_allclose(w2, 0.25)
+
+
+def test_pack_balanced_worked_example():
+    """Sequences of 10, 20, 5 and 65 tokens (T = 100) into 2 bins, worked by hand from the
+    midpoint rule: midpoints 5, 20, 32.5 and 67.5 give bins floor(2 m / 100) = 0, 0, 0, 1."""
+    start, tokens, weights = oracle.pack_balanced([0, 10, 30, 35, 100], 2)
+    np.testing.assert_array_equal(start, [0, 3, 4])
+    np.testing.assert_array_equal(tokens, [35, 65])
+    np.testing.assert_allclose(weights, [0.75, 0.25])
+
+
+def test_pack_balanced_weights_give_the_mean_over_sequences():
+    """The weighted sum of per-bin mean gradients is the mean of the per-sequence gradients."""
+    rng = np.random.default_rng(11)
+    lens = rng.integers(1, 3000, size=97)
+    off = np.concatenate([[0], np.cumsum(lens)])
+    start, _, weights = oracle.pack_balanced(off, 8)
+    g = rng.normal(size=(97, 5))
+    total = sum(weights[r] * g[start[r]:start[r + 1]].mean(0) for r in range(8) if start[r + 1] > start[r])
+    np.testing.assert_allclose(total, g.mean(0), rtol=1e-12, atol=1e-14)
 
 
 # ----------------------------------------------------------------------------
