@@ -40,6 +40,11 @@ MUTATIONS = [
     ("time_grad_scaled", "lt[ti] += dz;", "lt[ti] += dz * 1.0001;"),
     ("mfalcon_positions_swapped", "z += (double)rab_pos[pos_index(n, j, P)];",
      "z += (double)rab_pos[pos_index(j, n, P)];"),
+    ("mfalcon_self_term_dropped", "for (int64_t j = 0; j <= n; j++) {", "for (int64_t j = 0; j < n; j++) {"),
+    ("mfalcon_self_value_from_history", ": cand_v + c * ldv + h * dv;", ": hist_v + h0 * ldv + h * dv;"),
+    ("mfalcon_alpha_dropped", "for (int e = 0; e < dv; e++) out[e] /= alpha;", ";"),
+    ("pos_grad_scaled", "lp[pi] += dz;", "lp[pi] += 0.5 * dz;"),
+    ("static_sees_realtime", "if (ci == 0) return cj == 0;", "if (ci == 0) return cj <= 1;"),
 ]
 
 
