@@ -70,14 +70,15 @@ def test_partition_covers_and_balances():
     assert shard.partition_sequences([], 2) == [[], []]
 
 
-def test_two_rank_gloo_matches_single_process():
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_match_single_process(world):
     import oracle
     w = _global_batch()
     ref = oracle.layer_bwd(w)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in procs]
@@ -118,7 +119,8 @@ def _balanced_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_token_balanced_bins_give_the_batch_mean_gradient():
+@pytest.mark.parametrize("world", [2, 3])
+def test_token_balanced_bins_give_the_batch_mean_gradient(world):
     """MTGR's dynamic batches: each rank takes one token-balanced bin (different sample
     counts), and the weighted all-reduce of per-rank mean gradients is the batch mean."""
     import oracle
@@ -127,7 +129,7 @@ def test_two_rank_token_balanced_bins_give_the_batch_mean_gradient():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_balanced_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_balanced_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in procs]
@@ -136,9 +138,9 @@ def test_two_rank_token_balanced_bins_give_the_batch_mean_gradient():
         assert p.exitcode == 0
     seqs = sorted(b for _, sq, _, _ in res for b in sq)
     assert seqs == list(range(w.B))
-    assert len({len(sq) for _, sq, _, _ in res}) == 2            # the bins hold different sample counts
+    assert len({len(sq) for _, sq, _, _ in res}) > 1             # the bins hold different sample counts
     for _, _, tok, grads in res:
-        assert abs(tok - w.T / 2) <= w.lengths.max()
+        assert abs(tok - w.T / world) <= w.lengths.max()
         for k, rk in (("d_rab_pos", "d_rab_pos"), ("d_rab_time", "d_rab_time"), ("d_gamma", "dgamma"),
                       ("d_beta", "dbeta")):
             np.testing.assert_allclose(grads[k], ref[rk] / w.B, rtol=1e-12, atol=1e-14)
