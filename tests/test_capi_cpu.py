@@ -196,3 +196,19 @@ def test_fwd_noalloc_rejects_oversized_problems_on_the_host():
     assert st == capi.HSTU_ERR_WORKSPACE
     st = capi.LIB.hstu_attn_fwd_noalloc(None, C.byref(mask), *([None] * 15), None)
     assert st == capi.HSTU_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """No CPU fallback: with the shared library absent, importing the binding or the ops layer
+    raises and names the missing file."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "hstu_jagged_pointwise_b200"
+    pkg.mkdir()
+    for f in ("__init__.py", "capi.py", "ops.py", "shard.py", "workloads.py"):
+        shutil.copy(os.path.join(ROOT, "hstu_jagged_pointwise_b200", f), pkg / f)
+    for mod in ("hstu_jagged_pointwise_b200.capi", "hstu_jagged_pointwise_b200.ops"):
+        r = subprocess.run([sys.executable, "-c", f"import {mod}"], cwd=tmp_path, capture_output=True, text=True,
+                           env={**os.environ, "PYTHONPATH": str(tmp_path)})
+        assert r.returncode != 0 and "libhstu_b200.so is missing" in r.stderr, r.stderr[-800:]
