@@ -67,8 +67,24 @@ def _declare(L):
                                        _i32, _i32, _p, _p, _f64, _p, _p, _p, _p, _p, _p]
     L.hstu_oracle_mfalcon.argtypes = [_i32, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p,
                                       _p, _i32, _p, _i32, _f64, _i64, _p, _p]
+    L.hstu_oracle_set_bf16_operands.argtypes = [C.c_int]
     L.hstu_oracle_num_threads.restype = C.c_int
     L.hstu_oracle_set_num_threads.argtypes = [C.c_int]
+
+
+class bf16_operands:
+    """Inside this context the oracle's attention (forward, backward, M-FALCON) rounds the
+    operands a bf16 tensor-core implementation must hold in bf16 -- A = SiLU(z) before it
+    multiplies V or dY, and dz before it multiplies K or Q -- to bf16, round to nearest
+    even.  An error model used to derive tolerances, never a reference by itself."""
+
+    def __enter__(self):
+        lib().hstu_oracle_set_bf16_operands(1)
+        return self
+
+    def __exit__(self, *exc):
+        lib().hstu_oracle_set_bf16_operands(0)
+        return False
 
 
 def num_threads() -> int:

@@ -103,6 +103,27 @@ static int visible(int kind, int64_t i, int64_t j, int64_t S, int64_t R, const i
 
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
+/* Error model of a bf16 tensor-core implementation (off by default; used only to
+ * derive tolerances).  When on, the operands that such an implementation must hold
+ * in bf16 to multiply them on the tensor cores are rounded to bf16 (round to
+ * nearest even): A = SiLU(z) before it multiplies V (forward) and dY (dV), and dz
+ * before it multiplies K (dQ) and Q (dK).  The rab gradients keep the unrounded dz. */
+static int g_bf16_operands = 0;
+
+void hstu_oracle_set_bf16_operands(int on) { g_bf16_operands = on ? 1 : 0; }
+
+static double round_bf16(double x) {
+    float f = (float)x;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) != 0x7f800000u) u += 0x7fffu + ((u >> 16) & 1u);
+    u &= 0xffff0000u;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double operand(double x) { return g_bf16_operands ? round_bf16(x) : x; }
+
 /* derivative of z * sigmoid(z) */
 static double silu_grad(double z) {
     double s = 1.0 / (1.0 + exp(-z));
@@ -188,7 +209,7 @@ void hstu_oracle_attn_fwd(int32_t B, const int32_t* offsets, int32_t H, int32_t 
             for (int c = 0; c < dqk; c++) z += (double)qi[c] * (double)kj[c];
             z += (double)rab_pos[pos_index(token_pos(kind, i, S, R), token_pos(kind, j, S, R), P)];
             z += (double)rab_time[time_bucket(tsb[i], tsb[j], nb)];
-            double a = silu(z);
+            double a = operand(silu(z));
             const float* vj = v + (s0 + j) * ldv + h * dv;
             for (int c = 0; c < dv; c++) out[c] += a * (double)vj[c];
         }
@@ -308,13 +329,14 @@ void hstu_oracle_attn_bwd(int32_t B, const int32_t* offsets, int32_t H, int32_t 
                     for (int c = 0; c < dv; c++) dA += dyi[c] * (double)vj[c];
                     dA /= alpha;
                     double dz = dA * silu_grad(z);
-                    double a = silu(z) / alpha;
+                    double a = operand(silu(z)) / alpha;
+                    double dzo = operand(dz);
                     double* dqi = dq + (s0 + i) * ldq + h * dqk;
                     double* dkj = dk + (s0 + j) * ldq + h * dqk;
                     double* dvj = dvv + (s0 + j) * ldv + h * dv;
                     for (int c = 0; c < dqk; c++) {
-                        dqi[c] += dz * (double)kj[c];
-                        dkj[c] += dz * (double)qi[c];
+                        dqi[c] += dzo * (double)kj[c];
+                        dkj[c] += dzo * (double)qi[c];
                     }
                     for (int c = 0; c < dv; c++) dvj[c] += a * dyi[c];
                     lp[pi] += dz;
@@ -365,7 +387,7 @@ void hstu_oracle_mfalcon(int32_t B, const int32_t* hist_off, const int32_t* cand
             for (int e = 0; e < dqk; e++) z += (double)qc[e] * (double)kj[e];
             z += (double)rab_pos[pos_index(n, j, P)];
             z += (double)rab_time[time_bucket(cand_ts[c], tj, nb)];
-            double a = silu(z);
+            double a = operand(silu(z));
             for (int e = 0; e < dv; e++) out[e] += a * (double)vj[e];
         }
         for (int e = 0; e < dv; e++) out[e] /= alpha;

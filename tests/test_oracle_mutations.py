@@ -31,8 +31,10 @@ MUTATIONS = [
      "if (kind == ORACLE_MTGR && i >= S + R) return S + R;"),
     ("alpha_dropped_forward", "for (int c = 0; c < dv; c++) out[c] /= alpha;", ";"),
     ("silu_grad_wrong", "return s * (1.0 + z * (1.0 - s));", "return s * (1.0 + z * s);"),
-    ("alpha_dropped_backward", "double a = silu(z) / alpha;", "double a = silu(z);"),
-    ("dk_transposed_operand", "dkj[c] += dz * (double)qi[c];", "dkj[c] += dz * (double)kj[c];"),
+    ("alpha_dropped_backward", "double a = operand(silu(z)) / alpha;", "double a = operand(silu(z));"),
+    ("dk_transposed_operand", "dkj[c] += dzo * (double)qi[c];", "dkj[c] += dzo * (double)kj[c];"),
+    ("bf16_model_dz_not_rounded", "double dzo = operand(dz);", "double dzo = dz;"),
+    ("bf16_model_rounds_rab_sums", "lp[pi] += dz;", "lp[pi] += dzo;"),
     ("unbiased_variance",
      "        var /= D;\n        double rs = 1.0 / sqrt(var + eps);\n        for (int c = 0; c < D; c++) {\n            double ln",
      "        var /= (D - 1);\n        double rs = 1.0 / sqrt(var + eps);\n        for (int c = 0; c < D; c++) {\n            double ln"),

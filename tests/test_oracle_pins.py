@@ -106,6 +106,34 @@ def test_bidirectional_no_rab_equals_matmul_route():
     assert sum(L) == w.T
 
 
+def test_bf16_operand_model_equals_matmul_route_with_torch_rounding():
+    """The oracle's bf16 error model (used only for tolerances): all pairs visible, zero
+    rab, so A = SiLU(Q K^T) and dz = (dY V^T / alpha) * SiLU'(Q K^T); with the model on,
+    Y = bf16(A) V / alpha, dV = bf16(A)^T dY / alpha, dQ = bf16(dz) K, dK = bf16(dz)^T Q,
+    and the rab gradients keep the unrounded dz.  bf16() here is torch's rounding."""
+    w = W.make_mtgr(n_profile=[2], n_long=[30], n_rt=[0], n_cand=[0], H=1, d=8, dtype=torch.float32,
+                    seed=13, alpha=5.0)
+    _zero_rab(w)
+    dy = np.random.default_rng(14).standard_normal((w.T, 8))
+    with oracle.bf16_operands():
+        y = oracle.attn_fwd(w)
+        dq, dk, dv, drp, drt = oracle.attn_bwd(w, dy)
+    q, k, v = (oracle.f32(t).astype(np.float64) for t in (w.q, w.k, w.v))
+    s = q @ k.T
+    a = bf16_round(silu_np(s)).astype(np.float64)
+    sig = expit(s)
+    dz = (dy @ v.T / 5.0) * (sig + s * sig * (1 - sig))
+    dzb = bf16_round(dz).astype(np.float64)
+    np.testing.assert_allclose(y, a @ v / 5.0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dv, a.T @ dy / 5.0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dq, dzb @ k, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk, dzb.T @ q, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(drp.sum(), dz.sum(), rtol=1e-11)
+    assert not np.allclose(a, silu_np(s), rtol=1e-6)          # the rounding really happened
+    # and the model is off again outside the context
+    np.testing.assert_allclose(oracle.attn_fwd(w), silu_np(s) @ v / 5.0, rtol=1e-12, atol=1e-12)
+
+
 def test_causal_no_rab_equals_tril_matmul_route():
     w = _zero_rab(W.make_causal([1, 12, 40], H=3, d=16, dtype=torch.float32, seed=5, alpha=40.0))
     y = oracle.attn_fwd(w)
