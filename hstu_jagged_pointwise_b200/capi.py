@@ -33,7 +33,7 @@ EXPORTS = (
     "hstu_attn_fwd_noalloc", "hstu_mfalcon_cache_history", "hstu_attn_fwd_gln", "hstu_attn_bwd_gln",
     "hstu_attn_workspace_bytes_gln", "hstu_f1_fwd", "hstu_f2_fwd", "hstu_f1_bwd_workspace_bytes",
     "hstu_f2_bwd_workspace_bytes", "hstu_f1_bwd", "hstu_f2_bwd", "hstu_sl_sample", "hstu_gather_rows",
-    "hstu_pack_balanced",
+    "hstu_pack_balanced", "hstu_debug_set_wait_fault", "hstu_attn_bwd_dy",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20   # HSTU_NOALLOC_SCRATCH_BYTES
@@ -84,6 +84,8 @@ def load():
     lib.hstu_attn_fwd_noalloc.restype = C.c_int
     lib.hstu_attn_bwd.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec)] + [P] * 23 + [S, P]
     lib.hstu_attn_bwd.restype = C.c_int
+    lib.hstu_attn_bwd_dy.argtypes = [C.POINTER(HstuDims), C.POINTER(HstuMaskSpec)] + [P] * 14 + [S, P]
+    lib.hstu_attn_bwd_dy.restype = C.c_int
     NS = C.POINTER(HstuNormSpec)
     lib.hstu_attn_workspace_bytes_gln.argtypes = [C.POINTER(HstuDims), i32, i32, i32]
     lib.hstu_attn_workspace_bytes_gln.restype = S
@@ -123,6 +125,8 @@ def load():
     lib.hstu_status_string.restype = C.c_char_p
     lib.hstu_version.argtypes = []
     lib.hstu_version.restype = C.c_char_p
+    lib.hstu_debug_set_wait_fault.argtypes = [C.c_int64, i32]
+    lib.hstu_debug_set_wait_fault.restype = C.c_int
     lib.hstu_profile_enable.argtypes = [i32]
     lib.hstu_profile_enable.restype = C.c_int
     lib.hstu_profile_read.argtypes = [i32, P, P]
@@ -153,6 +157,24 @@ def profile_read() -> dict:
         raise HstuError(k, "hstu_profile_read")
     return {LIB.hstu_profile_kind_name(i).decode(): (int(launches[i]), float(ms[i]))
             for i in range(min(k, n)) if launches[i] > 0}
+
+
+class wait_fault:
+    """Context manager around hstu_debug_set_wait_fault (test hook): inside it, the
+    pipelined kernels' main-loop waits give up after `limit_cycles` SM cycles and,
+    with withhold=True, each CTA's producer withholds its first tile load so that
+    those waits run out.  Normal operation is restored on exit."""
+
+    def __init__(self, limit_cycles: int, withhold: bool = True):
+        self.limit, self.withhold = int(limit_cycles), bool(withhold)
+
+    def __enter__(self):
+        check(LIB.hstu_debug_set_wait_fault(self.limit, 1 if self.withhold else 0), "hstu_debug_set_wait_fault")
+        return self
+
+    def __exit__(self, *exc):
+        check(LIB.hstu_debug_set_wait_fault(0, 0), "hstu_debug_set_wait_fault")
+        return False
 
 
 def check(status: int, where: str) -> None:

@@ -249,6 +249,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int np = 2 * p.P - 1;
+    const long long wl = p.dbg.limit;   // main-loop wait limit (SM cycles)
     for (int i = tid; i < np; i += kThreads) s_rp[i] = p.rab_pos[i];
     for (int i = tid; i < p.nb; i += kThreads) {
         s_rt[i] = p.rab_time[i];
@@ -288,7 +289,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         while (ok) {
             const int slot = it_use & 1;
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort);
+                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort, wl);
                 if (ok) {
                     const int idx = atomicAdd(&p.ctrl->counter, 1);
                     s_item[slot] = idx < p.ctrl->n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
@@ -306,7 +307,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (it.x < 0) break;
             if (lane == 0) {
                 const KvItem s = load_kv_item<KIND>(p, it);
-                ok = mbar_wait(&bars[kKVEmpty], (kv_use & 1) ^ 1, s_abort);
+                ok = mbar_wait(&bars[kKVEmpty], (kv_use & 1) ^ 1, s_abort, wl);
+                if (ok && p.dbg.withhold_first_load && kv_use == 0) {
+                    // test hook: withhold this CTA's first K/V tile, so the waits for it run out
+                    wait_for_abort(s_abort, 2 * wl);
+                    ok = false;
+                }
                 if (ok) {
                     mbar_arrive_expect_tx(&bars[kKVFull], 2 * L::kTile);
                     for (int pn = 0; pn < kPanels; pn++) {
@@ -333,14 +339,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         t_pf++;
                     }
                     for (int hh = 0; ok && hh < 2; hh++) {
-                        ok = mbar_wait(&bars[kQEmpty0 + hh], (q_use[hh] & 1) ^ 1, s_abort);
+                        ok = mbar_wait(&bars[kQEmpty0 + hh], (q_use[hh] & 1) ^ 1, s_abort, wl);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&bars[kQFull0 + hh], L::kHalf);
                         for (int pn = 0; pn < kPanels; pn++)
                             tma_load_2d(sm + (hh ? L::q1 : L::q0) + pn * kHalfPanel, &tm_q, &bars[kQFull0 + hh],
                                         s.h * D + pn * 64, s.off0 + t * kTileM + 64 * hh);
                         q_use[hh]++;
-                        ok = mbar_wait(&bars[kDYEmpty0 + hh], (dy_use[hh] & 1) ^ 1, s_abort);
+                        ok = mbar_wait(&bars[kDYEmpty0 + hh], (dy_use[hh] & 1) ^ 1, s_abort, wl);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&bars[kDYFull0 + hh], L::kHalf);
                         for (int pn = 0; pn < kPanels; pn++)
@@ -381,7 +387,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
         // S^T_h once Q_h of the tile is loaded
         auto issue_s = [&](int hh) -> bool {
-            const bool w = mbar_wait(&bars[kQFull0 + hh], q_use[hh] & 1, s_abort);
+            const bool w = mbar_wait(&bars[kQFull0 + hh], q_use[hh] & 1, s_abort, wl);
             q_use[hh]++;
             if (!w) return false;
             tc_fence_after();
@@ -396,8 +402,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         };
         // dP^T_h once dY'_h is loaded and the previous dQ^T_h has left the columns
         auto issue_dp = [&](int hh) -> bool {
-            bool w = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort);
-            if (w) w = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort);
+            bool w = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort, wl);
+            if (w) w = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort, wl);
             if (!w) return false;
             dy_use[hh]++;
             tc_fence_after();
@@ -413,9 +419,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         };
         // dQ^T_h, dV and dK products of half hh once its elementwise step is done
         auto issue_prods = [&](int hh, bool init) -> bool {
-            if (!mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort)) return false;
+            if (!mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort, wl)) return false;
             p_use[hh]++;
-            if (init && !mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort)) return false;
+            if (init && !mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort, wl)) return false;
             tc_fence_after();
             // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys); first,
             // so that its drain overlaps the two products below
@@ -450,7 +456,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
                 if (ok) it = s_item[slot];
             }
             ok = __shfl_sync(kFull, ok, 0);
@@ -461,7 +467,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (lane == 0) {
                 const KvItem s = load_kv_item<KIND>(p, it);
                 const int n_qt = (s.L + kTileM - 1) / kTileM;
-                ok = mbar_wait(&bars[kKVFull], kv_use & 1, s_abort);
+                ok = mbar_wait(&bars[kKVFull], kv_use & 1, s_abort, wl);
                 kv_use++;
                 int t = next_visible<KIND>(s, -1, n_qt);
                 bool first = true;
@@ -486,7 +492,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (ok) {
                     tc_commit(&bars[kKVEmpty]);
-                    if (first) ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort);
+                    if (first) ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort, wl);
                 }
                 if (ok) {
                     acc_use++;
@@ -521,7 +527,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
-            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             const int4 it = s_item[slot];
             it_use++;
@@ -610,8 +616,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                     __syncwarp();
-                    ok = mbar_wait(&bars[kSFull0 + hh], s_use[hh] & 1, s_abort);
-                    if (ok) ok = mbar_wait(&bars[kDZEmpty0 + hh], (dz_use[hh] & 1) ^ 1, s_abort);
+                    ok = mbar_wait(&bars[kSFull0 + hh], s_use[hh] & 1, s_abort, wl);
+                    if (ok) ok = mbar_wait(&bars[kDZEmpty0 + hh], (dz_use[hh] & 1) ^ 1, s_abort, wl);
                     if (!__all_sync(kFull, ok)) { ok = false; break; }
                     s_use[hh]++;
                     dz_use[hh]++;
@@ -716,7 +722,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // 16*wq .. +15 in the first 16 lanes of the lane quarter.  Queries past the
                 // sequence end carry exact zeros (their dZ is zero).
                 for (int hh = 0; hh < 2; hh++) {
-                    ok = mbar_wait(&bars[kDQFull0 + hh], dq_use[hh] & 1, s_abort);
+                    ok = mbar_wait(&bars[kDQFull0 + hh], dq_use[hh] & 1, s_abort, wl);
                     if (!__all_sync(kFull, ok)) { ok = false; break; }
                     dq_use[hh]++;
                     tc_fence_after();
@@ -746,7 +752,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             if (!ok) break;
             // ---------------- epilogue: dV, dK rows of this key tile (D / kEwGroups columns per warp)
-            ok = mbar_wait(&bars[kAccFull], acc_use & 1, s_abort);
+            ok = mbar_wait(&bars[kAccFull], acc_use & 1, s_abort, wl);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             acc_use++;
             tc_fence_after();
@@ -797,14 +803,8 @@ template <int KIND, int D>
 cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdy, const CUtensorMap& tdq, const BwdParams& p, int grid,
                        cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<KIND, D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             BwdSmem<D>::alloc(kMaxPos));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = ensure_smem_limit((const void*)attn_bwd_tc_kernel<KIND, D>, BwdSmem<D>::alloc(kMaxPos));
+    if (e != cudaSuccess) return e;
     prof_begin(kProfAttnBwdTc, s);
     attn_bwd_tc_kernel<KIND, D><<<grid, kThreads, BwdSmem<D>::alloc(p.P), s>>>(tq, tk, tv, tdy, tdq, p);
     prof_end(kProfAttnBwdTc, s);
@@ -819,6 +819,22 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
         o.x = pack_bf16x2(v.x, v.y);
         o.y = pack_bf16x2(v.z, v.w);
         dst[i] = o;
+    }
+}
+
+__global__ void scale_bf16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, float scale,
+                                  long long n8) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+         i += (long long)gridDim.x * blockDim.x) {
+        const uint4 v = src[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+            o[e] = pack_bf16x2(lo * scale, hi * scale);
+        }
+        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
@@ -856,6 +872,19 @@ cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
     HSTU_BWD_CASE(HSTU_KIND_MTGR, 64)
 #undef HSTU_BWD_CASE
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_scale_bf16(const __nv_bfloat16* src, __nv_bfloat16* dst, float scale, long long n,
+                              cudaStream_t s) {
+    const long long n8 = n / 8;   // n is a multiple of 8 (H*d with d in {64, 128})
+    long long blocks = (n8 + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    prof_begin(kProfScaleDy, s);
+    scale_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(src),
+                                                        reinterpret_cast<uint4*>(dst), scale, n8);
+    prof_end(kProfScaleDy, s);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t s) {

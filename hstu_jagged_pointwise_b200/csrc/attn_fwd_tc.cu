@@ -8,12 +8,13 @@
 // in the epilogue).  There is no softmax, so no running maximum and no
 // rescaling: P = SiLU(Z) is written once per tile and accumulated.
 //
-// One CTA = 6 warps, two CTAs per SM (each owns 256 TMEM columns and ~108 KB
+// One CTA = 10 warps, two CTAs per SM (each owns 256 TMEM columns and ~110 KB
 // of shared memory, so one CTA's elementwise phase overlaps the other's MMAs):
-//   warps 0-3  elementwise: TMEM S -> bias, mask, SiLU -> bf16 P back into TMEM;
+//   warps 0-7  elementwise (warp w: TMEM lane quarter w % 4, key half w / 4):
+//              TMEM S -> bias, mask, SiLU -> bf16 P back into TMEM;
 //              epilogue O/alpha -> global (and the M-FALCON self term)
-//   warp 4     producer: dynamic work fetch + TMA loads of Q, K, V tiles
-//   warp 5     MMA issuer: S = Q K^T (SS), O += P V (TS, P from TMEM)
+//   warp 8     producer: dynamic work fetch + TMA loads of Q, K, V tiles
+//   warp 9     MMA issuer: S = Q K^T (SS), O += P V (TS, P from TMEM)
 // TMEM columns: S/P at [0, 128), O at [128, 128 + D).
 // Every wait is bounded; on timeout the CTA records a status bit, drains its
 // copies and MMAs, frees TMEM and exits.
@@ -172,6 +173,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::abort_flag);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long wl = p.dbg.limit;   // main-loop wait limit (SM cycles)
 
     for (int i = tid; i < 2 * p.P - 1; i += kThreads) s_rp[i] = p.rab_pos[i];
     for (int i = tid; i < p.nb; i += kThreads) {
@@ -218,7 +220,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         while (ok) {
             const int slot = it_use & 1;
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort);
+                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort, wl);
                 if (ok) {
                     const int idx = atomicAdd(&p.ctrl->counter, 1);
                     const int4 it = idx < p.ctrl->n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
@@ -237,7 +239,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (it.x < 0) break;
             const Item s = load_item<KIND>(p, it);
             if (lane == 0) {
-                ok = mbar_wait(&bars[kQEmpty], (q_use & 1) ^ 1, s_abort);
+                ok = mbar_wait(&bars[kQEmpty], (q_use & 1) ^ 1, s_abort, wl);
+                if (ok && p.dbg.withhold_first_load && q_use == 0) {
+                    // test hook: withhold this CTA's first Q tile, so the waits for it run out
+                    wait_for_abort(s_abort, 2 * wl);
+                    ok = false;
+                }
                 if (ok) {
                     mbar_arrive_expect_tx(&bars[kQFull], L::kTileBytes);
                     for (int pn = 0; pn < kPanels; pn++)
@@ -259,13 +266,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         t_pf++;
                     }
                     const int y = s.kv0 + t * kTileN;
-                    ok = mbar_wait(&bars[kKEmpty], (k_use & 1) ^ 1, s_abort);
+                    ok = mbar_wait(&bars[kKEmpty], (k_use & 1) ^ 1, s_abort, wl);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bars[kKFull], L::kTileBytes);
                     for (int pn = 0; pn < kPanels; pn++)
                         tma_load_2d(sK + pn * kPanelBytes, &tm_k, &bars[kKFull], s.h * D + pn * 64, y);
                     k_use++;
-                    ok = mbar_wait(&bars[kVEmpty], (v_use & 1) ^ 1, s_abort);
+                    ok = mbar_wait(&bars[kVEmpty], (v_use & 1) ^ 1, s_abort, wl);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bars[kVFull], L::kTileBytes);
                     for (int pn = 0; pn < kPanels; pn++)
@@ -297,7 +304,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
                 if (ok) it = s_item[slot];
             }
             ok = __shfl_sync(kFull, ok, 0);
@@ -311,13 +318,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 int last = -1;
                 for (int t = 0; t < n_kt; t++)
                     if (kv_class<KIND>(s, t) != 0) last = t;
-                ok = mbar_wait(&bars[kQFull], q_use & 1, s_abort);
+                ok = mbar_wait(&bars[kQFull], q_use & 1, s_abort, wl);
                 q_use++;
                 tc_fence_after();
                 int n_done = 0;
                 for (int t = 0; ok && t <= last; t++) {
                     if (kv_class<KIND>(s, t) == 0) continue;
-                    ok = mbar_wait(&bars[kKFull], k_use & 1, s_abort);
+                    ok = mbar_wait(&bars[kKFull], k_use & 1, s_abort, wl);
                     if (!ok) break;
                     k_use++;
                     tc_fence_after();
@@ -329,14 +336,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tc_commit(&bars[kSFull]);
                     tc_commit(&bars[kKEmpty]);
                     if (t == last) tc_commit(&bars[kQEmpty]);
-                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort);
+                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort, wl);
                     if (!ok) break;
                     p_use++;
-                    ok = mbar_wait(&bars[kVFull], v_use & 1, s_abort);
+                    ok = mbar_wait(&bars[kVFull], v_use & 1, s_abort, wl);
                     if (!ok) break;
                     v_use++;
                     if (n_done == 0) {
-                        ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort);
+                        ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort, wl);
                         if (!ok) break;
                     }
                     tc_fence_after();
@@ -352,7 +359,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (ok && n_done == 0) {
                     tc_commit(&bars[kQEmpty]);
-                    ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort);
+                    ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort, wl);
                 }
                 if (ok) {
                     o_use++;
@@ -385,7 +392,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
-            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort);
+            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             const int4 it = s_item[slot];
             it_use++;
@@ -486,10 +493,30 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int r_hi = min(r0 + 31, s.row_end - 1);
                 // every row of the block is a candidate sharing one position
                 const bool rows_shared = KIND == HSTU_KIND_MFALCON || (KIND != HSTU_KIND_CAUSAL && r0 >= s.S + s.R);
-                // real-time / history rows against real-time / history keys: the mask is j <= i
+                // real-time / history rows against non-candidate keys: the mask is j <= i (a
+                // static key precedes every real-time row)
                 const bool causal_rows = KIND == HSTU_KIND_CAUSAL ||
                                          (KIND != HSTU_KIND_MFALCON && r0 >= s.S && r_hi < s.S + s.R &&
-                                          n0 >= s.S && n0 + 63 < s.S + s.R);
+                                          n0 < s.S + s.R);
+                // keys n0 + k with k >= jlim are masked for every row of the block: static rows
+                // against a key block that crosses the end of the static segment, real-time rows
+                // against one that crosses the end of the history
+                int jlim = 64;
+                if (KIND == HSTU_KIND_MTGR || KIND == HSTU_KIND_MFSEQ) {
+                    if (r_hi < s.S && n0 < s.S && n0 + 63 >= s.S && wcls != 0) {
+                        jlim = s.S - n0;
+                        wcls = 2;
+                    } else if (causal_rows && n0 + 63 >= s.S + s.R) {
+                        jlim = s.S + s.R - n0;
+                    }
+                }
+                // MTGR candidate rows against history keys: the timestamp filter passes every
+                // pair when the rows' earliest time is after the keys' latest, and no pair when
+                // the rows' latest time is at or before the keys' earliest
+                if (KIND == HSTU_KIND_MTGR && wcls == 1 && r0 >= s.S + s.R && n0 + 63 < s.S + s.R) {
+                    if (rmin > cmax) wcls = 2;
+                    else if (rmax <= cmin) wcls = 0;
+                }
                 const bool dense = wcls != 0 && n0 + 64 <= s.Lk && (wcls == 2 || causal_rows);
                 if (dense) {
                     tc = classify_time(rmin, rmax, cmin, cmax, p.nb);
@@ -537,7 +564,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 __syncwarp();
                 const int32_t a_i = (int32_t)(uint32_t)((uint64_t)ts_i - (uint64_t)cmin);
-                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort);
+                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort, wl);
                 if (!__all_sync(kFull, ok)) { ok = false; break; }
                 s_use++;
                 tc_fence_after();
@@ -562,7 +589,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     else if (pm >= 0 && tm == kTimeTwo)
                         fwd_block<kBiasRowTwo>(v, dg, cr, a_i, c0, s_rth, nbm1, pk, tc.thr, s_rth[tc.tb_lo], s_rth[tc.tb_hi]);
                     else if (pm >= 0 && tm >= 0) fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
-                    else {
+                    if (pm >= 0 && jlim - 32 * cc < 32) {
+                        // keys past the block's column limit: P = 0 (bf16 pairs, key 2e in the low half)
+                        const int lim = jlim - 32 * cc;
+#pragma unroll
+                        for (int e = 0; e < 16; e++)
+                            pk[e] &= 2 * e + 1 < lim ? 0xffffffffu : (2 * e < lim ? 0x0000ffffu : 0u);
+                    }
+                    if (pm < 0) {
                         // element by element: MTGR candidates, ragged key tiles, int64-wide time spans
                         float pv[32];
 #pragma unroll
@@ -614,7 +648,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 a_self = silu_fast(dot + rp_self + rt_zero);
                 vself = p.self_v + ro;
             }
-            ok = mbar_wait(&bars[kOFull], o_use & 1, s_abort);
+            ok = mbar_wait(&bars[kOFull], o_use & 1, s_abort, wl);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             o_use++;
             tc_fence_after();
@@ -671,14 +705,8 @@ template <int KIND, int D>
 cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t s) {
     const uint32_t smem = FwdSmem<D>::alloc(p.P);
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             FwdSmem<D>::alloc(kMaxPos));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = ensure_smem_limit((const void*)attn_fwd_tc_kernel<KIND, D>, FwdSmem<D>::alloc(kMaxPos));
+    if (e != cudaSuccess) return e;
     prof_begin(kProfAttnFwdTc, s);
     attn_fwd_tc_kernel<KIND, D><<<grid, kThreads, smem, s>>>(tq, tk, tv, p);
     prof_end(kProfAttnFwdTc, s);
@@ -690,8 +718,7 @@ int ctas_per_sm_one() {
     // Shared memory decides: each CTA holds ~110 KB (plus the 1 KB the driver
     // reserves per CTA) and 256 TMEM columns, so at most two fit on an SM.
     constexpr uint32_t smem = FwdSmem<D>::alloc(kMaxPos);
-    cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         smem);
+    ensure_smem_limit((const void*)attn_fwd_tc_kernel<KIND, D>, smem);
     cudaFuncSetAttribute(attn_fwd_tc_kernel<KIND, D>, cudaFuncAttributePreferredSharedMemoryCarveout,
                          100);
     int dev = 0, per_sm = 0;

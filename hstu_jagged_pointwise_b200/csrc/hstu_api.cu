@@ -7,10 +7,12 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/hstu.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace hstu {
 namespace {
@@ -40,6 +42,42 @@ const DevInfo* dev_info() {
     }
     return &d;
 }
+
+}  // namespace
+
+// Test hook settings of the pipelined kernels' bounded waits (hstu_debug_set_wait_fault).
+std::atomic<long long> g_wait_limit{0};
+std::atomic<int> g_withhold{0};
+
+DebugWait debug_wait() {
+    DebugWait w;
+    const long long l = g_wait_limit.load();
+    w.limit = l > 0 ? l : ptx::kWaitLimitCycles;
+    w.withhold_first_load = g_withhold.load();
+    return w;
+}
+
+// The dynamic shared-memory limit is a per-device attribute of a kernel: set it once
+// per (device, kernel), under a lock, the first time that kernel is launched on the
+// current device.
+cudaError_t ensure_smem_limit(const void* fn, int bytes) {
+    struct Entry { int dev; const void* fn; int bytes; };
+    static std::mutex mu;
+    static Entry done[256];
+    static int n_done = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n_done; i++)
+        if (done[i].dev == dev && done[i].fn == fn && done[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (n_done < 256) done[n_done++] = Entry{dev, fn, bytes};
+    return cudaSuccess;
+}
+
+namespace {
 
 // ------------------------------------------------------------------ TMA descriptors
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -262,6 +300,14 @@ extern "C" {
 
 const char* hstu_version(void) { return "0.1.0"; }
 
+int hstu_debug_set_wait_fault(int64_t wait_limit_cycles, int32_t withhold_first_load) {
+    if (wait_limit_cycles < 0 || (withhold_first_load != 0 && withhold_first_load != 1))
+        return HSTU_ERR_INVALID_ARG;
+    g_wait_limit.store(wait_limit_cycles);
+    g_withhold.store(withhold_first_load);
+    return HSTU_OK;
+}
+
 const char* hstu_status_string(int s) {
     switch (s) {
         case HSTU_OK: return "ok";
@@ -365,6 +411,7 @@ int attn_fwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
             return HSTU_ERR_CUDA;
         FwdParams fp;
         memset(&fp, 0, sizeof(fp));
+        fp.dbg = debug_wait();
         fp.q_off = fp.kv_off = seq_offsets;
         fp.q_ts = fp.kv_ts = timestamps;
         fp.n_static = mask->n_static;
@@ -415,7 +462,10 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
                   const float* ln_gamma, const float* ln_beta, const void* y, const float* ln_mean,
                   const float* ln_rstd, const void* d_o_pre, void* dq, void* dk, void* dv, void* du,
                   float* d_rab_pos, float* d_rab_time, float* d_gamma, float* d_beta, void* workspace,
-                  size_t workspace_bytes, void* stream) {
+                  size_t workspace_bytes, void* stream, const void* dy_in = nullptr) {
+    // dy_in != nullptr: attention-only backward from dL/dY (no LayerNorm backward; u, ln_*,
+    // y, d_o_pre, du, d_gamma and d_beta are not used)
+    const bool from_dy = dy_in != nullptr;
     int st = check_dims(dims);
     if (st != HSTU_OK) return st;
     int G = 1;
@@ -430,24 +480,27 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     const Layout L = attn_layout(d, 1, G);
     if (!aligned(workspace, 256)) return HSTU_ERR_WORKSPACE;
     if (workspace_bytes < L.total) return HSTU_ERR_WORKSPACE;
-    if (!aligned(d_rab_pos, 4) || !aligned(d_rab_time, 4) || !aligned(d_gamma, 4) ||
-        !aligned(d_beta, 4))
+    if (!aligned(d_rab_pos, 4) || !aligned(d_rab_time, 4) ||
+        (!from_dy && (!aligned(d_gamma, 4) || !aligned(d_beta, 4))))
         return HSTU_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int D = d.H * d.d_v;
     cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * d.n_pos - 1), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * d.n_tbuckets, s);
-    if (e == cudaSuccess && d.T == 0) {
+    if (e == cudaSuccess && d.T == 0 && !from_dy) {
         e = cudaMemsetAsync(d_gamma, 0, sizeof(float) * D * G, s);
         if (e == cudaSuccess) e = cudaMemsetAsync(d_beta, 0, sizeof(float) * D * G, s);
     }
     if (e != cudaSuccess) return cuda_status(e);
     if (d.T == 0) return HSTU_OK;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(u, 16) || !aligned(y, 16) ||
-        !aligned(d_o_pre, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
-        !aligned(du, 16) || !aligned(seq_offsets, 4) || !aligned(timestamps, 8) ||
-        !aligned(rab_pos, 4) || !aligned(rab_time, 4) || !aligned(ln_gamma, 16) ||
-        !aligned(ln_beta, 16) || !aligned(ln_mean, 4) || !aligned(ln_rstd, 4))
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+        !aligned(dv, 16) || !aligned(seq_offsets, 4) || !aligned(timestamps, 8) || !aligned(rab_pos, 4) ||
+        !aligned(rab_time, 4))
+        return HSTU_ERR_INVALID_ARG;
+    if (from_dy ? !aligned(dy_in, 16)
+                : (!aligned(u, 16) || !aligned(y, 16) || !aligned(d_o_pre, 16) || !aligned(du, 16) ||
+                   !aligned(ln_gamma, 16) || !aligned(ln_beta, 16) || !aligned(ln_mean, 4) ||
+                   !aligned(ln_rstd, 4)))
         return HSTU_ERR_INVALID_ARG;
     Control* ctrl = at<Control>(workspace, 0);
 
@@ -472,7 +525,21 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     st = cuda_status(launch_schedule(sp, s));
     if (st != HSTU_OK) return st;
 
-    // 2. LayerNorm backward: dY (into the workspace), dU, dgamma, dbeta
+    // 2. LayerNorm backward: dY (into the workspace), dU, dgamma, dbeta; or, from dL/dY,
+    //    only the scaled copy of dY the tensor-core backward reads
+    // the tensor-core backward takes dY / (2 alpha): its elementwise step then needs no scaling
+    const float dy_scale = d.dtype == HSTU_F32 ? 1.0f : 0.5f / d.alpha;
+    const void* dy_ws = at<void>(workspace, L.dy);
+    if (from_dy) {
+        if (d.dtype == HSTU_F32) {
+            dy_ws = dy_in;                        // the CUDA-core backward reads dY as it is
+        } else {
+            st = cuda_status(launch_scale_bf16(static_cast<const __nv_bfloat16*>(dy_in),
+                                               at<__nv_bfloat16>(workspace, L.dy), dy_scale,
+                                               (long long)d.T * D, s));
+            if (st != HSTU_OK) return st;
+        }
+    }
     LnParams lp;
     memset(&lp, 0, sizeof(lp));
     lp.T = d.T;
@@ -485,9 +552,8 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     lp.mean = const_cast<float*>(ln_mean);
     lp.rstd = const_cast<float*>(ln_rstd);
     lp.g = d_o_pre;
-    lp.dy = at<void>(workspace, L.dy);
-    // the tensor-core backward takes dY / (2 alpha): its elementwise step then needs no scaling
-    lp.dy_scale = d.dtype == HSTU_F32 ? 1.0f : 0.5f / d.alpha;
+    lp.dy = const_cast<void*>(dy_ws);
+    lp.dy_scale = dy_scale;
     lp.du = du;
     lp.part = at<float>(workspace, L.part);
     lp.n_part = L.n_part;
@@ -497,8 +563,10 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     lp.group = group;
     lp.status = &ctrl->status;
     if (G > 1) lp.gmask = at<int>(workspace, L.gmask);
-    st = cuda_status(launch_ln_bwd(d.dtype == HSTU_F32, lp, s));
-    if (st != HSTU_OK) return st;
+    if (!from_dy) {
+        st = cuda_status(launch_ln_bwd(d.dtype == HSTU_F32, lp, s));
+        if (st != HSTU_OK) return st;
+    }
 
     // 3. attention backward
     if (d.dtype == HSTU_F32) {
@@ -529,6 +597,7 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     if (st != HSTU_OK) return st;
     BwdParams bp;
     memset(&bp, 0, sizeof(bp));
+    bp.dbg = debug_wait();
     bp.off = seq_offsets;
     bp.ts = timestamps;
     bp.n_static = mask->n_static;
@@ -583,6 +652,17 @@ int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask, const void*
     return attn_bwd_impl(dims, mask, nullptr, q, k, v, u, seq_offsets, timestamps, rab_pos, rab_time, ln_gamma,
                          ln_beta, y, ln_mean, ln_rstd, d_o_pre, dq, dk, dv, du, d_rab_pos, d_rab_time, d_gamma,
                          d_beta, workspace, workspace_bytes, stream);
+}
+
+int hstu_attn_bwd_dy(const hstu_dims* dims, const hstu_mask_spec* mask, const void* q, const void* k,
+                     const void* v, const int32_t* seq_offsets, const int64_t* timestamps, const float* rab_pos,
+                     const float* rab_time, const void* dy, void* dq, void* dk, void* dv, float* d_rab_pos,
+                     float* d_rab_time, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!dy && dims && dims->T > 0) return HSTU_ERR_INVALID_ARG;
+    static const char kNoDy = 0;   // stands for dY when T == 0 (nothing is read)
+    return attn_bwd_impl(dims, mask, nullptr, q, k, v, nullptr, seq_offsets, timestamps, rab_pos, rab_time,
+                         nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, dk, dv, nullptr, d_rab_pos,
+                         d_rab_time, nullptr, nullptr, workspace, workspace_bytes, stream, dy ? dy : &kNoDy);
 }
 
 int hstu_attn_bwd_gln(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_norm_spec* norm,
@@ -670,6 +750,7 @@ int hstu_mfalcon_score(const hstu_mfalcon_dims* dims, const void* hist_k, const 
         return HSTU_ERR_CUDA;
     FwdParams fp;
     memset(&fp, 0, sizeof(fp));
+    fp.dbg = debug_wait();
     fp.q_off = cand_offsets;
     fp.kv_off = hist_offsets;
     fp.q_ts = cand_ts;

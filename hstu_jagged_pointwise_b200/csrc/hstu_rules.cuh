@@ -109,9 +109,10 @@ __device__ __forceinline__ int tile_class(int kind, int qa, int qb, int ka, int 
         if (max(clo, ka) <= min(chi, kb)) any = true;
     }
     if (!any) return 0;
-    // full tiles: every row and column static, or every row real-time and
-    // every column at or before the first row (static or earlier real-time)
-    if (qb < S && kb < S) return 2;
+    // full tiles: every column static and every row a non-candidate (static rows see
+    // all static tokens, real-time rows too), or every row real-time and every column
+    // at or before the first row (static or earlier real-time)
+    if (kb < S && qb < H) return 2;
     if (qa >= S && qb < H && kb <= qa) return 2;
     if (kind == HSTU_KIND_MFSEQ && qa >= H && kb < H) return 2;   // candidates x history: no filter
     return 1;

@@ -33,6 +33,18 @@ static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Bounded waits of the pipelined (TMA + tcgen05) kernels.  limit: SM cycles a
+// main-loop wait may last before the kernel records kStatusTimeout and leaves
+// (about a second by default; the drain waits at exit always keep the default).
+// withhold_first_load (test hook, 0 in normal use): each CTA's producer withholds
+// its first tile load and waits for the abort, so that the consumers' bounded
+// waits run out.  Both come from hstu_debug_set_wait_fault.
+struct DebugWait {
+    long long limit;
+    int withhold_first_load;
+};
+DebugWait debug_wait();
+
 // Work item: sequence b, query rows [row0, row_end) local to the sequence, head h.
 // Stored as int4 {b, row0, h, row_end}.
 
@@ -68,6 +80,7 @@ struct FwdParams {
     const __nv_bfloat16* self_v;
     int H, P, nb, ld;
     float inv_alpha;
+    DebugWait dbg;
 };
 
 // tcgen05 backward: one work item = (sequence, head, 128-key tile).
@@ -85,6 +98,7 @@ struct BwdParams {
     __nv_bfloat16* dv;
     float* rab_part;          // [grid][2P-1 + nb] per-CTA rab gradient partial sums, zeroed
     int H, P, nb, ld;
+    DebugWait dbg;
 };
 
 constexpr int kMaxBwdCtas = 1024;   // bound on the backward's persistent grid (workspace sizing)
@@ -157,6 +171,7 @@ struct GemmParams {
     __nv_bfloat16* z;                   // kEpiF1: pre-activation [M, N] or nullptr
     int D;                              // kEpiF1: width of each output block
     int* status;                        // kStatusTimeout is OR-ed here, or nullptr
+    DebugWait dbg;
 };
 
 // Output tensor maps of the epilogue: out[0..3] (kEpiF1: U, V, Q, K; otherwise out[0] only)
@@ -178,12 +193,16 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long 
 // [rows, cols] fp32 row-major, 128-byte swizzle, box = 32 columns x box_rows rows
 bool make_tmap_f32_sw128(CUtensorMap* m, void* base, long long rows, long long cols, int box_rows);
 int device_sms();
+// cudaFuncAttributeMaxDynamicSharedMemorySize of kernel fn on the current device, set
+// once per (device, kernel) and thread-safe.
+cudaError_t ensure_smem_limit(const void* fn, int bytes);
 
 // ---- opt-in per-kernel timing (profile.cu)
 enum ProfKind {
     kProfSchedule = 0, kProfAttnFwdTc, kProfAttnFwdSimt, kProfLnFwd, kProfLnBwd, kProfLnBwdReduce,
     kProfAttnBwdDkvSimt, kProfAttnBwdDqSimt, kProfDebugIndices, kProfAttnBwdTc, kProfDqConvert,
-    kProfRabReduce, kProfCacheScan, kProfCacheCopy, kProfGemm, kProfSiluGrad, kProfColSum, kProfSlSample, kProfGather, kProfKinds
+    kProfRabReduce, kProfCacheScan, kProfCacheCopy, kProfGemm, kProfSiluGrad, kProfColSum, kProfSlSample, kProfGather,
+    kProfScaleDy, kProfKinds
 };
 void prof_begin(int kind, cudaStream_t s);
 void prof_end(int kind, cudaStream_t s);
@@ -206,6 +225,9 @@ cudaError_t launch_attn_bwd_tc(int kind, int d, const CUtensorMap& tq, const CUt
                                const CUtensorMap& tv, const CUtensorMap& tdy, const CUtensorMap& tdq,
                                const BwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t s);
+// dst = bf16(src * scale), n a multiple of 8 (16-byte vectors)
+cudaError_t launch_scale_bf16(const __nv_bfloat16* src, __nv_bfloat16* dst, float scale, long long n,
+                              cudaStream_t s);
 cudaError_t launch_rab_reduce(const float* part, int n_part, int P, int nb, float* d_rab_pos,
                               float* d_rab_time, cudaStream_t s);
 cudaError_t launch_ln_fwd(int dtype_f32, const LnParams& p, cudaStream_t s);

@@ -31,7 +31,7 @@ const char* const kNames[kProfKinds] = {
     "ln_bwd_kernel", "ln_bwd_reduce_kernel", "attn_bwd_dkv_simt_kernel", "attn_bwd_dq_simt_kernel",
     "debug_indices_kernel", "attn_bwd_tc_kernel", "dq_convert_kernel", "rab_reduce_kernel",
     "cache_scan_kernel", "cache_copy_kernel", "gemm_tc_kernel", "silu_grad_kernel", "col_sum_kernel",
-    "sl_sample_kernels", "gather_rows_kernel"};
+    "sl_sample_kernels", "gather_rows_kernel", "scale_dy_kernel"};
 
 cudaEvent_t take_event() {
     if (!g_pool.empty()) {

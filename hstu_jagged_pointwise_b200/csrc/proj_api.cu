@@ -199,6 +199,7 @@ GemmParams gemm_params(int M, int N, int K, int32_t* status) {
     p.K = K;
     p.k_splits = 1;
     p.status = status;
+    p.dbg = debug_wait();
     return p;
 }
 

@@ -14,9 +14,9 @@
 // ring, one thread issues tcgen05.mma (M = 128, N = 256, K = 16) into a double-buffered
 // TMEM accumulator (2 x 256 fp32 columns), and eight epilogue warps drain one accumulator
 // while the next tile is being multiplied.  Each epilogue warp owns 32 rows x 128 columns
-// of a tile; it stages 32 x 64 output chunks in 128-byte-swizzled shared memory (two
-// buffers per warp) and writes them with TMA tensor stores, so every global write is a
-// full line.  Split-K (for the weight gradients, whose K is the token count) adds fp32
+// of a tile; it stages 32 x 64 output chunks in 128-byte-swizzled shared memory (one
+// buffer per warp, reused once the previous store has read it) and writes them with TMA
+// tensor stores, so every global write is a full line.  Split-K (for the weight gradients, whose K is the token count) adds fp32
 // partial tiles with TMA reduce-adds.
 //
 // Every wait is bounded; on timeout the CTA records kStatusTimeout in *status, drains
@@ -171,6 +171,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Smem::tmem);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + Smem::abort_flag);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long wl = p.dbg.limit;   // main-loop wait limit (SM cycles)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; s++) {
@@ -209,7 +210,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
                 const TileCoord c = tile_coord(p, t);
                 for (int kb = c.kb0; kb < c.kb1; kb++) {
                     const int st = use % kStages;
-                    ok = mbar_wait(&bars[kEmptyBar + st], ((use / kStages) & 1) ^ 1, s_abort);
+                    ok = mbar_wait(&bars[kEmptyBar + st], ((use / kStages) & 1) ^ 1, s_abort, wl);
+                    if (ok && p.dbg.withhold_first_load && use == 0) {
+                        // test hook: withhold this CTA's first k-step, so the waits for it run out
+                        wait_for_abort(s_abort, 2 * wl);
+                        ok = false;
+                    }
                     if (!ok) break;
                     uint8_t* sa = sm + st * kStage;
                     uint8_t* sb = sa + kATile;
@@ -251,13 +257,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
                 const TileCoord c = tile_coord(p, t);
                 if (c.kb1 <= c.kb0) { tile_i--; continue; }
                 const int buf = tile_i & 1;
-                ok = mbar_wait(&bars[kAccEmpty + buf], ((tile_i >> 1) & 1) ^ 1, s_abort);
+                ok = mbar_wait(&bars[kAccEmpty + buf], ((tile_i >> 1) & 1) ^ 1, s_abort, wl);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * kBN;
                 for (int kb = c.kb0; kb < c.kb1; kb++) {
                     const int st = use % kStages;
-                    ok = mbar_wait(&bars[kFullBar + st], (use / kStages) & 1, s_abort);
+                    ok = mbar_wait(&bars[kFullBar + st], (use / kStages) & 1, s_abort, wl);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sa = a_base + st * kStage, sb = b_base + st * kStage;
@@ -294,7 +300,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
             const TileCoord c = tile_coord(p, t);
             if (c.kb1 <= c.kb0) { tile_i--; continue; }
             const int buf = tile_i & 1;
-            ok = mbar_wait(&bars[kAccFull + buf], (tile_i >> 1) & 1, s_abort);
+            ok = mbar_wait(&bars[kAccFull + buf], (tile_i >> 1) & 1, s_abort, wl);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             tc_fence_after();
             const int row0 = c.m0 + wq * 32;              // this warp's 32 rows
@@ -388,13 +394,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
 template <bool A_MN, bool B_MN, int EPI>
 cudaError_t launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmOutMaps& to, const GemmParams& p,
                      int grid, cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, EPI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::alloc);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = ensure_smem_limit((const void*)gemm_tc_kernel<A_MN, B_MN, EPI>, Smem::alloc);
+    if (e != cudaSuccess) return e;
     gemm_tc_kernel<A_MN, B_MN, EPI><<<grid, kThreads, Smem::alloc, s>>>(ta, tb, to, p);
     return cudaGetLastError();
 }

@@ -48,15 +48,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false when
-// the wait runs past kWaitLimitCycles or *abort becomes non-zero.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// the wait runs past `limit` SM cycles or *abort becomes non-zero.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
+}
+
+// Waits until *abort becomes non-zero or `limit` SM cycles pass (the withheld-load
+// test hook of the pipelined kernels: their producer stops here while the
+// consumers' bounded waits run out).
+__device__ __forceinline__ void wait_for_abort(volatile int* abort, long long limit) {
+    const long long t0 = clock64();
+    while (!*abort && clock64() - t0 <= limit) __nanosleep(256);
 }
 
 // ---------------------------------------------------------------- named barrier

@@ -158,6 +158,20 @@ class Layer:
         capi.check(st, "hstu_attn_bwd")
         return out
 
+    def backward_from_dy(self, q, k, v, rab_pos, rab_time, dy, out: Optional[dict] = None) -> dict:
+        """Attention-only backward (hstu_attn_bwd_dy): dy = dL/dY in; dq, dk, dv and the
+        bias-table gradients out."""
+        _need(dy, "dy", self.dtype)
+        if out is None:
+            out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                       d_rab_pos=torch.empty_like(rab_pos), d_rab_time=torch.empty_like(rab_time))
+        st = capi.LIB.hstu_attn_bwd_dy(C.byref(self.dims), C.byref(self.mask), _p(q), _p(k), _p(v),
+                                       _p(self.seq_offsets), _p(self.timestamps), _p(rab_pos), _p(rab_time),
+                                       _p(dy), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]), _p(out["d_rab_pos"]),
+                                       _p(out["d_rab_time"]), _p(self.ws), self.ws.numel(), _stream())
+        capi.check(st, "hstu_attn_bwd_dy")
+        return out
+
     def check_device_error(self) -> int:
         return int(capi.LIB.hstu_check_device_error(_p(self.ws), _stream()))
 

@@ -178,7 +178,10 @@ HSTU_API int hstu_attn_fwd_gln(const hstu_dims* dims, const hstu_mask_spec* mask
  *    use hstu_attn_fwd with a workspace for larger problems.
  *  - First call per device: looks up the scratch address (cudaGetSymbolAddress),
  *    which may load the library's module on that device.  Make the first call on
- *    each device before any stream capture begins.
+ *    each device before any stream capture begins.  The address is kept for the
+ *    life of the process: after cudaDeviceReset (or anything else that destroys
+ *    the device's primary context) this entry point must not be called again on
+ *    that device in the same process.
  *  - Each call clears the scratch's control block (status word and work counter)
  *    on `stream` before the forward's launches.
  *  - One scratch per device: calls whose work can overlap on the device (other
@@ -213,6 +216,26 @@ HSTU_API int hstu_attn_bwd(const hstu_dims* dims, const hstu_mask_spec* mask,
                   const void* d_o_pre,
                   void* dq, void* dk, void* dv, void* du,
                   float* d_rab_pos, float* d_rab_time, float* d_gamma, float* d_beta,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Attention-only backward: the gradient of the attention output Y itself in,
+ * the gradients of q, k, v and the two bias tables out.  Y = (1/alpha) sum_j
+ * mask(i, j) SiLU(z_ij) v_j (Meta HSTU blog, section 3 formula and 3.1; rab
+ * from section 3.2) is the A(X)V(X) part of the HSTU layer; this entry point is
+ * hstu_attn_bwd without its LayerNorm-times-U step, for callers that apply their
+ * own normalisation after the attention (or none).  Derivatives as in
+ * hstu_attn_bwd; A is recomputed, never stored.
+ * In:  dy [T, H*d_v] = dL/dY (element type dims.dtype); q, k, v, offsets,
+ *      timestamps, bias tables and mask as hstu_attn_fwd.
+ * Out: dq, dk [T, H*d_qk], dv [T, H*d_v]; d_rab_pos fp32 [2P-1], d_rab_time fp32
+ *      [nb]; all overwritten.
+ * Workspace: hstu_attn_workspace_bytes(dims, mask->kind, 1).  Errors as
+ * hstu_attn_bwd (dy NULL with T > 0: HSTU_ERR_INVALID_ARG). */
+HSTU_API int hstu_attn_bwd_dy(const hstu_dims* dims, const hstu_mask_spec* mask,
+                  const void* q, const void* k, const void* v,
+                  const int32_t* seq_offsets, const int64_t* timestamps,
+                  const float* rab_pos, const float* rab_time, const void* dy,
+                  void* dq, void* dk, void* dv, float* d_rab_pos, float* d_rab_time,
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward of hstu_attn_fwd_gln: ln_gamma, ln_beta, d_gamma and d_beta are fp32
@@ -415,6 +438,24 @@ HSTU_API const char* hstu_status_string(int status);
 HSTU_API int hstu_profile_enable(int32_t on);
 HSTU_API int hstu_profile_read(int32_t n_kinds, int32_t* launches, double* total_ms);
 HSTU_API const char* hstu_profile_kind_name(int32_t kind);
+
+/* Test hook for the bounded waits of the pipelined kernels (the tcgen05
+ * attention forward and backward, the M-FALCON scorer and the projection GEMM).
+ * Not part of the pages' method: it exists so that tests can make a device wait
+ * run out without a fault.  Applies to the launches that follow, in every host
+ * thread, until it is called again.
+ *  - wait_limit_cycles > 0: a main-loop wait gives up after that many SM cycles
+ *    (the default, used when it is 0, is about one second); waits that drain a
+ *    kernel's own copies and MMAs at exit keep the default.
+ *  - withhold_first_load = 1: each CTA's TMA producer withholds its first tile
+ *    load and waits for the abort, so the consumers' waits for that tile run
+ *    out.  The kernel then records the timeout bit in the status word, drains
+ *    what it issued, frees its tensor memory and returns without writing its
+ *    outputs; hstu_check_device_error reports HSTU_ERR_DEVICE_TIMEOUT (the GEMM
+ *    entry points set bit 2 of device_status).  The context stays usable.
+ * Call hstu_debug_set_wait_fault(0, 0) to restore normal operation.  Returns
+ * HSTU_ERR_INVALID_ARG for a negative limit or a flag other than 0 or 1. */
+HSTU_API int hstu_debug_set_wait_fault(int64_t wait_limit_cycles, int32_t withhold_first_load);
 
 /* Library version, e.g. "0.1.0". */
 HSTU_API const char* hstu_version(void);
