@@ -18,7 +18,7 @@ def header_functions():
 
 def test_exports_match_header():
     names = header_functions()
-    assert len(names) == 26, names
+    assert len(names) == 28, names
     assert set(names) == set(capi.EXPORTS)
     for n in names:
         assert hasattr(capi.LIB, n), n
@@ -212,3 +212,12 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
         r = subprocess.run([sys.executable, "-c", f"import {mod}"], cwd=tmp_path, capture_output=True, text=True,
                            env={**os.environ, "PYTHONPATH": str(tmp_path)})
         assert r.returncode != 0 and "libhstu_b200.so is missing" in r.stderr, r.stderr[-800:]
+
+
+def test_debug_wait_fault_checks_its_arguments():
+    assert capi.LIB.hstu_debug_set_wait_fault(-1, 0) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_debug_set_wait_fault(1000, 2) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_debug_set_wait_fault(0, 0) == capi.HSTU_OK
+    with capi.wait_fault(1000):
+        pass                                   # host-side setting only: nothing launches
+    assert capi.LIB.hstu_debug_set_wait_fault(0, 0) == capi.HSTU_OK

@@ -660,7 +660,41 @@ def _sub_workload(w, b):
     return ws, s0, s1
 
 
-def test_large_layer_sampled_forward_and_per_sequence_backward():
+def _golden_reduced(path):
+    """name -> (exact, storage) arrays from a reduced-gradient golden file."""
+    rows = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, i, a, b = line.split()
+            rows.setdefault(name, []).append((int(i), float(a), float(b)))
+    out = {}
+    for name, r in rows.items():
+        r.sort()
+        out[name] = (np.array([x[1] for x in r]), np.array([x[2] for x in r]))
+    return out
+
+
+def _check_seq_backward(out, w, b, label):
+    """Every per-token backward output of sequence b of a batch against the oracle run on
+    that sequence alone (sequences are independent)."""
+    ws, s0, s1 = _sub_workload(w, b)
+    ref = oracle.layer_bwd(ws)
+    st = storage_bwd(ws)
+    for k in ("dq", "dk", "dv", "du"):
+        assert_bf16(out[k][s0:s1], ref[k], f"{k}[{label}]", st[k])
+    return ws, ref, st
+
+
+def test_large_layer_sampled_forward_and_full_size_backward():
+    """The large layer (262,144 tokens, 165 sequences up to 7,585 long, 8 heads x 128) in the
+    bench's launch configuration.  Forward: sampled rows.  Backward: the reduced gradients
+    (d_rab_pos, d_rab_time, d_gamma, d_beta: sums over all 3.1e9 visible pairs or all tokens)
+    against the fp64 oracle's values for this seeded batch (tests/golden, written by
+    make_large_layer_reduced.py from the oracle alone), and every per-token gradient of the
+    longest sequence, of the shortest and of one near 1000 tokens."""
+    import os
     w = W.large_layer(seed=0)
     out, _, _ = run_layer(w, backward=True)
     rng = np.random.default_rng(4)
@@ -670,15 +704,33 @@ def test_large_layer_sampled_forward_and_per_sequence_backward():
     rt = torch.as_tensor(rows).cuda()
     assert_bf16(out["y"][rt], y, "y", st["y"])
     assert_bf16(out["o_pre"][rt], o, "o_pre", st["o_pre"])
-    # full backward of two whole sequences (the shortest and one near 1000 tokens)
+    gold = _golden_reduced(os.path.join(os.path.dirname(__file__), "golden",
+                                        "large_layer_T262144_seed0_reduced.txt"))
+    for k, name in (("d_rab_pos", "d_rab_pos"), ("d_rab_time", "d_rab_time"), ("d_gamma", "dgamma"),
+                    ("d_beta", "dbeta")):
+        exact, storage = gold[name]
+        assert_bf16(out[k], exact, f"{k} (all 165 sequences)", storage)
     L = w.lengths
-    picks = [int(np.argmin(L)), int(np.argmin(np.abs(L - 1000)))]
-    for b in picks:
-        ws, s0, s1 = _sub_workload(w, b)
-        ref = oracle.layer_bwd(ws)
-        st = storage_bwd(ws)
-        for k in ("dq", "dk", "dv", "du"):
-            assert_bf16(out[k][s0:s1], ref[k], f"{k}[seq {b}]", st[k])
+    for b in (int(np.argmax(L)), int(np.argmin(L)), int(np.argmin(np.abs(L - 1000)))):
+        _check_seq_backward(out, w, b, f"seq {b}, L={int(L[b])}")
+
+
+def test_large_layer_longest_sequence_as_its_own_batch():
+    """The longest sequence of the large layer (7,585 tokens: the most query tiles per key
+    tile and the most time-bucket runs) as a batch of one: all eight backward outputs."""
+    w = W.large_layer(seed=0)
+    b = int(np.argmax(w.lengths))
+    ws, _, _ = _sub_workload(w, b)
+    out, _, _ = run_layer(ws, backward=True)
+    ref = oracle.layer_bwd(ws)
+    st = storage_bwd(ws)
+    _, o, _, _ = oracle.layer_fwd(ws)
+    assert_bf16(out["y"], ref["y"], "y", st["y"])
+    assert_bf16(out["o_pre"], o, "o_pre", storage_fwd(ws)["o_pre"])
+    for k in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+        assert_bf16(out[k], ref[k], k, st[k])
+    assert_bf16(out["d_gamma"], ref["dgamma"], "d_gamma", st["dgamma"])
+    assert_bf16(out["d_beta"], ref["dbeta"], "d_beta", st["dbeta"])
 
 
 # ----------------------------------------------------------------------------

@@ -50,7 +50,9 @@ def _worker(rank, world, port, q):
     try:
         w = _global_batch()
         parts = shard.partition_sequences(w.lengths, world)
-        s, rows = _sub(w, parts[rank])
+        mine = shard.rank_sequences(w.lengths, world, rank)       # what bench.py's ranks take
+        assert mine == parts[rank]
+        s, rows = _sub(w, mine)
         g = oracle.layer_bwd(s)
         grads = {"d_rab_pos": torch.tensor(g["d_rab_pos"]), "d_rab_time": torch.tensor(g["d_rab_time"]),
                  "d_gamma": torch.tensor(g["dgamma"]), "d_beta": torch.tensor(g["dbeta"])}
