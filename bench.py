@@ -287,10 +287,34 @@ def time_oracle(sample):
 # our arm
 # ----------------------------------------------------------------------------
 
-def run_ours(args, world, rank, local):
-    from hstu_jagged_pointwise_b200 import capi, ops
+def rank_workload(args, world, rank):
+    """This rank's batch.  One GPU: the large layer (lognormal lengths summing to
+    args.tokens).  N GPUs (weak scaling): one global batch of N * args.tokens tokens whose
+    sequences are split across the ranks by shard.rank_sequences (whole sequences,
+    balanced on sum(L^2)); each rank draws the dense tensors of its own sequences."""
+    if world == 1:
+        return W.large_layer(seed=args.seed, total=args.tokens)
+    from hstu_jagged_pointwise_b200 import shard
+    rng = np.random.Generator(np.random.PCG64(args.seed))
+    lengths = W.lognormal_lengths(rng, args.tokens * world)
+    mine = lengths[shard.rank_sequences(lengths, world, rank)]
+    return W.make_causal(mine, H=8, d=128, dtype=torch.bfloat16, seed=args.seed + 404 + rank, with_grad=True,
+                         alpha=float(lengths.max()), name=f"large_layer_T{args.tokens}_H8_d128")
 
-    w = W.large_layer(seed=args.seed + rank, total=args.tokens)
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t)
+    return float(t.item())
+
+
+def run_ours(args, world, rank, local):
+    from hstu_jagged_pointwise_b200 import capi, ops, shard
+
+    w = rank_workload(args, world, rank)
     dev = torch.device("cuda", local)
     H, d = w.H, w.d
     P_head = causal_pairs(w.lengths)
@@ -308,18 +332,13 @@ def run_ours(args, world, rank, local):
     bwd_out = dict(dq=torch.empty_like(dv["q"]), dk=torch.empty_like(dv["k"]), dv=torch.empty_like(dv["v"]),
                    du=torch.empty_like(dv["u"]), d_rab_pos=torch.empty_like(rp), d_rab_time=torch.empty_like(rt),
                    d_gamma=torch.empty_like(g), d_beta=torch.empty_like(b))
-    small = None
-    if world > 1:
-        import torch.distributed as dist
-        small = torch.empty(rp.numel() + rt.numel() + 2 * g.numel(), dtype=torch.float32, device=dev)
 
     def step():
         layer.forward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, out=fwd_out)
         layer.backward(dv["q"], dv["k"], dv["v"], dv["u"], rp, rt, g, b, fwd_out, dv["grad"], out=bwd_out)
         if world > 1:
-            torch.cat([bwd_out["d_rab_pos"], bwd_out["d_rab_time"], bwd_out["d_gamma"], bwd_out["d_beta"]],
-                      out=small)
-            dist.all_reduce(small)
+            # the only exchange: data-parallel sum of the parameter gradients
+            shard.allreduce_param_grads(bwd_out)
 
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -369,45 +388,84 @@ def run_ours(args, world, rank, local):
         extra["data_step"] = run_data_step(args, world, rank, w)
     if not args.no_layer:
         extra["full_layer"] = run_full_layer(args, world, w, f_fwd + f_bwd)
+    if not args.no_configs:
+        extra["training_sl"] = run_training_sl(args, world, rank)
+        extra["mtgr_medium"] = run_mtgr_medium(args, world, rank)
 
     # ---- end to end through the C ABI with host buffers
     if args.no_e2e:
         return finish(args, world, w, kernels, ms, ms_max, ms_fwd, None, None, None, None, clocks, f_fwd, f_bwd, P, d,
                       extra)
+    # Pipelined over three streams: the host->device copies of step k+1 and the
+    # device->host copies of step k-1 run while step k computes (PCIe carries both
+    # directions at once), on double-buffered device inputs and outputs.  Every copy is
+    # one cudaMemcpyAsync from or to pinned host memory.
+    small_names = (("rp", w.rab_pos), ("rt", w.rab_time), ("g", w.gamma), ("b", w.beta))
     pin = {n: t.pin_memory() for n, t in host.items()}
-    small_in = {n: t.pin_memory() for n, t in (("rp", w.rab_pos), ("rt", w.rab_time), ("g", w.gamma),
-                                                ("b", w.beta))}
-    off_h = torch.as_tensor(w.offsets).pin_memory()
-    ts_h = torch.as_tensor(w.ts).pin_memory()
-    outs_h = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in
-              list(bwd_out.items()) + [("o_pre", fwd_out["o_pre"])]}
-    h2d = sum(t.numel() * t.element_size() for t in list(pin.values()) + list(small_in.values()) + [off_h, ts_h])
-    d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
+    pin.update({n: t.pin_memory() for n, t in small_names})
+    pin["off"] = torch.as_tensor(w.offsets).pin_memory()
+    pin["ts"] = torch.as_tensor(w.ts).pin_memory()
+    out_names = list(bwd_out) + ["o_pre"]
+    outs_h = [{n: torch.empty(bwd_out[n].shape if n in bwd_out else fwd_out[n].shape,
+                              dtype=(bwd_out[n] if n in bwd_out else fwd_out[n]).dtype, pin_memory=True)
+               for n in out_names} for _ in range(2)]
+    dev_in = [dict(q=dv["q"], k=dv["k"], v=dv["v"], u=dv["u"], grad=dv["grad"], rp=rp, rt=rt, g=g, b=b, off=off,
+                   ts=ts)]
+    dev_in.append({n: torch.empty_like(t) for n, t in dev_in[0].items()})
+    dev_fo = [fwd_out, {n: torch.empty_like(t) for n, t in fwd_out.items()}]
+    dev_bo = [bwd_out, {n: torch.empty_like(t) for n, t in bwd_out.items()}]
+    layers = [layer, ops.Layer(dev_in[1]["off"], dev_in[1]["ts"], H, d, torch.bfloat16, w.alpha, w.max_len)]
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h[0].values())
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def e2e_step():
-        for n, t in pin.items():
-            dv[n].copy_(t, non_blocking=True)
-        rp.copy_(small_in["rp"], non_blocking=True)
-        rt.copy_(small_in["rt"], non_blocking=True)
-        g.copy_(small_in["g"], non_blocking=True)
-        b.copy_(small_in["b"], non_blocking=True)
-        off.copy_(off_h, non_blocking=True)
-        ts.copy_(ts_h, non_blocking=True)
-        step()
-        for n, t in outs_h.items():
-            src = fwd_out["o_pre"] if n == "o_pre" else bwd_out[n]
-            t.copy_(src, non_blocking=True)
+    def run_pipeline(n_steps):
+        """n_steps end-to-end steps: inputs from pinned host memory, outputs back to it."""
+        in_ready = [torch.cuda.Event() for _ in range(n_steps)]
+        done = [torch.cuda.Event() for _ in range(n_steps)]
+        out_free = [torch.cuda.Event() for _ in range(n_steps)]
 
-    e2e_step()
+        def upload(k):
+            with torch.cuda.stream(s_h2d):
+                if k >= 2:
+                    s_h2d.wait_event(done[k - 2])          # buffer k % 2 was read by step k - 2
+                for n, t in pin.items():
+                    dev_in[k % 2][n].copy_(t, non_blocking=True)
+                in_ready[k].record(s_h2d)
+
+        upload(0)
+        for k in range(n_steps):
+            if k + 1 < n_steps:
+                upload(k + 1)
+            stream.wait_event(in_ready[k])
+            if k >= 2:
+                stream.wait_event(out_free[k - 2])         # outputs k % 2 read back by step k - 2
+            x, fo, bo, ly = dev_in[k % 2], dev_fo[k % 2], dev_bo[k % 2], layers[k % 2]
+            ly.forward(x["q"], x["k"], x["v"], x["u"], x["rp"], x["rt"], x["g"], x["b"], out=fo)
+            ly.backward(x["q"], x["k"], x["v"], x["u"], x["rp"], x["rt"], x["g"], x["b"], fo, x["grad"], out=bo)
+            if world > 1:
+                shard.allreduce_param_grads(bo)
+            done[k].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(done[k])
+                for n, t in outs_h[k % 2].items():
+                    t.copy_(fo[n] if n == "o_pre" else bo[n], non_blocking=True)
+                out_free[k].record(s_d2h)
+        stream.wait_stream(s_d2h)
+        stream.wait_stream(s_h2d)
+
+    run_pipeline(2)
     torch.cuda.synchronize()
-    n_e2e = max(1, min(args.steps, 3))
+    n_e2e = max(2, min(args.steps, 8))
     barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
+    run_pipeline(n_e2e)
     e1.record(stream)
     torch.cuda.synchronize()
+    for ly in layers:
+        if ly.check_device_error() != 0:
+            raise RuntimeError("device status set in the end-to-end leg")
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
 
     # ---- M-FALCON candidates / s
@@ -541,6 +599,109 @@ def run_full_layer(args, world, w, attn_flops):
             "pct_bf16_sustained": round(tf / world / pk["bf16_tflops_sustained"], 4),
             "kernel_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in sorted(prof.items(),
                                                                                       key=lambda kv: -kv[1][1])}}
+
+
+def mtgr_pairs(w) -> int:
+    """Visible (i, j) pairs of one head under the MTGR dynamic mixed mask (MTGR deep-dive
+    section 2): static rows see the S static tokens; real-time row i sees S + (its index
+    among the real-time tokens + 1); a candidate sees itself and the non-candidates with
+    a strictly smaller timestamp."""
+    off = np.asarray(w.offsets, np.int64)
+    total = 0
+    for b in range(len(off) - 1):
+        L = int(off[b + 1] - off[b])
+        S, R = int(w.n_static[b]), int(w.n_realtime[b])
+        total += S * S + R * S + R * (R + 1) // 2
+        ts = np.asarray(w.ts[off[b]:off[b + 1]], np.int64)
+        hist = np.sort(ts[:S + R])
+        total += int(np.searchsorted(hist, ts[S + R:], side="left").sum()) + (L - S - R)
+    return total
+
+
+def _timed(args, world, fn):
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    from hstu_jagged_pointwise_b200 import capi
+    capi.profile_enable(True)
+    e0.record(s)
+    for _ in range(args.steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    prof = capi.profile_read()
+    capi.profile_enable(False)
+    return max_over_ranks(e0.elapsed_time(e1) / args.steps, world), prof
+
+
+def _attn_leg(args, world, w, backward: bool, pairs_per_head: int):
+    """One attention layer of workload w (forward, or forward + backward) timed on its own,
+    with the useful TFLOP/s of the step and of the attention kernels."""
+    from hstu_jagged_pointwise_b200 import ops
+    dev = torch.device("cuda", torch.cuda.current_device())
+    t = {n: getattr(w, n).to(dev) for n in ("q", "k", "v", "u", "rab_pos", "rab_time", "gamma", "beta")}
+    if backward:
+        t["grad"] = w.grad.to(dev)
+    d = {n: torch.as_tensor(np.asarray(getattr(w, n), np.int32)).to(dev)
+         for n in ("offsets", "n_static", "n_realtime") if getattr(w, n) is not None}
+    layer = ops.Layer(d["offsets"], torch.as_tensor(w.ts).to(dev), w.H, w.d, w.dtype, w.alpha, w.max_len,
+                      mask_kind=w.kind, n_static=d.get("n_static"), n_realtime=d.get("n_realtime"))
+    fo = dict(y=torch.empty_like(t["q"]), o_pre=torch.empty_like(t["q"]),
+              mean=torch.empty(w.T, dtype=torch.float32, device=dev),
+              rstd=torch.empty(w.T, dtype=torch.float32, device=dev))
+    bo = None
+    if backward:
+        bo = dict(dq=torch.empty_like(t["q"]), dk=torch.empty_like(t["k"]), dv=torch.empty_like(t["v"]),
+                  du=torch.empty_like(t["u"]), d_rab_pos=torch.empty_like(t["rab_pos"]),
+                  d_rab_time=torch.empty_like(t["rab_time"]), d_gamma=torch.empty_like(t["gamma"]),
+                  d_beta=torch.empty_like(t["beta"]))
+
+    def fwd():
+        layer.forward(t["q"], t["k"], t["v"], t["u"], t["rab_pos"], t["rab_time"], t["gamma"], t["beta"], out=fo)
+
+    def step():
+        fwd()
+        if backward:
+            layer.backward(t["q"], t["k"], t["v"], t["u"], t["rab_pos"], t["rab_time"], t["gamma"], t["beta"], fo,
+                           t["grad"], out=bo)
+
+    ms, prof = _timed(args, world, step)
+    if layer.check_device_error() != 0:
+        raise RuntimeError(f"device status set in {w.name}")
+    pk, _ = peaks()
+    P = pairs_per_head * w.H
+    f_fwd, f_bwd = 4 * w.d * P, 8 * w.d * P
+    out = {"workload": w.name, "tokens": int(w.T), "sequences": int(w.B), "max_seq_len": int(w.max_len),
+           "alpha": w.alpha, "visible_pairs": int(P), "ms_per_step": round(ms, 4)}
+    flops = f_fwd + (f_bwd if backward else 0)
+    tf = world * flops / (ms * 1e-3) / 1e12
+    out["tflops_step"] = round(tf, 2)
+    out["pct_bf16_sustained_step"] = round(tf / world / pk["bf16_tflops_sustained"], 4)
+    for name, units in (("attn_fwd_tc_kernel", f_fwd), ("attn_bwd_tc_kernel", f_bwd)):
+        if name in prof:
+            n, tot = prof[name]
+            kt = units / (tot / n * 1e-3) / 1e12
+            out[name] = {"ms_per_launch": round(tot / n, 4), "tflops": round(kt, 2),
+                         "frac_bf16_burst": round(kt / pk["bf16_tflops"], 4),
+                         "frac_bf16_sustained": round(kt / pk["bf16_tflops_sustained"], 4)}
+    return out
+
+
+def run_training_sl(args, world, rank):
+    """The training shape (64 Zipf(1.2) sequences in [16, 4096], Stochastic Length at
+    alpha 1.6, cap 776; 4 heads x 128; causal + rab): forward and backward."""
+    w = W.training_sl(seed=args.seed + rank)
+    return _attn_leg(args, world, w, True, causal_pairs(w.lengths))
+
+
+def run_mtgr_medium(args, world, rank):
+    """MTGR-Medium-style users (128 rows of 24 profile + U[200, 3000] behaviour + 0-64
+    real-time + 20-200 candidates; 6 heads x 128) under the dynamic mixed mask: forward."""
+    w = W.mtgr_medium(seed=args.seed + rank)
+    return _attn_leg(args, world, w, False, mtgr_pairs(w))
 
 
 def run_data_step(args, world, rank, w):
@@ -678,14 +839,18 @@ def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, cl
             "peak_source": f"{pk_src} ({'bf16_tflops_sustained' if dk.get('bound') == 'tensor' else ('hbm_gbs' if dk.get('bound') == 'hbm' else 'FP32 FFMA from unit counts x sm_max_mhz')})"}
 
     flops_step = f_fwd + f_bwd
-    value = world * flops_step / (ms_max * 1e-3) / 1e12
-    fwd_tflops = world * f_fwd / (ms_fwd * 1e-3) / 1e12
+    # useful FLOPs of all ranks (their shards differ slightly in size) over the slowest rank's time
+    all_flops = sum_over_ranks(float(flops_step), world)
+    all_fwd = sum_over_ranks(float(f_fwd), world)
+    value = all_flops / (ms_max * 1e-3) / 1e12
+    fwd_tflops = all_fwd / (ms_fwd * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded lognormal lengths, N(0,1) activations, N(0,0.02) rab tables)",
-        "config": {"workload": w.name, "global_batch_tokens": w.T * world, "sequences_per_gpu": w.B,
+        "config": {"workload": w.name, "global_batch_tokens": int(sum_over_ranks(float(w.T), world)),
+                   "sequences_per_gpu": w.B,
                    "max_seq_len": w.max_len, "H": H, "d": d, "mask": "causal+rab_pos+rab_time",
                    "parallelism": f"dp{world}", "l2": "inputs larger than L2 (512 MiB per tensor)"},
         "pct_bf16_peak_fwd_bwd": round(value / world / pk["bf16_tflops_sustained"], 4),
@@ -693,7 +858,7 @@ def finish(args, world, w, kernels, ms, ms_max, ms_fwd, ms_e2e, h2d, d2h, mf, cl
         "pct_bf16_peak_fwd": round(fwd_tflops / world / pk["bf16_tflops_sustained"], 4),
         "peak_source": pk_src,
         "e2e": None if ms_e2e is None else {
-            "value": round(world * flops_step / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "value": round(all_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches_total),
         "roofline": roof,
@@ -860,6 +1025,10 @@ def main():
     ap.add_argument("--no-proj", action="store_true", help="skip the f1 / f2 projections")
     ap.add_argument("--no-data", action="store_true", help="skip the Stochastic Length / packing data step")
     ap.add_argument("--no-layer", action="store_true", help="skip the whole-layer (f1, attention, f2) step")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the training-shape (Stochastic Length) and MTGR-Medium legs")
+    ap.add_argument("--only-configs", action="store_true",
+                    help="run only the training-shape and MTGR-Medium legs and print their JSON (profiling aid)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--tokens", type=int, default=262144,
@@ -883,6 +1052,12 @@ def main():
         line = run_proj(args, world, rank)
         if rank == 0:
             print(json.dumps({"projections": line}), flush=True)
+        return
+    if args.only_configs:
+        torch.cuda.set_device(local)
+        line = {"training_sl": run_training_sl(args, world, rank), "mtgr_medium": run_mtgr_medium(args, world, rank)}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
         return
     if args.only_layer:
         torch.cuda.set_device(local)

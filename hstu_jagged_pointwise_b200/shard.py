@@ -36,6 +36,12 @@ def partition_sequences(lengths: Sequence[int], world: int) -> List[List[int]]:
     return [sorted(p) for p in parts]
 
 
+def rank_sequences(lengths: Sequence[int], world: int, rank: int) -> List[int]:
+    """The sequences of a global batch that rank `rank` of `world` processes (the
+    cost-balanced partition above; every rank computes the same partition)."""
+    return partition_sequences(lengths, world)[rank]
+
+
 def shard_rows(offsets: np.ndarray, seqs: Sequence[int]):
     """(new offsets, global row indices) of the listed sequences, in order."""
     off = np.asarray(offsets, dtype=np.int64)
