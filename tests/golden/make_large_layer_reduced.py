@@ -55,7 +55,7 @@ def main():
         f.write("# from the fp64 oracle; written by make_large_layer_reduced.py.  Columns: name index exact model\n")
         for k in KEYS:
             for i, (a, b) in enumerate(zip(exact[k], storage[k])):
-                f.write(f"{k} {i} {a!r} {b!r}\n")
+                f.write(f"{k} {i} {float(a)!r} {float(b)!r}\n")
     print("wrote", OUT)
 
 
