@@ -249,7 +249,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int np = 2 * p.P - 1;
-    const long long wl = p.dbg.limit;   // main-loop wait limit (SM cycles)
     for (int i = tid; i < np; i += kThreads) s_rp[i] = p.rab_pos[i];
     for (int i = tid; i < p.nb; i += kThreads) {
         s_rt[i] = p.rab_time[i];
@@ -289,7 +288,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         while (ok) {
             const int slot = it_use & 1;
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort, wl);
+                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort, p.dbg.limit);
                 if (ok) {
                     const int idx = atomicAdd(&p.ctrl->counter, 1);
                     s_item[slot] = idx < p.ctrl->n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
@@ -307,10 +306,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (it.x < 0) break;
             if (lane == 0) {
                 const KvItem s = load_kv_item<KIND>(p, it);
-                ok = mbar_wait(&bars[kKVEmpty], (kv_use & 1) ^ 1, s_abort, wl);
+                ok = mbar_wait(&bars[kKVEmpty], (kv_use & 1) ^ 1, s_abort, p.dbg.limit);
                 if (ok && p.dbg.withhold_first_load && kv_use == 0) {
                     // test hook: withhold this CTA's first K/V tile, so the waits for it run out
-                    wait_for_abort(s_abort, 2 * wl);
+                    wait_for_abort(s_abort, 2 * p.dbg.limit);
                     ok = false;
                 }
                 if (ok) {
@@ -339,14 +338,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         t_pf++;
                     }
                     for (int hh = 0; ok && hh < 2; hh++) {
-                        ok = mbar_wait(&bars[kQEmpty0 + hh], (q_use[hh] & 1) ^ 1, s_abort, wl);
+                        ok = mbar_wait(&bars[kQEmpty0 + hh], (q_use[hh] & 1) ^ 1, s_abort, p.dbg.limit);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&bars[kQFull0 + hh], L::kHalf);
                         for (int pn = 0; pn < kPanels; pn++)
                             tma_load_2d(sm + (hh ? L::q1 : L::q0) + pn * kHalfPanel, &tm_q, &bars[kQFull0 + hh],
                                         s.h * D + pn * 64, s.off0 + t * kTileM + 64 * hh);
                         q_use[hh]++;
-                        ok = mbar_wait(&bars[kDYEmpty0 + hh], (dy_use[hh] & 1) ^ 1, s_abort, wl);
+                        ok = mbar_wait(&bars[kDYEmpty0 + hh], (dy_use[hh] & 1) ^ 1, s_abort, p.dbg.limit);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&bars[kDYFull0 + hh], L::kHalf);
                         for (int pn = 0; pn < kPanels; pn++)
@@ -387,7 +386,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t aDZ[2] = {smem_u32(sm + L::dz0), smem_u32(sm + L::dz1)};
         // S^T_h once Q_h of the tile is loaded
         auto issue_s = [&](int hh) -> bool {
-            const bool w = mbar_wait(&bars[kQFull0 + hh], q_use[hh] & 1, s_abort, wl);
+            const bool w = mbar_wait(&bars[kQFull0 + hh], q_use[hh] & 1, s_abort, p.dbg.limit);
             q_use[hh]++;
             if (!w) return false;
             tc_fence_after();
@@ -402,8 +401,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         };
         // dP^T_h once dY'_h is loaded and the previous dQ^T_h has left the columns
         auto issue_dp = [&](int hh) -> bool {
-            bool w = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort, wl);
-            if (w) w = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort, wl);
+            bool w = mbar_wait(&bars[kDYFull0 + hh], dy_use[hh] & 1, s_abort, p.dbg.limit);
+            if (w) w = mbar_wait(&bars[kDQDrained0 + hh], (dq_use[hh] & 1) ^ 1, s_abort, p.dbg.limit);
             if (!w) return false;
             dy_use[hh]++;
             tc_fence_after();
@@ -417,20 +416,22 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tc_commit(&bars[kSFull0 + hh]);
             return true;
         };
-        // dQ^T_h, dV and dK products of half hh once its elementwise step is done
+        // dK, dV and dQ^T products of half hh once its elementwise step is done.  dK goes
+        // first so that Q_h is released (and the next Q_h can load) as early as possible,
+        // then dV (releases dY'_h); dQ^T_h is drained only after the other half's step.
         auto issue_prods = [&](int hh, bool init) -> bool {
-            if (!mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort, wl)) return false;
+            if (!mbar_wait(&bars[kPFull0 + hh], p_use[hh] & 1, s_abort, p.dbg.limit)) return false;
             p_use[hh]++;
-            if (init && !mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort, wl)) return false;
+            if (init && !mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort, p.dbg.limit)) return false;
             tc_fence_after();
-            // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys); first,
-            // so that its drain overlaps the two products below
-            const uint64_t dKm = sdesc_sw128(aK, kPanel, 1024), dZm = sdesc_sw128(aDZ[hh], 16, 1024);
+            const uint64_t dZk = sdesc_sw128(aDZ[hh], 16, 1024), dQm = sdesc_sw128(aQ[hh], kHalfPanel, 1024);
+            // dK += dZ^T_h Q_h
 #pragma unroll
-            for (int kk = 0; kk < 8; kk++)
-                mma_ss(tmem + kPCol + 64 * hh, dKm + (kk * 2048 >> 4), dZm + (kk * 2048 >> 4), kIdQ, kk > 0 ? 1u : 0u);
-            dq_use[hh]++;
-            tc_commit(&bars[kDQFull0 + hh]);
+            for (int kk = 0; kk < 4; kk++) {
+                mma_ss(tmem + kKCol, dZk + (kk * 32 >> 4), dQm + (kk * 2048 >> 4), kIdK,
+                       (!init || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars[kQEmpty0 + hh]);
             const uint64_t dYm = sdesc_sw128(aDY[hh], kHalfPanel, 1024);
             // dV += A^T_h dY'_h   (A^T_h: the kEwCols queries of group c packed into columns
             // 64h + kEwCols*c .. +kEwCols/2)
@@ -441,22 +442,27 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                        kIdV, (!init || kk > 0) ? 1u : 0u);
             }
             tc_commit(&bars[kDYEmpty0 + hh]);
-            const uint64_t dZk = sdesc_sw128(aDZ[hh], 16, 1024), dQm = sdesc_sw128(aQ[hh], kHalfPanel, 1024);
-            // dK += dZ^T_h Q_h
+            // dQ^T_h = K^T dZ^T_h   (M = head dims, N = 64 queries, K = 128 keys)
+            const uint64_t dKm = sdesc_sw128(aK, kPanel, 1024), dZm = sdesc_sw128(aDZ[hh], 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) {
-                mma_ss(tmem + kKCol, dZk + (kk * 32 >> 4), dQm + (kk * 2048 >> 4), kIdK,
-                       (!init || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 8; kk++)
+                mma_ss(tmem + kPCol + 64 * hh, dKm + (kk * 2048 >> 4), dZm + (kk * 2048 >> 4), kIdQ, kk > 0 ? 1u : 0u);
+            dq_use[hh]++;
+            tc_commit(&bars[kDQFull0 + hh]);
             tc_commit(&bars[kDZEmpty0 + hh]);
-            tc_commit(&bars[kQEmpty0 + hh]);
             return true;
         };
+        // Order per visible query tile t (t' = previous tile, tn = next):
+        //   dP^T_0(t) [after dQ^T_0(t') is drained];  products of half 1 of t';  S^T_1(t);
+        //   dP^T_1(t) [after dQ^T_1(t') is drained];  products of half 0 of t;  S^T_0(tn).
+        // The elementwise warps run half 0 of t, drain dQ^T_1(t'), run half 1 of t, drain
+        // dQ^T_0(t): each drain sits between two elementwise steps, and each dP^T waits only
+        // for the drain just before it.
         while (ok) {
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
+                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, p.dbg.limit);
                 if (ok) it = s_item[slot];
             }
             ok = __shfl_sync(kFull, ok, 0);
@@ -467,32 +473,27 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (lane == 0) {
                 const KvItem s = load_kv_item<KIND>(p, it);
                 const int n_qt = (s.L + kTileM - 1) / kTileM;
-                ok = mbar_wait(&bars[kKVFull], kv_use & 1, s_abort, wl);
+                ok = mbar_wait(&bars[kKVFull], kv_use & 1, s_abort, p.dbg.limit);
                 kv_use++;
                 int t = next_visible<KIND>(s, -1, n_qt);
-                bool first = true;
-                if (ok && t < n_qt) {
-                    ok = issue_s(0);
-                    if (ok) ok = issue_dp(0);
-                    if (ok) ok = issue_s(1);
-                    if (ok) ok = issue_dp(1);
-                }
+                bool first = true, pend1 = false;
+                if (ok && t < n_qt) ok = issue_s(0);
                 while (ok && t < n_qt) {
                     const int tn = next_visible<KIND>(s, t, n_qt);
-                    ok = issue_prods(0, first);
+                    ok = issue_dp(0);
+                    if (ok && pend1) ok = issue_prods(1, false);
+                    if (ok) ok = issue_s(1);
+                    if (ok) ok = issue_dp(1);
+                    if (ok) ok = issue_prods(0, first);
                     if (ok && tn < n_qt) ok = issue_s(0);
-                    if (ok) ok = issue_prods(1, false);
-                    if (ok && tn < n_qt) {
-                        ok = issue_dp(0);
-                        if (ok) ok = issue_s(1);
-                        if (ok) ok = issue_dp(1);
-                    }
                     first = false;
+                    pend1 = true;
                     t = tn;
                 }
+                if (ok && pend1) ok = issue_prods(1, false);
                 if (ok) {
                     tc_commit(&bars[kKVEmpty]);
-                    if (first) ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort, wl);
+                    if (first) ok = mbar_wait(&bars[kAccEmpty], (acc_use & 1) ^ 1, s_abort, p.dbg.limit);
                 }
                 if (ok) {
                     acc_use++;
@@ -527,7 +528,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
-            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
+            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, p.dbg.limit);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             const int4 it = s_item[slot];
             it_use++;
@@ -552,7 +553,41 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const bool kmin_ok = (uint64_t)kmin + (1ull << 62) < (1ull << 63);
             const int n_qt = (s.L + kTileM - 1) / kTileM;
             int n_done = 0;
-            int t = next_visible<KIND>(s, -1, n_qt);
+            int t = next_visible<KIND>(s, -1, n_qt), t_prev = -1;
+            // ---- drain dQ^T_hh of query tile tq (lanes = head dims, columns = queries): one slab
+            // of C queries x kDqDims head dims (row-major) per warp, one TMA reduce-add.  M = 128
+            // puts head dim 32*wq + lane in this lane; M = 64 puts head dims 16*wq .. +15 in the
+            // first 16 lanes of the lane quarter.  Queries past the sequence end carry exact
+            // zeros (their dZ is zero).
+            auto drain = [&](int hh, int tq) -> bool {
+                const bool w = mbar_wait(&bars[kDQFull0 + hh], dq_use[hh] & 1, s_abort, p.dbg.limit);
+                if (!__all_sync(kFull, w)) return false;
+                dq_use[hh]++;
+                tc_fence_after();
+                uint32_t v[C];
+                tmem_ld(tmem + lane_base + kPCol + 64 * hh + C * g, v);
+                tmem_ld_wait(v);
+                tc_fence_before();
+                mbar_arrive(&bars[kDQDrained0 + hh]);      // the columns are free again
+                const int qi = tq * kTileM + 64 * hh + C * g;   // first query of the columns
+                if (qi < s.L) {
+                    if (lane == 0) bulk_wait_read_all();       // the previous slab has been read
+                    __syncwarp();
+                    if (D == 128 || lane < 16) {
+#pragma unroll
+                        for (int e = 0; e < C; e++) w_stg[e * kDqDims + lane] = __uint_as_float(v[e]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_2d(&tm_dq, w_stg, s.h * D + wq * kDqDims, s.off0 + qi);
+                        bulk_commit_group();
+                    }
+                }
+                return true;
+            };
+            // Per visible query tile t: half 0 of t, drain dQ^T_1 of the previous tile, half 1
+            // of t, drain dQ^T_0 of t.
             while (ok && t < n_qt) {
                 const int t_nx = next_visible<KIND>(s, t, n_qt);
                 for (int hh = 0; hh < 2; hh++) {
@@ -616,8 +651,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                     __syncwarp();
-                    ok = mbar_wait(&bars[kSFull0 + hh], s_use[hh] & 1, s_abort, wl);
-                    if (ok) ok = mbar_wait(&bars[kDZEmpty0 + hh], (dz_use[hh] & 1) ^ 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kSFull0 + hh], s_use[hh] & 1, s_abort, p.dbg.limit);
+                    if (ok) ok = mbar_wait(&bars[kDZEmpty0 + hh], (dz_use[hh] & 1) ^ 1, s_abort, p.dbg.limit);
                     if (!__all_sync(kFull, ok)) { ok = false; break; }
                     s_use[hh]++;
                     dz_use[hh]++;
@@ -714,45 +749,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     fence_proxy_async_smem();
                     tc_fence_before();
                     mbar_arrive(&bars[kPFull0 + hh]);
+                    // dQ^T of the other half: half 1 of the previous tile, or half 0 of this one
+                    const int dt = hh == 0 ? t_prev : t;
+                    if (dt >= 0 && !drain(1 - hh, dt)) { ok = false; break; }
                 }
                 if (!ok) break;
-                // ---- drain dQ^T of both halves (lanes = head dims, columns = queries): one
-                // slab of C queries x kDqDims head dims (row-major) per warp, one TMA reduce-add.
-                // M = 128 puts head dim 32*wq + lane in this lane; M = 64 puts head dims
-                // 16*wq .. +15 in the first 16 lanes of the lane quarter.  Queries past the
-                // sequence end carry exact zeros (their dZ is zero).
-                for (int hh = 0; hh < 2; hh++) {
-                    ok = mbar_wait(&bars[kDQFull0 + hh], dq_use[hh] & 1, s_abort, wl);
-                    if (!__all_sync(kFull, ok)) { ok = false; break; }
-                    dq_use[hh]++;
-                    tc_fence_after();
-                    uint32_t v[C];
-                    tmem_ld(tmem + lane_base + kPCol + 64 * hh + C * g, v);
-                    tmem_ld_wait(v);
-                    tc_fence_before();
-                    mbar_arrive(&bars[kDQDrained0 + hh]);      // the columns are free again
-                    const int qi = t * kTileM + 64 * hh + C * g;   // first query of the columns
-                    if (qi < s.L) {
-                        if (lane == 0) bulk_wait_read_all();       // the previous slab has been read
-                        __syncwarp();
-                        if (D == 128 || lane < 16) {
-#pragma unroll
-                            for (int e = 0; e < C; e++) w_stg[e * kDqDims + lane] = __uint_as_float(v[e]);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_reduce_add_2d(&tm_dq, w_stg, s.h * D + wq * kDqDims, s.off0 + qi);
-                            bulk_commit_group();
-                        }
-                    }
-                }
                 n_done++;
+                t_prev = t;
                 t = t_nx;
             }
+            if (ok && t_prev >= 0) ok = drain(1, t_prev);   // the last tile's dQ^T_1
             if (!ok) break;
             // ---------------- epilogue: dV, dK rows of this key tile (D / kEwGroups columns per warp)
-            ok = mbar_wait(&bars[kAccFull], acc_use & 1, s_abort, wl);
+            ok = mbar_wait(&bars[kAccFull], acc_use & 1, s_abort, p.dbg.limit);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             acc_use++;
             tc_fence_after();

@@ -47,6 +47,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, but a thread whose phase has not completed is suspended until it
+// completes or about `ns` nanoseconds pass (the PTX suspend-time hint), so that a waiting
+// warp issues nothing meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspend-time hint of the bounded waits: long enough that a waiting warp stays parked
+// (a spinning warp would take issue and shared-memory slots from the warps it waits
+// for), short enough that an abort or the limit is noticed within microseconds.
+constexpr uint32_t kWaitSleepNs = 20000;
+
 // Waits for the phase with the given parity to complete.  Returns false when
 // the wait runs past `limit` SM cycles or *abort becomes non-zero.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -54,7 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
         if (*abort) return false;
         if (clock64() - t0 > limit) return false;
     }
@@ -318,6 +338,17 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
                  "f"(d)
                  : "memory");
+}
+
+// fp32 add to shared memory (no return value), and the same add issued only where p holds.
+__device__ __forceinline__ void red_add_smem(float* addr, float v) {
+    asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(addr)), "f"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_smem_if(bool p, float* addr, float v) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %2, 0;\n@q red.shared.add.f32 [%0], %1;\n}" ::"r"(smem_u32(addr)),
+        "f"(v), "r"((int)p)
+        : "memory");
 }
 
 // ---------------------------------------------------------------- math
