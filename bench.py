@@ -394,7 +394,8 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the C ABI with host buffers
     if args.no_e2e:
-        return finish(args, world, w, kernels, ms, ms_max, ms_fwd, None, None, None, None, clocks, f_fwd, f_bwd, P, d,
+        mf = None if args.no_mfalcon else run_mfalcon(args, world, rank, local)
+        return finish(args, world, w, kernels, ms, ms_max, ms_fwd, None, None, None, mf, clocks, f_fwd, f_bwd, P, d,
                       extra)
     # Pipelined over three streams: the host->device copies of step k+1 and the
     # device->host copies of step k-1 run while step k computes (PCIe carries both
@@ -1037,6 +1038,9 @@ def main():
                     help="run only the f1 / f2 projections leg and print its JSON (profiling aid)")
     ap.add_argument("--only-layer", action="store_true",
                     help="run only the whole-layer leg and print its JSON (profiling aid)")
+    ap.add_argument("--only-mfalcon", action="store_true",
+                    help="run only the M-FALCON legs (cached scorer, one-row forward, KV-cache producer) "
+                         "and print their JSON (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -1058,6 +1062,12 @@ def main():
         line = {"training_sl": run_training_sl(args, world, rank), "mtgr_medium": run_mtgr_medium(args, world, rank)}
         if rank == 0:
             print(json.dumps(line), flush=True)
+        return
+    if args.only_mfalcon:
+        torch.cuda.set_device(local)
+        line = run_mfalcon(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps({"mfalcon": line}), flush=True)
         return
     if args.only_layer:
         torch.cuda.set_device(local)

@@ -173,7 +173,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::abort_flag);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long wl = p.dbg.limit;   // main-loop wait limit (SM cycles)
 
     for (int i = tid; i < 2 * p.P - 1; i += kThreads) s_rp[i] = p.rab_pos[i];
     for (int i = tid; i < p.nb; i += kThreads) {
@@ -220,7 +219,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         while (ok) {
             const int slot = it_use & 1;
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort, wl);
+                ok = mbar_wait(&bars[kItEmpty0 + slot], ((it_use >> 1) & 1) ^ 1, s_abort, p.dbg.limit);
                 if (ok) {
                     const int idx = atomicAdd(&p.ctrl->counter, 1);
                     const int4 it = idx < p.ctrl->n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
@@ -239,10 +238,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (it.x < 0) break;
             const Item s = load_item<KIND>(p, it);
             if (lane == 0) {
-                ok = mbar_wait(&bars[kQEmpty], (q_use & 1) ^ 1, s_abort, wl);
+                ok = mbar_wait(&bars[kQEmpty], (q_use & 1) ^ 1, s_abort, p.dbg.limit);
                 if (ok && p.dbg.withhold_first_load && q_use == 0) {
                     // test hook: withhold this CTA's first Q tile, so the waits for it run out
-                    wait_for_abort(s_abort, 2 * wl);
+                    wait_for_abort(s_abort, 2 * p.dbg.limit);
                     ok = false;
                 }
                 if (ok) {
@@ -266,13 +265,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         t_pf++;
                     }
                     const int y = s.kv0 + t * kTileN;
-                    ok = mbar_wait(&bars[kKEmpty], (k_use & 1) ^ 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kKEmpty], (k_use & 1) ^ 1, s_abort, p.dbg.limit);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bars[kKFull], L::kTileBytes);
                     for (int pn = 0; pn < kPanels; pn++)
                         tma_load_2d(sK + pn * kPanelBytes, &tm_k, &bars[kKFull], s.h * D + pn * 64, y);
                     k_use++;
-                    ok = mbar_wait(&bars[kVEmpty], (v_use & 1) ^ 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kVEmpty], (v_use & 1) ^ 1, s_abort, p.dbg.limit);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bars[kVFull], L::kTileBytes);
                     for (int pn = 0; pn < kPanels; pn++)
@@ -304,7 +303,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int slot = it_use & 1;
             int4 it = make_int4(-1, 0, 0, 0);
             if (lane == 0) {
-                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
+                ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, p.dbg.limit);
                 if (ok) it = s_item[slot];
             }
             ok = __shfl_sync(kFull, ok, 0);
@@ -318,13 +317,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 int last = -1;
                 for (int t = 0; t < n_kt; t++)
                     if (kv_class<KIND>(s, t) != 0) last = t;
-                ok = mbar_wait(&bars[kQFull], q_use & 1, s_abort, wl);
+                ok = mbar_wait(&bars[kQFull], q_use & 1, s_abort, p.dbg.limit);
                 q_use++;
                 tc_fence_after();
                 int n_done = 0;
                 for (int t = 0; ok && t <= last; t++) {
                     if (kv_class<KIND>(s, t) == 0) continue;
-                    ok = mbar_wait(&bars[kKFull], k_use & 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kKFull], k_use & 1, s_abort, p.dbg.limit);
                     if (!ok) break;
                     k_use++;
                     tc_fence_after();
@@ -336,14 +335,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tc_commit(&bars[kSFull]);
                     tc_commit(&bars[kKEmpty]);
                     if (t == last) tc_commit(&bars[kQEmpty]);
-                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kPFull], p_use & 1, s_abort, p.dbg.limit);
                     if (!ok) break;
                     p_use++;
-                    ok = mbar_wait(&bars[kVFull], v_use & 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kVFull], v_use & 1, s_abort, p.dbg.limit);
                     if (!ok) break;
                     v_use++;
                     if (n_done == 0) {
-                        ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort, wl);
+                        ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort, p.dbg.limit);
                         if (!ok) break;
                     }
                     tc_fence_after();
@@ -359,7 +358,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (ok && n_done == 0) {
                     tc_commit(&bars[kQEmpty]);
-                    ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort, wl);
+                    ok = mbar_wait(&bars[kOEmpty], (o_use & 1) ^ 1, s_abort, p.dbg.limit);
                 }
                 if (ok) {
                     o_use++;
@@ -392,7 +391,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         while (ok) {
             const int slot = it_use & 1;
-            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, wl);
+            ok = mbar_wait(&bars[kItFull0 + slot], (it_use >> 1) & 1, s_abort, p.dbg.limit);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             const int4 it = s_item[slot];
             it_use++;
@@ -564,7 +563,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 __syncwarp();
                 const int32_t a_i = (int32_t)(uint32_t)((uint64_t)ts_i - (uint64_t)cmin);
-                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort, wl);
+                ok = mbar_wait(&bars[kSFull], s_use & 1, s_abort, p.dbg.limit);
                 if (!__all_sync(kFull, ok)) { ok = false; break; }
                 s_use++;
                 tc_fence_after();
@@ -579,6 +578,34 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_st16(tmem + lane_base + kSCol + 32 * c, pk);
                         continue;
                     }
+                    if (pm < 0) {
+                        // element by element (MTGR candidates, ragged key tiles, int64-wide time
+                        // spans): a compact loop over key pairs that reads S and writes P in TMEM
+                        // pair by pair, so that this rare path adds little code
+                        const uint32_t col = tmem + lane_base + kSCol + 32 * c;
+#pragma unroll 1
+                        for (int e = 0; e < 32; e += 2) {
+                            uint32_t s0, s1;
+                            tmem_ld2(col + e, s0, s1);
+                            float pv[2];
+#pragma unroll
+                            for (int f = 0; f < 2; f++) {
+                                const int jj = 32 * cc + e + f;
+                                const int j = n0 + jj;
+                                const int64_t ts_j = w_cts[jj];
+                                bool vis = row_ok && j < s.Lk;
+                                if (KIND != HSTU_KIND_MFALCON)
+                                    vis = vis && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
+                                const int pidx = pos_index(pos_i, col_pos<KIND>(s, j), p.P);
+                                const int tb = time_bucket(ts_i, ts_j, p.nb);
+                                const float h = fmaf(__uint_as_float(f ? s1 : s0), 0.5f, 0.5f * s_rp[pidx] + s_rth[tb]);
+                                pv[f] = vis ? fmaf(h, tanh_approx(h), h) : 0.f;
+                            }
+                            // P pair e/2 into column e/2 of the chunk: its S values were read already
+                            tmem_st1(col + (e >> 1), pack_bf16x2(pv[0], pv[1]));
+                        }
+                        continue;
+                    }
                     uint32_t v[32];
                     tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
                     tmem_ld_wait(v);
@@ -588,32 +615,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     else if (pm >= 0 && tm == kTimeUniform) fwd_block<kBiasRow>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else if (pm >= 0 && tm == kTimeTwo)
                         fwd_block<kBiasRowTwo>(v, dg, cr, a_i, c0, s_rth, nbm1, pk, tc.thr, s_rth[tc.tb_lo], s_rth[tc.tb_hi]);
-                    else if (pm >= 0 && tm >= 0) fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
-                    if (pm >= 0 && jlim - 32 * cc < 32) {
+                    else fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                    if ((KIND == HSTU_KIND_MTGR || KIND == HSTU_KIND_MFSEQ) && pm >= 0 && jlim - 32 * cc < 32) {
                         // keys past the block's column limit: P = 0 (bf16 pairs, key 2e in the low half)
                         const int lim = jlim - 32 * cc;
 #pragma unroll
                         for (int e = 0; e < 16; e++)
                             pk[e] &= 2 * e + 1 < lim ? 0xffffffffu : (2 * e < lim ? 0x0000ffffu : 0u);
-                    }
-                    if (pm < 0) {
-                        // element by element: MTGR candidates, ragged key tiles, int64-wide time spans
-                        float pv[32];
-#pragma unroll
-                        for (int e = 0; e < 32; e++) {
-                            const int jj = 32 * cc + e;
-                            const int j = n0 + jj;
-                            const int64_t ts_j = w_cts[jj];
-                            bool vis = row_ok && j < s.Lk;
-                            if (KIND != HSTU_KIND_MFALCON)
-                                vis = vis && visible(KIND, i, j, s.S, s.R, ts_i, ts_j);
-                            const int pidx = pos_index(pos_i, col_pos<KIND>(s, j), p.P);
-                            const int tb = time_bucket(ts_i, ts_j, p.nb);
-                            const float h = fmaf(__uint_as_float(v[e]), 0.5f, 0.5f * s_rp[pidx] + s_rth[tb]);
-                            pv[e] = vis ? fmaf(h, tanh_approx(h), h) : 0.f;
-                        }
-#pragma unroll
-                        for (int e = 0; e < 16; e++) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
                     }
                     // P (bf16 pairs) into the chunk's own, already read, S columns: two warps
                     // share these TMEM lanes and each may only overwrite what it has read
@@ -648,7 +656,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 a_self = silu_fast(dot + rp_self + rt_zero);
                 vself = p.self_v + ro;
             }
-            ok = mbar_wait(&bars[kOFull], o_use & 1, s_abort, wl);
+            ok = mbar_wait(&bars[kOFull], o_use & 1, s_abort, p.dbg.limit);
             if (!__all_sync(kFull, ok)) { ok = false; break; }
             o_use++;
             tc_fence_after();

@@ -47,26 +47,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// The same test, but a thread whose phase has not completed is suspended until it
-// completes or about `ns` nanoseconds pass (the PTX suspend-time hint), so that a waiting
-// warp issues nothing meanwhile.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-
-// Suspend-time hint of the bounded waits: long enough that a waiting warp stays parked
-// (a spinning warp would take issue and shared-memory slots from the warps it waits
-// for), short enough that an abort or the limit is noticed within microseconds.
-constexpr uint32_t kWaitSleepNs = 20000;
-
 // Waits for the phase with the given parity to complete.  Returns false when
 // the wait runs past `limit` SM cycles or *abort becomes non-zero.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -74,7 +54,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (clock64() - t0 > limit) return false;
     }
@@ -283,6 +263,17 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
 // Loads of 16 or 32 columns by array size.
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32(taddr, r); }
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16(taddr, r); }
+
+// 32 lanes x 2 consecutive 32-bit columns (runtime column address, small code)
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t& a, uint32_t& b) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(a), "+r"(b) : : "memory");
+}
+
+// 32 lanes x 1 32-bit column
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t a) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
+}
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
