@@ -27,8 +27,11 @@
 //   dz = dP' * 2 SiLU'(z) with dP' = V dY'^T,   dV = 2 A_raw^T dY' (the 2 in the epilogue).
 // dQ^T leaves TMEM through registers and a per-warp shared-memory slab; a TMA
 // tensor reduce-add sends each slab to the fp32 accumulation buffer.
-// Warps 0-7 elementwise (warp w owns TMEM lanes 32*(w%4)..+31 and 32 of the
-// half's 64 columns, [32*(w/4), +32)), warp 8 producer (TMA), warp 9 MMA issuer.
+// Warps 0-15 elementwise (warp w owns TMEM lanes 32*(w%4)..+31 and 16 of the
+// half's 64 columns, [16*(w/4), +16)), warp 16 producer (TMA), warp 17 MMA issuer.
+// Per visible query tile the elementwise warps run half 0, drain dQ^T_1 of the
+// previous tile, run half 1, then drain dQ^T_0 of this tile, so that each drain
+// overlaps the tensor core's work on the other half.
 // rab gradients: register sums per warp block (uniform bias), per-diagonal sums
 // gathered with warp shuffles (position), run-length sums per thread (time),
 // sent with fire-and-forget global reductions into this CTA's own partial row;
@@ -119,6 +122,8 @@ __device__ __forceinline__ int q_class(const KvItem& s, int t) {
 // first query tile after t that sees the item's keys, n_qt when none
 template <int KIND>
 __device__ __forceinline__ int next_visible(const KvItem& s, int t, int n_qt) {
+    // causal: once a query tile sees the key tile, every later one does
+    if (KIND == HSTU_KIND_CAUSAL && t >= 0) return t + 1 < n_qt ? t + 1 : n_qt;
     for (t++; t < n_qt; t++)
         if (q_class<KIND>(s, t) != 0) break;
     return t;
@@ -371,12 +376,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        // Order per tile t (next visible tile tn):
-        //   [p_full 0] products of half 0 of t;  [Q_0 of tn] S^T_0 of tn;
-        //   [p_full 1] products of half 1 of t;  dP^T_0 of tn;  [Q_1 of tn] S^T_1, dP^T_1 of tn.
-        // Q_h is released after the dK product of half h.
-        // The next tile's scores are then in flight while the elementwise warps
-        // drain dQ and set up, instead of after them.
+        // Issue order (below, above the item loop) keeps the next half's scores in flight
+        // while the elementwise warps work on the current one.  Q_h is released after the
+        // dK product of half h, dY'_h after the dV product.
         int it_use = 0, kv_use = 0, acc_use = 0;
         int q_use[2] = {0, 0}, dy_use[2] = {0, 0}, p_use[2] = {0, 0}, dq_use[2] = {0, 0};
         bool ok = true;
@@ -729,7 +731,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         const uint32_t ch = (uint32_t)(((C / 8) * g + e) ^ (r & 7));
                         st_shared_v4(row_addr + ch * 16, pz[4 * e], pz[4 * e + 1], pz[4 * e + 2], pz[4 * e + 3]);
                     }
-                    // ---- rab gradients of the block
+                    tmem_st_wait();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(&bars[kPFull0 + hh]);
+                    // dQ^T of the other half: half 1 of the previous tile, or half 0 of this one
+                    const int dt = hh == 0 ? t_prev : t;
+                    if (dt >= 0 && !drain(1 - hh, dt)) { ok = false; break; }
+                    // ---- rab gradients of the block, sent once the MMA warp and the other half's
+                    // dP^T are unblocked
                     if (pm == kPosUniform || tm == kTimeUniform) {
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
@@ -745,13 +755,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         if (lane > 32 - C && dhi != 0.f)
                             red_add_f32(&g_rp[min(max(dmin + lane + C - 33, -np1), np1) + np1], dhi);
                     }
-                    tmem_st_wait();
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(&bars[kPFull0 + hh]);
-                    // dQ^T of the other half: half 1 of the previous tile, or half 0 of this one
-                    const int dt = hh == 0 ? t_prev : t;
-                    if (dt >= 0 && !drain(1 - hh, dt)) { ok = false; break; }
                 }
                 if (!ok) break;
                 n_done++;
