@@ -258,19 +258,27 @@ def oracle_sample(w, target_s: float = 12.0):
     import oracle
     L = w.lengths
     order = np.argsort(L)
-    # calibrate on the shortest sequence
-    cal = sub_workload(w, [int(order[0])])
-    t0 = time.perf_counter()
-    oracle.layer_bwd(cal)
-    dt = max(time.perf_counter() - t0, 1e-3)
-    rate = 12 * w.d * w.H * causal_pairs([L[order[0]]]) / dt
-    seqs, flops = [], 0.0
-    for b in order[1:]:
-        f = 12 * w.d * w.H * causal_pairs([L[b]])
-        if seqs and (flops + f) / rate > target_s:
-            break
-        seqs.append(int(b))
-        flops += f
+    def pick(rate, budget_s):
+        seqs, flops = [], 0.0
+        for b in order:
+            f = 12 * w.d * w.H * causal_pairs([L[b]])
+            if seqs and (flops + f) / rate > budget_s:
+                break
+            seqs.append(int(b))
+            flops += f
+        return seqs, flops
+
+    def measure(seqs, flops):
+        t0 = time.perf_counter()
+        oracle.layer_bwd(sub_workload(w, seqs))
+        return flops / max(time.perf_counter() - t0, 1e-3)
+
+    # calibrate on the shortest sequence, then on about one and three seconds of work (short
+    # sequences alone under-use the host threads, which would make the sample too small)
+    rate = measure([int(order[0])], 12 * w.d * w.H * causal_pairs([L[order[0]]]))
+    rate = measure(*pick(rate, 1.0))
+    rate = measure(*pick(rate, 3.0))
+    seqs, _ = pick(rate, target_s)
     return sub_workload(w, seqs), seqs
 
 
