@@ -114,10 +114,34 @@ __device__ __forceinline__ void flag_timeout(const FwdParams& p, volatile int* a
 // the instruction cache.
 enum { kBiasConst = 0, kBiasRow = 1, kBiasRowTime = 2, kBiasRowTwo = 3 };
 
+// Half of a block: keys E0 .. E0+15 of the chunk, S values in v.
+template <int BM, int E0>
+__device__ __forceinline__ void fwd_half(const uint32_t (&v)[16], const float* dg, const int32_t (&b)[32], int32_t a_i,
+                                         float c0, const float* rth, int nbm1, uint32_t (&pk)[16],
+                                         uint32_t thr, float t_lo, float t_hi) {
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+        float hb[2];
+#pragma unroll
+        for (int f = 0; f < 2; f++) {
+            const int k = E0 + e + f;
+            hb[f] = BM == kBiasConst ? c0 : dg[k];
+            if (BM == kBiasRowTime) hb[f] += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
+            if (BM == kBiasRowTwo) hb[f] += (uint32_t)abs(b[k] - a_i) >= thr ? t_hi : t_lo;
+        }
+        const float2 h = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), make_float2(0.5f, 0.5f),
+                              make_float2(hb[0], hb[1]));
+        const float2 a = fma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
+        pk[(E0 + e) >> 1] = pack_bf16x2(a.x, a.y);
+    }
+}
+
+// The chunk's S is read from TMEM in two 16-column halves: the second half's load is in
+// flight while the first half is computed.
 template <int BM>
-__device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* dg, const int32_t* cr, int32_t a_i,
-                                          float c0, const float* rth, int nbm1, uint32_t (&pk)[16],
-                                          uint32_t thr = 0, float t_lo = 0.f, float t_hi = 0.f) {
+__device__ __forceinline__ void fwd_block2(uint32_t taddr, const float* dg, const int32_t* cr, int32_t a_i, float c0,
+                                           const float* rth, int nbm1, uint32_t (&pk)[16], uint32_t thr = 0,
+                                           float t_lo = 0.f, float t_hi = 0.f) {
     int32_t b[32];
     if (BM == kBiasRowTime || BM == kBiasRowTwo) {
         const int4* b4 = reinterpret_cast<const int4*>(cr);
@@ -127,22 +151,13 @@ __device__ __forceinline__ void fwd_block(const uint32_t (&v)[32], const float* 
             b[4 * e] = x.x; b[4 * e + 1] = x.y; b[4 * e + 2] = x.z; b[4 * e + 3] = x.w;
         }
     }
-    // key pairs through packed fp32 arithmetic: h = z / 2, SiLU(z) = h + h tanh(h)
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        float hb[2];
-#pragma unroll
-        for (int f = 0; f < 2; f++) {
-            const int k = e + f;
-            hb[f] = BM == kBiasConst ? c0 : dg[k];
-            if (BM == kBiasRowTime) hb[f] += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
-            if (BM == kBiasRowTwo) hb[f] += (uint32_t)abs(b[k] - a_i) >= thr ? t_hi : t_lo;
-        }
-        const float2 h = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), make_float2(0.5f, 0.5f),
-                              make_float2(hb[0], hb[1]));
-        const float2 a = fma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
-        pk[e >> 1] = pack_bf16x2(a.x, a.y);
-    }
+    uint32_t va[16], vb[16];
+    tmem_ld16(taddr, va);
+    tmem_ld_wait(va);
+    tmem_ld16(taddr + 16, vb);
+    fwd_half<BM, 0>(va, dg, b, a_i, c0, rth, nbm1, pk, thr, t_lo, t_hi);
+    tmem_ld_wait(vb);
+    fwd_half<BM, 16>(vb, dg, b, a_i, c0, rth, nbm1, pk, thr, t_lo, t_hi);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -606,16 +621,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                         continue;
                     }
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + kSCol + 32 * c, v);
-                    tmem_ld_wait(v);
+                    const uint32_t sa = tmem + lane_base + kSCol + 32 * c;
                     const float* dg = w_diag + 31 - (KIND != HSTU_KIND_CAUSAL && pm == kPosCol ? 0 : lane) + 32 * cc;
                     const int32_t* cr = w_crel + 32 * cc;
-                    if (pm == kPosUniform && tm == kTimeUniform) fwd_block<kBiasConst>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
-                    else if (pm >= 0 && tm == kTimeUniform) fwd_block<kBiasRow>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                    if (pm == kPosUniform && tm == kTimeUniform) fwd_block2<kBiasConst>(sa, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                    else if (pm >= 0 && tm == kTimeUniform) fwd_block2<kBiasRow>(sa, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     else if (pm >= 0 && tm == kTimeTwo)
-                        fwd_block<kBiasRowTwo>(v, dg, cr, a_i, c0, s_rth, nbm1, pk, tc.thr, s_rth[tc.tb_lo], s_rth[tc.tb_hi]);
-                    else fwd_block<kBiasRowTime>(v, dg, cr, a_i, c0, s_rth, nbm1, pk);
+                        fwd_block2<kBiasRowTwo>(sa, dg, cr, a_i, c0, s_rth, nbm1, pk, tc.thr, s_rth[tc.tb_lo], s_rth[tc.tb_hi]);
+                    else fwd_block2<kBiasRowTime>(sa, dg, cr, a_i, c0, s_rth, nbm1, pk);
                     if ((KIND == HSTU_KIND_MTGR || KIND == HSTU_KIND_MFSEQ) && pm >= 0 && jlim - 32 * cc < 32) {
                         // keys past the block's column limit: P = 0 (bf16 pairs, key 2e in the low half)
                         const int lim = jlim - 32 * cc;
