@@ -116,7 +116,7 @@ enum { kBiasConst = 0, kBiasRow = 1, kBiasRowTime = 2, kBiasRowTwo = 3 };
 
 // Half of a block: keys E0 .. E0+15 of the chunk, S values in v.
 template <int BM, int E0>
-__device__ __forceinline__ void fwd_half(const uint32_t (&v)[16], const float* dg, const int32_t (&b)[32], int32_t a_i,
+__device__ __forceinline__ void fwd_half(const uint32_t (&v)[16], const float* dg, const int32_t (&b)[16], int32_t a_i,
                                          float c0, const float* rth, int nbm1, uint32_t (&pk)[16],
                                          uint32_t thr, float t_lo, float t_hi) {
 #pragma unroll
@@ -126,8 +126,8 @@ __device__ __forceinline__ void fwd_half(const uint32_t (&v)[16], const float* d
         for (int f = 0; f < 2; f++) {
             const int k = E0 + e + f;
             hb[f] = BM == kBiasConst ? c0 : dg[k];
-            if (BM == kBiasRowTime) hb[f] += rth[time_bucket_u32((uint32_t)abs(b[k] - a_i), nbm1)];
-            if (BM == kBiasRowTwo) hb[f] += (uint32_t)abs(b[k] - a_i) >= thr ? t_hi : t_lo;
+            if (BM == kBiasRowTime) hb[f] += rth[time_bucket_u32((uint32_t)abs(b[k - E0] - a_i), nbm1)];
+            if (BM == kBiasRowTwo) hb[f] += (uint32_t)abs(b[k - E0] - a_i) >= thr ? t_hi : t_lo;
         }
         const float2 h = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), make_float2(0.5f, 0.5f),
                               make_float2(hb[0], hb[1]));
@@ -142,20 +142,24 @@ template <int BM>
 __device__ __forceinline__ void fwd_block2(uint32_t taddr, const float* dg, const int32_t* cr, int32_t a_i, float c0,
                                            const float* rth, int nbm1, uint32_t (&pk)[16], uint32_t thr = 0,
                                            float t_lo = 0.f, float t_hi = 0.f) {
-    int32_t b[32];
-    if (BM == kBiasRowTime || BM == kBiasRowTwo) {
-        const int4* b4 = reinterpret_cast<const int4*>(cr);
+    int32_t b[16];
+    auto load_b = [&](int h) {
+        if (BM == kBiasRowTime || BM == kBiasRowTwo) {
+            const int4* b4 = reinterpret_cast<const int4*>(cr + 16 * h);
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
-            const int4 x = b4[e];
-            b[4 * e] = x.x; b[4 * e + 1] = x.y; b[4 * e + 2] = x.z; b[4 * e + 3] = x.w;
+            for (int e = 0; e < 4; e++) {
+                const int4 x = b4[e];
+                b[4 * e] = x.x; b[4 * e + 1] = x.y; b[4 * e + 2] = x.z; b[4 * e + 3] = x.w;
+            }
         }
-    }
+    };
     uint32_t va[16], vb[16];
     tmem_ld16(taddr, va);
+    load_b(0);
     tmem_ld_wait(va);
     tmem_ld16(taddr + 16, vb);
     fwd_half<BM, 0>(va, dg, b, a_i, c0, rth, nbm1, pk, thr, t_lo, t_hi);
+    load_b(1);
     tmem_ld_wait(vb);
     fwd_half<BM, 16>(vb, dg, b, a_i, c0, rth, nbm1, pk, thr, t_lo, t_hi);
 }
