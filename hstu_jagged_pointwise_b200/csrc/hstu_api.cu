@@ -483,6 +483,18 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     if (!aligned(d_rab_pos, 4) || !aligned(d_rab_time, 4) ||
         (!from_dy && (!aligned(d_gamma, 4) || !aligned(d_beta, 4))))
         return HSTU_ERR_INVALID_ARG;
+    // every argument is checked before the first CUDA call
+    if (d.T > 0) {
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+            !aligned(dv, 16) || !aligned(seq_offsets, 4) || !aligned(timestamps, 8) || !aligned(rab_pos, 4) ||
+            !aligned(rab_time, 4))
+            return HSTU_ERR_INVALID_ARG;
+        if (from_dy ? !aligned(dy_in, 16)
+                    : (!aligned(u, 16) || !aligned(y, 16) || !aligned(d_o_pre, 16) || !aligned(du, 16) ||
+                       !aligned(ln_gamma, 16) || !aligned(ln_beta, 16) || !aligned(ln_mean, 4) ||
+                       !aligned(ln_rstd, 4)))
+            return HSTU_ERR_INVALID_ARG;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int D = d.H * d.d_v;
     cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * d.n_pos - 1), s);
@@ -493,15 +505,6 @@ int attn_bwd_impl(const hstu_dims* dims, const hstu_mask_spec* mask, const hstu_
     }
     if (e != cudaSuccess) return cuda_status(e);
     if (d.T == 0) return HSTU_OK;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
-        !aligned(dv, 16) || !aligned(seq_offsets, 4) || !aligned(timestamps, 8) || !aligned(rab_pos, 4) ||
-        !aligned(rab_time, 4))
-        return HSTU_ERR_INVALID_ARG;
-    if (from_dy ? !aligned(dy_in, 16)
-                : (!aligned(u, 16) || !aligned(y, 16) || !aligned(d_o_pre, 16) || !aligned(du, 16) ||
-                   !aligned(ln_gamma, 16) || !aligned(ln_beta, 16) || !aligned(ln_mean, 4) ||
-                   !aligned(ln_rstd, 4)))
-        return HSTU_ERR_INVALID_ARG;
     Control* ctrl = at<Control>(workspace, 0);
 
     // 1. validation + work list of (sequence, head, key tile)

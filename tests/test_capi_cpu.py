@@ -93,6 +93,35 @@ def test_fwd_rejects_bad_arguments_before_launch():
     assert capi.LIB.hstu_attn_fwd(C.byref(d0), C.byref(m), *args, 2048, None) == capi.HSTU_OK
 
 
+def test_bwd_rejects_bad_arguments_before_any_cuda_call():
+    """hstu_attn_bwd and hstu_attn_bwd_dy check every argument before their first CUDA call,
+    so on a machine without a GPU each bad call returns its own status, not a CUDA error."""
+    d = dims()
+    m = capi.HstuMaskSpec(kind=0, n_static=None, n_realtime=None)
+    nulls23, nulls14 = [None] * 23, [None] * 14
+    assert capi.LIB.hstu_attn_bwd(None, C.byref(m), *nulls23, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), None, *nulls23, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    assert capi.LIB.hstu_attn_bwd_dy(None, C.byref(m), *nulls14, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    d2 = dims(d_qk=48, d_v=48)
+    assert capi.LIB.hstu_attn_bwd(C.byref(d2), C.byref(m), *nulls23, 0, None) == capi.HSTU_ERR_UNSUPPORTED
+    m2 = capi.HstuMaskSpec(kind=1, n_static=None, n_realtime=None)
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), C.byref(m2), *nulls23, 0, None) == capi.HSTU_ERR_INVALID_ARG
+    # missing or small workspace
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), C.byref(m), *nulls23, 0, None) == capi.HSTU_ERR_WORKSPACE
+    need = capi.LIB.hstu_attn_workspace_bytes(C.byref(d), 0, 1)
+    ws = (C.c_uint8 * (need + 256))()
+    wsa = C.c_void_p((C.addressof(ws) + 255) // 256 * 256)
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), C.byref(m), *nulls23[:22], wsa, need - 256, None) == capi.HSTU_ERR_WORKSPACE
+    # enough workspace: missing gradient outputs, then missing inputs (T > 0)
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), C.byref(m), *nulls23[:22], wsa, need, None) == capi.HSTU_ERR_INVALID_ARG
+    grads = (C.c_float * 1024)()
+    g = C.c_void_p((C.addressof(grads) + 15) // 16 * 16)
+    args = [None] * 18 + [g, g, g, g] + [wsa]
+    assert capi.LIB.hstu_attn_bwd(C.byref(d), C.byref(m), *args, need, None) == capi.HSTU_ERR_INVALID_ARG
+    args_dy = [None] * 11 + [g, g] + [wsa]
+    assert capi.LIB.hstu_attn_bwd_dy(C.byref(d), C.byref(m), *args_dy, need, None) == capi.HSTU_ERR_INVALID_ARG
+
+
 def test_full_sequence_mfalcon_mask_is_forward_only():
     """The [history ; candidates] mask has a forward workspace, no backward, and needs n_realtime."""
     d = dims()
